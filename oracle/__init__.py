@@ -1,0 +1,171 @@
+"""CPU oracle for the INT8-quantised attention forward pass.
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference leg import this package.  The product
+path (the CUDA library and its Python binding) never imports or calls it.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64 for the softmax and the
+value path, IEEE fp32 for the quantiser); this module only builds it with gcc
+and marshals numpy arrays.  Each function cites the passage it follows:
+
+* ``quantize_per_token`` / ``quantize_per_tensor`` -- IntAttention (A Fully
+  Integer Attention Pipeline for Efficient Edge Inference), section 2.1,
+  eq. 3; per-token granularity from INT-FlashAttention (Enabling Flash
+  Attention for INT8 Quantization), abstract.
+* ``qk_int32`` -- IntAttention section 2.1, eq. 4 (INT8 x INT8 -> INT32).
+* ``attention_rows`` -- IntAttention eqs. 4-6 and section 3.2 (P x 127 as
+  INT8), eq. 5 for the value path.
+* ``attention_fp64_rows`` -- IntAttention section 2.1, eq. 1.
+
+All functions are pinned by ``tests/test_oracle_*.py`` (closed forms,
+invariants, brute force on tiny inputs).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into oracle/liboracle.so with plain gcc (no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", _LIB_PATH, "-lm"]
+        subprocess.check_call(cmd)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    lib.oracle_set_threads.argtypes = [ctypes.c_int]
+    lib.oracle_get_threads.restype = ctypes.c_int
+    lib.oracle_quantize_per_token.argtypes = [P, I64, I64, P, P]
+    lib.oracle_quantize_per_tensor.argtypes = [P, I64, I64, P, P]
+    lib.oracle_qk_int32.argtypes = [P, P, I64, I64, I64, P]
+    lib.oracle_attention_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
+                                          ctypes.c_int, I64, I64, P, P, P, P]
+    lib.oracle_attention_fp64_rows.argtypes = [P, P, P, I64, I64, ctypes.c_int, I64, I64, P]
+    _lib = lib
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(_load().oracle_get_threads())
+
+
+def quantize_per_token(x):
+    """x: float32 [..., d] (exact widening of fp16).  Returns (int8 [..., d], fp32 [...])."""
+    x = _c(x, np.float32)
+    d = x.shape[-1]
+    rows = x.size // d if d else 0
+    q = np.empty(x.shape, np.int8)
+    s = np.empty(x.shape[:-1], np.float32)
+    _load().oracle_quantize_per_token(_ptr(x), rows, d, _ptr(q), _ptr(s))
+    return q, s
+
+
+def quantize_per_tensor(x, groups: int):
+    """x: float32 with x.size divisible by groups; one scale per contiguous group."""
+    x = _c(x, np.float32)
+    n = x.size // groups
+    q = np.empty(x.shape, np.int8)
+    s = np.empty((groups,), np.float32)
+    _load().oracle_quantize_per_tensor(_ptr(x), groups, n, _ptr(q), _ptr(s))
+    return q, s
+
+
+def qk_int32(Qq, Kq):
+    """Qq, Kq: int8 [heads, L, d].  Returns int32 [heads, L, L]."""
+    Qq = _c(Qq, np.int8)
+    Kq = _c(Kq, np.int8)
+    heads, L, d = Qq.shape
+    S = np.empty((heads, L, L), np.int32)
+    _load().oracle_qk_int32(_ptr(Qq), _ptr(Kq), heads, L, d, _ptr(S))
+    return S
+
+
+def attention_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, r0: int = 0, r1=None,
+                   want_stats: bool = False, want_P: bool = False):
+    """One head: Qq/Kq/Vq int8 [L, d], sQ/sK fp32 [L], sV the head's scale.
+
+    Returns O fp64 [r1 - r0, d]; with want_stats also (m, l); with want_P also
+    the int32 P codes [r1 - r0, L]."""
+    Qq = _c(Qq, np.int8)
+    Kq = _c(Kq, np.int8)
+    Vq = _c(Vq, np.int8)
+    sQ = _c(sQ, np.float32)
+    sK = _c(sK, np.float32)
+    L, d = Qq.shape
+    r1 = L if r1 is None else r1
+    n = r1 - r0
+    O = np.empty((n, d), np.float64)
+    m = np.empty((n,), np.float64) if want_stats else None
+    l = np.empty((n,), np.float64) if want_stats else None
+    P = np.empty((n, L), np.int32) if want_P else None
+    _load().oracle_attention_rows(_ptr(Qq), _ptr(Kq), _ptr(Vq), _ptr(sQ), _ptr(sK),
+                                  float(sV), L, d, int(bool(causal)), r0, r1,
+                                  _ptr(O), _ptr(m), _ptr(l), _ptr(P))
+    out = [O]
+    if want_stats:
+        out += [m, l]
+    if want_P:
+        out.append(P)
+    return out[0] if len(out) == 1 else tuple(out)
+
+
+def attention_fp64_rows(Q, K, V, causal: bool, r0: int = 0, r1=None):
+    """One head, unquantised: Q/K/V float32 [L, d].  Returns fp64 [r1 - r0, d]."""
+    Q = _c(Q, np.float32)
+    K = _c(K, np.float32)
+    V = _c(V, np.float32)
+    L, d = Q.shape
+    r1 = L if r1 is None else r1
+    O = np.empty((r1 - r0, d), np.float64)
+    _load().oracle_attention_fp64_rows(_ptr(Q), _ptr(K), _ptr(V), L, d, int(bool(causal)),
+                                       r0, r1, _ptr(O))
+    return O
+
+
+def attention_fwd(Qq, Kq, Vq, sQ, sK, sV, causal: bool):
+    """All heads: Qq/Kq/Vq int8 [BH, L, d] (V_hat row-major, not transposed),
+    sQ/sK fp32 [BH, L], sV fp32 [BH].  Returns O fp64 [BH, L, d]."""
+    BH, L, d = Qq.shape
+    O = np.empty((BH, L, d), np.float64)
+    for h in range(BH):
+        O[h] = attention_rows(Qq[h], Kq[h], Vq[h], sQ[h], sK[h], float(sV[h]), causal)
+    return O
+
+
+def attention_fp64(Q, K, V, causal: bool):
+    """All heads, unquantised: float32 [BH, L, d] -> fp64 [BH, L, d]."""
+    BH, L, d = Q.shape
+    O = np.empty((BH, L, d), np.float64)
+    for h in range(BH):
+        O[h] = attention_fp64_rows(Q[h], K[h], V[h], causal)
+    return O

@@ -1,0 +1,228 @@
+/*
+ * oracle.c -- plain, slow, CPU reference for the INT8-quantised attention
+ * forward pass.  TEST INFRASTRUCTURE ONLY: it is loaded by the tests, by the
+ * smoke check and by the benchmark's CPU-baseline leg, never by the product
+ * path.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes, and where each step comes from:
+ *
+ *   quantiser       IntAttention: A Fully Integer Attention Pipeline for
+ *                   Efficient Edge Inference, section 2.1, eq. 3:
+ *                   s_X = max|X| / 127, X ~= s_X * X_hat, zero-point 0.
+ *                   Granularity: one scale per token row for Q and K
+ *                   (INT-FlashAttention: Enabling Flash Attention for INT8
+ *                   Quantization, abstract: "token-level" quantisation), one
+ *                   scale per L x d tensor for V (IntAttention section 2.1
+ *                   applies eq. 3 per tensor to V in R^{L x d}).
+ *   integer logits  IntAttention section 2.1, eq. 4: A_hat = Q_hat K_hat^T in
+ *                   INT8 x INT8 -> INT32; the rescale alpha is
+ *                   s_Q[i] s_K[j] / sqrt(d) (section 3.1, eq. 8 gives
+ *                   c_int = round(c / alpha) = round(c sqrt(d) / (s_Q s_K))).
+ *   softmax         IntAttention section 2.2, eq. 6: row-max subtraction,
+ *                   two passes over the full row (max, then exp and sum).
+ *   P quantisation  IntAttention section 3.2: probabilities times 127 stored
+ *                   as signed INT8; applied to the unnormalised
+ *                   p = exp(t - m) in (0, 1].
+ *   value path      IntAttention section 2.1, eq. 5: O ~= s_V P V_hat.
+ *   reference       IntAttention section 2.1, eq. 1: O = softmax(Q K^T /
+ *                   sqrt(d)) V in fp64 from the unquantised inputs.
+ *
+ * Causal masking keeps keys j <= i (square, top-left aligned).
+ *
+ * Parity status: every function here is pinned by the CPU tests (closed
+ * forms, invariants, brute force on tiny inputs); see tests/test_oracle_*.py.
+ *
+ * Built with plain gcc -O2 -fopenmp, no fast-math: fp32 divisions are IEEE
+ * round-to-nearest-even, nearbyint() uses the default rounding mode (to
+ * nearest, ties to even).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* threads                                                             */
+/* ------------------------------------------------------------------ */
+
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_get_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------ */
+/* quantiser (IntAttention section 2.1, eq. 3)                         */
+/* ------------------------------------------------------------------ */
+
+/* One symmetric INT8 code: RNE(x / s) clamped to [-127, 127]; s == 0 -> 0.
+ * x / s is one IEEE fp32 division. */
+static int8_t quant_one(float x, float s) {
+    if (s == 0.0f) return 0;
+    float r = nearbyintf(x / s);
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/* Scale of a set of values: max|x| / 127, one IEEE fp32 division. */
+static float scale_of(const float *x, int64_t n) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < n; ++k) {
+        float a = fabsf(x[k]);
+        if (a > amax) amax = a;
+    }
+    return amax / 127.0f;
+}
+
+/* Per-token: `rows` rows of `d` values, one scale per row. */
+void oracle_quantize_per_token(const float *x, int64_t rows, int64_t d,
+                               int8_t *xq, float *scale) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *xr = x + r * d;
+        float s = scale_of(xr, d);
+        scale[r] = s;
+        for (int64_t k = 0; k < d; ++k) xq[r * d + k] = quant_one(xr[k], s);
+    }
+}
+
+/* Per-tensor: `groups` contiguous groups of `group_len` values, one scale
+ * per group (for V: groups = B*H, group_len = L*d). */
+void oracle_quantize_per_tensor(const float *x, int64_t groups,
+                                int64_t group_len, int8_t *xq, float *scale) {
+    for (int64_t g = 0; g < groups; ++g) {
+        const float *xg = x + g * group_len;
+        float s = scale_of(xg, group_len);
+        scale[g] = s;
+#pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < group_len; ++k) xq[g * group_len + k] = quant_one(xg[k], s);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* integer logits (IntAttention section 2.1, eq. 4)                    */
+/* ------------------------------------------------------------------ */
+
+static int32_t dot_i8(const int8_t *a, const int8_t *b, int64_t d) {
+    int32_t acc = 0;
+    for (int64_t k = 0; k < d; ++k) acc += (int32_t)a[k] * (int32_t)b[k];
+    return acc;
+}
+
+/* S[h][i][j] = sum_k Qq[h][i][k] * Kq[h][j][k] for `heads` heads of L x d. */
+void oracle_qk_int32(const int8_t *Qq, const int8_t *Kq, int64_t heads,
+                     int64_t L, int64_t d, int32_t *S) {
+    for (int64_t h = 0; h < heads; ++h) {
+        const int8_t *q = Qq + h * L * d, *k = Kq + h * L * d;
+        int32_t *s = S + h * L * L;
+#pragma omp parallel for schedule(static)
+        for (int64_t i = 0; i < L; ++i)
+            for (int64_t j = 0; j < L; ++j) s[i * L + j] = dot_i8(q + i * d, k + j * d, d);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* quantised attention, rows [r0, r1) of one head                       */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Qq, Kq, Vq: int8 [L][d] of one (b, h); sQ, sK: fp32 [L]; sV: the head's
+ * per-tensor scale.  Writes O[(i - r0) * d + c] in fp64.  Optional outputs
+ * (may be NULL): m_out / l_out [r1 - r0] (row max of t in natural-log units
+ * and the row sum of p), P_out [(r1 - r0) * L] (the INT8 P codes, 0 for
+ * masked keys).
+ */
+void oracle_attention_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
+                           const float *sQ, const float *sK, float sV,
+                           int64_t L, int64_t d, int causal, int64_t r0, int64_t r1,
+                           double *O, double *m_out, double *l_out, int32_t *P_out) {
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = r0; i < r1; ++i) {
+        const int64_t n = causal ? (i + 1) : L; /* keys j < n are visible */
+        double *t = (double *)malloc((size_t)n * sizeof(double));
+        int32_t *ph = (int32_t *)malloc((size_t)n * sizeof(int32_t));
+        int64_t *acc = (int64_t *)calloc((size_t)d, sizeof(int64_t));
+        /* step 1: integer logits and their float rescale (eq. 4, alpha) */
+        for (int64_t j = 0; j < n; ++j) {
+            int32_t sij = dot_i8(Qq + i * d, Kq + j * d, d);
+            t[j] = (double)sij * (double)sQ[i] * (double)sK[j] * inv_sqrt_d;
+        }
+        /* step 2: pass 1, the row max (eq. 6) */
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) if (t[j] > m) m = t[j];
+        /* step 3: pass 2, p = exp(t - m), the row sum, and P codes = RNE(127 p) */
+        double l = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            double p = exp(t[j] - m);
+            l += p;
+            ph[j] = (int32_t)nearbyint(127.0 * p);
+        }
+        /* step 4: integer P V_hat (eq. 5, before the scale) */
+        for (int64_t j = 0; j < n; ++j) {
+            const int8_t *v = Vq + j * d;
+            for (int64_t c = 0; c < d; ++c) acc[c] += (int64_t)ph[j] * (int64_t)v[c];
+        }
+        /* step 5: O = s_V * (P_hat V_hat) / (127 l) */
+        double *o = O + (i - r0) * d;
+        for (int64_t c = 0; c < d; ++c) o[c] = (double)sV * (double)acc[c] / (127.0 * l);
+        if (m_out) m_out[i - r0] = m;
+        if (l_out) l_out[i - r0] = l;
+        if (P_out) {
+            int32_t *pr = P_out + (i - r0) * L;
+            for (int64_t j = 0; j < L; ++j) pr[j] = (j < n) ? ph[j] : 0;
+        }
+        free(t);
+        free(ph);
+        free(acc);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* unquantised fp64 attention (IntAttention section 2.1, eq. 1)         */
+/* ------------------------------------------------------------------ */
+
+/* Q, K, V: fp32 [L][d] of one head (the exact widening of the fp16 inputs).
+ * Writes O[(i - r0) * d + c] for rows [r0, r1). */
+void oracle_attention_fp64_rows(const float *Q, const float *K, const float *V,
+                                int64_t L, int64_t d, int causal, int64_t r0,
+                                int64_t r1, double *O) {
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = r0; i < r1; ++i) {
+        const int64_t n = causal ? (i + 1) : L;
+        double *a = (double *)malloc((size_t)n * sizeof(double));
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (int64_t k = 0; k < d; ++k) s += (double)Q[i * d + k] * (double)K[j * d + k];
+            a[j] = s * inv_sqrt_d;
+            if (a[j] > m) m = a[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            a[j] = exp(a[j] - m);
+            l += a[j];
+        }
+        double *o = O + (i - r0) * d;
+        for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+        for (int64_t j = 0; j < n; ++j)
+            for (int64_t c = 0; c < d; ++c) o[c] += a[j] * (double)V[j * d + c];
+        for (int64_t c = 0; c < d; ++c) o[c] /= l;
+        free(a);
+    }
+}

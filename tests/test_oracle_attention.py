@@ -1,0 +1,195 @@
+"""Pins for the oracle's integer logits and quantised attention.
+
+Sources: IntAttention (A Fully Integer Attention Pipeline for Efficient Edge
+Inference) section 2.1 eq. 1 (attention), eq. 4 (INT8 x INT8 -> INT32 logits,
+alpha = s_Q s_K / sqrt(d) as section 3.1 eq. 8 spells out), eq. 5
+(O ~= s_V P V_hat), section 2.2 eq. 6 (row-max-stable softmax) and section
+3.2 (P x 127 stored as INT8).
+
+Expected values come from closed forms, special cases, hand-built inputs with
+known logits, or brute-force loops on tiny inputs -- never from the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+
+
+def rand_i8(rng, *shape):
+    return rng.integers(-127, 128, shape).astype(np.int8)
+
+
+# ---------------------------------------------------------------- Q K^T ---
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_qk_int32_brute_force(d):
+    rng = np.random.default_rng(10 + d)
+    Qq, Kq = rand_i8(rng, 2, 5, d), rand_i8(rng, 2, 5, d)
+    S = oracle.qk_int32(Qq, Kq)
+    for h in range(2):
+        for i in range(5):
+            for j in range(5):
+                want = 0
+                for k in range(d):
+                    want += int(Qq[h, i, k]) * int(Kq[h, j, k])
+                assert S[h, i, j] == want
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_qk_int32_extremes(d):
+    Qq = np.full((1, 2, d), 127, np.int8)
+    Kq = np.full((1, 2, d), 127, np.int8)
+    Kq[0, 1] = -127
+    S = oracle.qk_int32(Qq, Kq)
+    assert S[0, 0, 0] == 127 * 127 * d and S[0, 0, 1] == -127 * 127 * d
+
+
+# ----------------------------------------------------- quantised attention ---
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_logits_give_mean_of_values(causal):
+    # Q_hat = 0: every logit is 0, p = 1, every P code is 127, so
+    # O_i = s_V * mean over visible keys of V_hat (exact up to fp64 rounding).
+    rng = np.random.default_rng(11)
+    L, d = 37, 64
+    Qq = np.zeros((L, d), np.int8)
+    Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d)
+    sQ = rng.uniform(0.01, 0.1, L).astype(np.float32)
+    sK = rng.uniform(0.01, 0.1, L).astype(np.float32)
+    sV = 0.037
+    O, m, l, P = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, sV, causal, want_stats=True, want_P=True)
+    for i in range(L):
+        n = i + 1 if causal else L
+        want = np.float32(sV) * Vq[:n].astype(np.float64).mean(axis=0)
+        np.testing.assert_allclose(O[i], want, rtol=1e-13, atol=1e-15)
+        assert m[i] == 0.0 and l[i] == n
+        assert np.all(P[i, :n] == 127) and np.all(P[i, n:] == 0)
+
+
+def test_causal_first_row_is_first_value():
+    rng = np.random.default_rng(12)
+    L, d = 9, 128
+    Qq, Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d), rand_i8(rng, L, d)
+    s = rng.uniform(0.01, 0.1, L).astype(np.float32)
+    O = oracle.attention_rows(Qq, Kq, Vq, s, s, 0.5, True)
+    np.testing.assert_array_equal(O[0], 0.5 * Vq[0].astype(np.float64))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_hand_built_logits(d):
+    # Q_hat row 0 = a e_0, K_hat row j = b_j e_0, so S_0j = a b_j exactly and
+    # t_j = a b_j s_Q s_K[j] / sqrt(d); the rest follows eq. 6, section 3.2 and eq. 5.
+    a, b = 100, [127, 50, -127, 0, 90]
+    L = len(b)
+    Qq = np.zeros((L, d), np.int8)
+    Qq[0, 0] = a
+    Kq = np.zeros((L, d), np.int8)
+    Kq[:, 0] = b
+    rng = np.random.default_rng(13)
+    Vq = rand_i8(rng, L, d)
+    sQ = np.full(L, 0.03125, np.float32)
+    sK = np.array([0.02, 0.05, 0.01, 0.07, 0.04], np.float32)
+    sV = 0.02
+    O, m, l, P = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, sV, False, 0, 1,
+                                       want_stats=True, want_P=True)
+    t = [a * b[j] * float(sQ[0]) * float(sK[j]) / math.sqrt(d) for j in range(L)]
+    mx = max(t)
+    p = [math.exp(tj - mx) for tj in t]
+    codes = [round(127 * pj) for pj in p]   # Python round: ties to even
+    assert P[0].tolist() == codes
+    assert m[0] == pytest.approx(mx, rel=1e-15)
+    assert l[0] == pytest.approx(sum(p), rel=1e-15)
+    want = [float(np.float32(sV)) * sum(codes[j] * int(Vq[j, c]) for j in range(L)) / (127 * sum(p))
+            for c in range(d)]
+    np.testing.assert_allclose(O[0], want, rtol=1e-13)
+
+
+def test_causal_rows_ignore_future_keys():
+    rng = np.random.default_rng(14)
+    L, d = 20, 64
+    Qq, Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d), rand_i8(rng, L, d)
+    sQ = rng.uniform(0.005, 0.05, L).astype(np.float32)
+    sK = rng.uniform(0.005, 0.05, L).astype(np.float32)
+    O1 = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, 0.03, True)
+    K2, V2, sK2 = Kq.copy(), Vq.copy(), sK.copy()
+    K2[12:] = rand_i8(rng, L - 12, d)
+    V2[12:] = rand_i8(rng, L - 12, d)
+    sK2[12:] *= 3
+    O2 = oracle.attention_rows(Qq, K2, V2, sQ, sK2, 0.03, True)
+    np.testing.assert_array_equal(O1[:12], O2[:12])
+    assert not np.array_equal(O1[12:], O2[12:])
+
+
+def test_p_codes_range_and_argmax():
+    rng = np.random.default_rng(15)
+    L, d = 50, 128
+    Qq, Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d), rand_i8(rng, L, d)
+    sQ = rng.uniform(0.005, 0.05, L).astype(np.float32)
+    sK = rng.uniform(0.005, 0.05, L).astype(np.float32)
+    _, m, l, P = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, 0.03, False, want_stats=True, want_P=True)
+    S = Qq.astype(np.int64) @ Kq.astype(np.int64).T
+    t = S * sQ[:, None].astype(np.float64) * sK[None, :].astype(np.float64) / math.sqrt(d)
+    assert P.min() >= 0 and P.max() == 127
+    for i in range(L):
+        assert P[i, np.argmax(t[i])] == 127
+        order = np.argsort(t[i])
+        assert np.all(np.diff(P[i, order]) >= 0)   # codes are monotone in the logit
+        assert 1.0 <= l[i] <= L
+
+
+def test_on_grid_inputs_error_is_only_p_rounding():
+    # Q, K, V exactly on the INT8 grid (power-of-two scales, a +-127 per row):
+    # quantisation is lossless, so the gap to fp64 attention comes from the P
+    # codes alone: |O - O_ref| <= 0.5 s_V n max|V_hat| / (127 l).
+    rng = np.random.default_rng(16)
+    L, d = 64, 64
+    def grid(sc):
+        k = rng.integers(-127, 128, (L, d))
+        k[:, 3] = 127
+        return k, (k * sc).astype(np.float32)
+    kq, Q = grid(2.0 ** -6)
+    kk, K = grid(2.0 ** -6)
+    kv, V = grid(2.0 ** -5)
+    V = V.copy()
+    Qq, sQ = oracle.quantize_per_token(Q)
+    Kq, sK = oracle.quantize_per_token(K)
+    Vq, sV = oracle.quantize_per_tensor(V, 1)
+    assert np.array_equal(Qq.astype(np.int64), kq) and np.array_equal(Vq.astype(np.int64), kv)
+    for causal in (False, True):
+        O, m, l = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), causal, want_stats=True)
+        ref = oracle.attention_fp64_rows(Q, K, V, causal)
+        n = (np.arange(L) + 1) if causal else np.full(L, L)
+        bound = 0.5 * float(sV[0]) * n * 127 / (127 * l)
+        assert np.all(np.abs(O - ref).max(axis=1) <= bound * (1 + 1e-9))
+
+
+# ------------------------------------------------------ fp64 reference ---
+
+def test_fp64_brute_force_tiny():
+    rng = np.random.default_rng(17)
+    L, d = 4, 3
+    Q, K, V = (rng.standard_normal((L, d)).astype(np.float32) for _ in range(3))
+    for causal in (False, True):
+        O = oracle.attention_fp64_rows(Q, K, V, causal)
+        for i in range(L):
+            n = i + 1 if causal else L
+            a = [sum(float(Q[i, k]) * float(K[j, k]) for k in range(d)) / math.sqrt(d) for j in range(n)]
+            w = [math.exp(x) for x in a]
+            z = sum(w)
+            for c in range(d):
+                assert O[i, c] == pytest.approx(sum(w[j] * float(V[j, c]) for j in range(n)) / z,
+                                                rel=1e-12, abs=1e-14)
+
+
+def test_fp64_special_cases():
+    rng = np.random.default_rng(18)
+    L, d = 16, 64
+    K, V = (rng.standard_normal((L, d)).astype(np.float32) for _ in range(2))
+    Q = np.zeros((L, d), np.float32)
+    O = oracle.attention_fp64_rows(Q, K, V, False)
+    np.testing.assert_allclose(O, np.broadcast_to(V.astype(np.float64).mean(0), (L, d)), rtol=1e-12, atol=1e-14)
+    Q = rng.standard_normal((L, d)).astype(np.float32)
+    O = oracle.attention_fp64_rows(Q, K, V, True)
+    np.testing.assert_array_equal(O[0], V[0].astype(np.float64))
