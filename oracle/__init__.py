@@ -14,7 +14,12 @@ and marshals numpy arrays.  Each function cites the passage it follows:
   Attention for INT8 Quantization), abstract.
 * ``qk_int32`` -- IntAttention section 2.1, eq. 4 (INT8 x INT8 -> INT32).
 * ``attention_rows`` -- IntAttention eqs. 4-6 and section 3.2 (P x 127 as
-  INT8), eq. 5 for the value path.
+  INT8), eq. 5 for the value path; two passes, P codes against the final
+  row max.
+* ``attention_online_rows`` -- the same steps in FlashAttention's block-wise
+  online order (INT-FlashAttention abstract; FlashAttention-3 abstract): P
+  codes against the running max of the key blocks seen so far.  This is the
+  form the fused kernel computes.
 * ``attention_fp64_rows`` -- IntAttention section 2.1, eq. 1.
 
 All functions are pinned by ``tests/test_oracle_*.py`` (closed forms,
@@ -58,6 +63,8 @@ def _load():
     lib.oracle_qk_int32.argtypes = [P, P, I64, I64, I64, P]
     lib.oracle_attention_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
                                           ctypes.c_int, I64, I64, P, P, P, P]
+    lib.oracle_attention_online_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
+                                                 ctypes.c_int, I64, I64, I64, P, P]
     lib.oracle_attention_fp64_rows.argtypes = [P, P, P, I64, I64, ctypes.c_int, I64, I64, P]
     _lib = lib
     return lib
@@ -139,6 +146,26 @@ def attention_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, r0: int = 0, r1=
     return out[0] if len(out) == 1 else tuple(out)
 
 
+def attention_online_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, block: int = 128,
+                          r0: int = 0, r1=None, want_l: bool = False):
+    """One head, block-wise online form (FlashAttention's forward workflow):
+    P codes against the running max over key blocks of ``block``.  Returns O
+    fp64 [r1 - r0, d] (and the row sums l with want_l)."""
+    Qq = _c(Qq, np.int8)
+    Kq = _c(Kq, np.int8)
+    Vq = _c(Vq, np.int8)
+    sQ = _c(sQ, np.float32)
+    sK = _c(sK, np.float32)
+    L, d = Qq.shape
+    r1 = L if r1 is None else r1
+    O = np.empty((r1 - r0, d), np.float64)
+    l = np.empty((r1 - r0,), np.float64) if want_l else None
+    _load().oracle_attention_online_rows(_ptr(Qq), _ptr(Kq), _ptr(Vq), _ptr(sQ), _ptr(sK),
+                                         float(sV), L, d, int(bool(causal)), int(block),
+                                         r0, r1, _ptr(O), _ptr(l))
+    return (O, l) if want_l else O
+
+
 def attention_fp64_rows(Q, K, V, causal: bool, r0: int = 0, r1=None):
     """One head, unquantised: Q/K/V float32 [L, d].  Returns fp64 [r1 - r0, d]."""
     Q = _c(Q, np.float32)
@@ -159,6 +186,15 @@ def attention_fwd(Qq, Kq, Vq, sQ, sK, sV, causal: bool):
     O = np.empty((BH, L, d), np.float64)
     for h in range(BH):
         O[h] = attention_rows(Qq[h], Kq[h], Vq[h], sQ[h], sK[h], float(sV[h]), causal)
+    return O
+
+
+def attention_online_fwd(Qq, Kq, Vq, sQ, sK, sV, causal: bool, block: int = 128):
+    """All heads, block-wise online form: int8 [BH, L, d] -> fp64 [BH, L, d]."""
+    BH, L, d = Qq.shape
+    O = np.empty((BH, L, d), np.float64)
+    for h in range(BH):
+        O[h] = attention_online_rows(Qq[h], Kq[h], Vq[h], sQ[h], sK[h], float(sV[h]), causal, block)
     return O
 
 

@@ -24,6 +24,9 @@
  *                   as signed INT8; applied to the unnormalised
  *                   p = exp(t - m) in (0, 1].
  *   value path      IntAttention section 2.1, eq. 5: O ~= s_V P V_hat.
+ *   online form     the same steps in FlashAttention's block-wise order
+ *                   (running max and running sum, P codes against the
+ *                   running max), see oracle_attention_online_rows.
  *   reference       IntAttention section 2.1, eq. 1: O = softmax(Q K^T /
  *                   sqrt(d)) V in fp64 from the unquantised inputs.
  *
@@ -189,6 +192,68 @@ void oracle_attention_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
         free(t);
         free(ph);
         free(acc);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* quantised attention in FlashAttention's block-wise online form       */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The same method as oracle_attention_rows, but in the order of
+ * FlashAttention's forward workflow (INT-FlashAttention abstract: the INT8
+ * architecture is compatible with that workflow; FlashAttention-3 abstract:
+ * block-wise softmax interleaved with the two matmuls).  Keys are visited in
+ * blocks of `block`; per block:
+ *   m_new = max(m, max_j t_ij);  alpha = exp(m - m_new)  (0 for the first)
+ *   p_ij  = exp(t_ij - m_new);   codes = RNE(127 p_ij)  (IntAttention 3.2)
+ *   acc   = alpha acc + sum_j codes_ij V_hat_j   (integer block sum, fp64)
+ *   l     = alpha l + sum_j p_ij
+ * and finally O = s_V acc / (127 l) (IntAttention eq. 5).  With one block
+ * this is exactly the two-pass function above.
+ */
+void oracle_attention_online_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
+                                  const float *sQ, const float *sK, float sV,
+                                  int64_t L, int64_t d, int causal, int64_t block,
+                                  int64_t r0, int64_t r1, double *O, double *l_out) {
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = r0; i < r1; ++i) {
+        const int64_t n = causal ? (i + 1) : L;
+        double *t = (double *)malloc((size_t)block * sizeof(double));
+        double *acc = (double *)calloc((size_t)d, sizeof(double));
+        int64_t *blk = (int64_t *)malloc((size_t)d * sizeof(int64_t));
+        double m = -INFINITY, l = 0.0;
+        for (int64_t j0 = 0; j0 < n; j0 += block) {
+            const int64_t nb = (n - j0 < block) ? (n - j0) : block;
+            double bm = -INFINITY;
+            for (int64_t jj = 0; jj < nb; ++jj) {
+                const int64_t j = j0 + jj;
+                int32_t sij = dot_i8(Qq + i * d, Kq + j * d, d);
+                t[jj] = (double)sij * (double)sQ[i] * (double)sK[j] * inv_sqrt_d;
+                if (t[jj] > bm) bm = t[jj];
+            }
+            const double m_new = (bm > m) ? bm : m;
+            const double alpha = (m == -INFINITY) ? 0.0 : exp(m - m_new);
+            double psum = 0.0;
+            for (int64_t c = 0; c < d; ++c) blk[c] = 0;
+            for (int64_t jj = 0; jj < nb; ++jj) {
+                double p = exp(t[jj] - m_new);
+                psum += p;
+                int64_t code = (int64_t)nearbyint(127.0 * p);
+                const int8_t *v = Vq + (j0 + jj) * d;
+                for (int64_t c = 0; c < d; ++c) blk[c] += code * (int64_t)v[c];
+            }
+            for (int64_t c = 0; c < d; ++c) acc[c] = alpha * acc[c] + (double)blk[c];
+            l = alpha * l + psum;
+            m = m_new;
+        }
+        double *o = O + (i - r0) * d;
+        for (int64_t c = 0; c < d; ++c) o[c] = (double)sV * acc[c] / (127.0 * l);
+        if (l_out) l_out[i - r0] = l;
+        free(t);
+        free(acc);
+        free(blk);
     }
 }
 

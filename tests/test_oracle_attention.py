@@ -193,3 +193,85 @@ def test_fp64_special_cases():
     Q = rng.standard_normal((L, d)).astype(np.float32)
     O = oracle.attention_fp64_rows(Q, K, V, True)
     np.testing.assert_array_equal(O[0], V[0].astype(np.float64))
+
+
+# ------------------------------------------------ block-wise online form ---
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_online_single_block_equals_two_pass(causal):
+    # One block of keys: the running max is the final max, so the online form
+    # performs exactly the two-pass arithmetic.
+    rng = np.random.default_rng(20)
+    L, d = 100, 64
+    Qq, Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d), rand_i8(rng, L, d)
+    sQ = rng.uniform(0.005, 0.05, L).astype(np.float32)
+    sK = rng.uniform(0.005, 0.05, L).astype(np.float32)
+    O2 = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, 0.03, causal)
+    O1 = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, 0.03, causal, block=128)
+    np.testing.assert_array_equal(O1, O2)
+
+
+def test_online_equals_two_pass_when_max_is_in_first_block():
+    # Key 0 is aligned with every query and much larger than the rest: the
+    # running max is final after the first block, alpha = 1 afterwards and the
+    # block sums add up to the two-pass integer sum exactly (only the order of
+    # the fp64 row-sum additions differs).
+    rng = np.random.default_rng(21)
+    L, d = 300, 128
+    Qq = rng.integers(1, 128, (L, d)).astype(np.int8)
+    Kq = rng.integers(-20, 21, (L, d)).astype(np.int8)
+    Kq[0] = 127
+    Vq = rand_i8(rng, L, d)
+    sQ = rng.uniform(0.005, 0.02, L).astype(np.float32)
+    sK = np.full(L, 0.01, np.float32)
+    for causal in (False, True):
+        O2 = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, 0.03, causal)
+        for block in (16, 64, 128):
+            O1 = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, 0.03, causal, block=block)
+            np.testing.assert_allclose(O1, O2, rtol=1e-13, atol=0)
+
+
+def test_online_hand_built_two_blocks():
+    # block = 2, keys with logits [0, 1 | 3, 2] (row 0): the P codes of the
+    # first block are taken against m = 1, rescaled by e^(1 - 3) when block 2
+    # raises the max to 3 (FlashAttention's running max / running sum).
+    d = 64
+    a, b = 64, [0, 1, 3, 2]                 # S_0j = a b_j; t_j = a b_j sQ sK / 8 = b_j
+    L = len(b)
+    Qq = np.zeros((L, d), np.int8)
+    Qq[0, 0] = a
+    Kq = np.zeros((L, d), np.int8)
+    Kq[:, 0] = b
+    sQ = np.full(L, 0.125, np.float32)
+    sK = np.full(L, 1.0, np.float32)
+    rng = np.random.default_rng(22)
+    Vq = rand_i8(rng, L, d)
+    O, l = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, 0.5, False, block=2, r0=0, r1=1,
+                                        want_l=True)
+    c1 = [round(127 * math.exp(t - 1)) for t in (0, 1)]
+    c2 = [round(127 * math.exp(t - 3)) for t in (3, 2)]
+    alpha = math.exp(1 - 3)
+    acc = [alpha * (c1[0] * int(Vq[0, c]) + c1[1] * int(Vq[1, c])) + (c2[0] * int(Vq[2, c]) + c2[1] * int(Vq[3, c]))
+           for c in range(d)]
+    lw = alpha * (math.exp(-1) + 1) + (1 + math.exp(-1))
+    assert l[0] == pytest.approx(lw, rel=1e-15)
+    np.testing.assert_allclose(O[0], [0.5 * x / (127 * lw) for x in acc], rtol=1e-13)
+    # and the two-pass form takes all four codes against m = 3
+    O2 = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, 0.5, False, 0, 1)
+    c = [round(127 * math.exp(t - 3)) for t in b]
+    want = [0.5 * sum(c[j] * int(Vq[j, k]) for j in range(4)) / (127 * sum(math.exp(t - 3) for t in b))
+            for k in range(d)]
+    np.testing.assert_allclose(O2[0], want, rtol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_online_constant_logits(causal):
+    rng = np.random.default_rng(23)
+    L, d = 300, 64
+    Qq = np.zeros((L, d), np.int8)
+    Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d)
+    s = rng.uniform(0.01, 0.1, L).astype(np.float32)
+    O = oracle.attention_online_rows(Qq, Kq, Vq, s, s, 0.25, causal, block=128)
+    for i in range(L):
+        n = i + 1 if causal else L
+        np.testing.assert_allclose(O[i], 0.25 * Vq[:n].astype(np.float64).mean(0), rtol=1e-13, atol=1e-15)
