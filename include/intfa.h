@@ -1,0 +1,167 @@
+/*
+ * intfa.h -- C ABI of libintfa: INT8-quantised attention forward pass on
+ * NVIDIA B200 (sm_100a), in the style of INT-FlashAttention.
+ *
+ * The method (sources are web pages; each entry point cites its passage):
+ *   - INT-FlashAttention: Enabling Flash Attention for INT8 Quantization,
+ *     abstract: an INT8 FlashAttention forward pass with token-level
+ *     (per-row) quantisation of Q and K.
+ *   - IntAttention: A Fully Integer Attention Pipeline for Efficient Edge
+ *     Inference, section 2.1: the symmetric quantiser (eq. 3), integer
+ *     logits with a float rescale (eq. 4), O ~= s_V P V_hat (eq. 5);
+ *     section 2.2: the row-max-stable softmax (eq. 6); section 3.2:
+ *     probabilities multiplied by 127 and stored as signed INT8.
+ *   - FlashAttention-3 (arXiv 2407.08608), abstract: block-wise softmax
+ *     interleaved with the two matmuls (running max and running sum).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, unless the
+ *     name ends in _host.  The library allocates no device memory; scratch
+ *     space is a caller-provided workspace whose size a *_workspace_size
+ *     function returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are asynchronous on that stream; INTFA_OK means the
+ *     arguments were valid and the kernels were launched.  Faults inside a
+ *     kernel surface at the caller's next synchronisation.
+ *   - Arguments are checked on the host before anything is launched; a
+ *     failed check returns an error code and launches nothing.
+ *   - Inputs must be finite; NaN or Inf inputs give unspecified results.
+ *   - Every entry point is thread-safe and keeps no state between calls,
+ *     except the device-side status word read by intfa_device_status.
+ */
+#ifndef INTFA_H_
+#define INTFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+typedef enum {
+    INTFA_OK = 0,
+    INTFA_ERR_INVALID_ARG = 1,    /* null pointer, negative or zero size, overflow */
+    INTFA_ERR_UNSUPPORTED = 2,    /* a shape the kernels do not implement (e.g. d) */
+    INTFA_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
+    INTFA_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+    INTFA_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up on a bounded wait (see
+                                     intfa_device_status) */
+    INTFA_ERR_WORKSPACE = 6       /* workspace missing or too small */
+} intfa_status;
+
+/* Static description of a status code; never NULL. */
+const char *intfa_status_string(int status);
+
+/*
+ * Per-token symmetric INT8 quantisation (IntAttention section 2.1, eq. 3,
+ * applied to each token row as INT-FlashAttention's abstract specifies).
+ *
+ *   x_f16  : fp16 [rows][d], row-major, 16-byte aligned.
+ *   x_q    : int8 [rows][d] out, 16-byte aligned (8-byte for d == 8).
+ *   scale  : fp32 [rows] out.
+ * For each row: s = max_k |x_k| / 127 (one IEEE fp32 division),
+ * x_q[k] = clamp(round-half-even(x_k / s), -127, 127) with x_k / s the IEEE
+ * fp32 quotient; an all-zero row gives s = 0 and codes 0.  Bit-exact.
+ * d must be one of 8, 16, 32, 64, 128, 256; rows >= 0 (0 is a no-op).
+ */
+int intfa_quantize_per_token(const void *x_f16, int64_t rows, int d, int8_t *x_q,
+                             float *scale, void *stream);
+
+/*
+ * Per-tensor symmetric INT8 quantisation (IntAttention section 2.1, eq. 3,
+ * one scale per L x d tensor, as that section applies it to V).
+ *
+ *   x_f16  : fp16 [groups][rows][cols], row-major, 16-byte aligned.
+ *   scale  : fp32 [groups] out: s_g = max |x| over group g / 127.
+ *   x_q    : int8 out, codes as in intfa_quantize_per_token with s_g.
+ *            transpose == 0: [groups][rows][cols] (same layout as x).
+ *            transpose == 1: [groups][cols][ld] with ld = intfa_vt_ld(rows):
+ *            the transpose of each group, rows padded with zero codes up to
+ *            ld.  This is the V_hat^T layout intfa_attention_fwd reads.
+ *   workspace : device scratch of at least
+ *            intfa_quantize_per_tensor_workspace_size(groups) bytes, 16-byte
+ *            aligned; its contents on entry do not matter.
+ * cols must be a multiple of 8 and, with transpose, at most 256.
+ */
+size_t intfa_quantize_per_tensor_workspace_size(int64_t groups);
+int64_t intfa_vt_ld(int64_t rows);
+int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int64_t rows, int cols,
+                              int transpose, int8_t *x_q, float *scale, void *workspace,
+                              size_t workspace_bytes, void *stream);
+
+/*
+ * Fused INT8 attention forward pass (INT-FlashAttention abstract; IntAttention
+ * eqs. 4-6, section 3.2 and eq. 5; FlashAttention-3's block-wise online
+ * softmax), one kernel:
+ *   S = Q_hat K_hat^T (INT8 x INT8 -> INT32, tcgen05 tensor cores, TMEM)
+ *   t_ij = S_ij s_Q[i] s_K[j] / sqrt(d), keys masked j > i when causal
+ *   per key block of 128: running max m, p = exp(t - m), P_hat = RNE(127 p),
+ *   O_blk = P_hat V_hat (INT8 x INT8 -> INT32), acc = alpha acc + O_blk,
+ *   l = alpha l + sum p, alpha = exp(m_old - m_new)
+ *   O = s_V acc / (127 l), written as fp16.
+ *
+ *   Q_q, K_q : int8 [B][H][L][d] (from intfa_quantize_per_token), 16-B aligned.
+ *   Vt_q     : int8 [B][H][d][intfa_vt_ld(L)] = V_hat transposed per head
+ *              (from intfa_quantize_per_tensor with transpose = 1), 16-B aligned.
+ *   s_Q, s_K : fp32 [B][H][L]; s_V : fp32 [B][H] (one scale per head).
+ *   O_f16    : fp16 [B][H][L][d] out, 16-byte aligned.
+ *   d in {64, 128}; L >= 1 (any value; the last key/query block is masked);
+ *   causal in {0, 1} (square, top-left aligned: key j visible to query i iff
+ *   j <= i).  Returns INTFA_ERR_DEVICE_TIMEOUT only via intfa_device_status.
+ */
+int intfa_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                        const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                        int L, int d, int causal, void *O_f16, void *stream);
+
+/*
+ * Debug: the integer logits S = Q_hat K_hat^T (IntAttention eq. 4) for every
+ * head, int32 [B][H][L][L], computed by the same TMA + tcgen05 path the fused
+ * kernel uses for its first contraction.  Same layout rules as
+ * intfa_attention_fwd for Q_q and K_q; S must be 16-byte aligned.
+ */
+int intfa_debug_qk(const int8_t *Q_q, const int8_t *K_q, int B, int H, int L, int d,
+                   int32_t *S, void *stream);
+
+/*
+ * Whole hot path on device buffers: quantise Q and K per token, V per head
+ * (transposed), then the fused attention.  Q, K, V, O: fp16 [B][H][L][d]
+ * device pointers; workspace: intfa_forward_workspace_size(B, H, L, d) bytes of
+ * device memory, 256-byte aligned.  Optional outputs of the quantisation live
+ * in the workspace at the offsets intfa_forward_workspace_layout reports.
+ */
+size_t intfa_forward_workspace_size(int B, int H, int L, int d);
+/* offsets[0..5] = byte offsets of Q_q, K_q, Vt_q, s_Q, s_K, s_V inside the
+ * workspace; returns INTFA_OK or INTFA_ERR_INVALID_ARG. */
+int intfa_forward_workspace_layout(int B, int H, int L, int d, size_t offsets[6]);
+int intfa_forward(const void *Q_f16, const void *K_f16, const void *V_f16, int B, int H, int L,
+                  int d, int causal, void *O_f16, void *workspace, size_t workspace_bytes,
+                  void *stream);
+
+/*
+ * The same from HOST memory: copies Q, K, V (fp16, host, pinned for
+ * asynchronous copies) to the device, runs intfa_forward and copies O back to
+ * O_f16_host.  workspace: intfa_forward_host_workspace_size(B, H, L, d) bytes
+ * of device memory, 256-byte aligned.  Asynchronous on `stream`: O_f16_host
+ * is valid after the stream is synchronised.
+ */
+size_t intfa_forward_host_workspace_size(int B, int H, int L, int d);
+int intfa_forward_host(const void *Q_f16_host, const void *K_f16_host, const void *V_f16_host,
+                       int B, int H, int L, int d, int causal, void *O_f16_host,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Device-side status: every wait inside the fused kernel is bounded; a kernel
+ * that gives up records a nonzero word and returns without hanging the GPU.
+ * Synchronises the current device, returns INTFA_OK if the word is zero,
+ * INTFA_ERR_DEVICE_TIMEOUT otherwise (and the word in *word if non-NULL);
+ * clear != 0 resets it to zero.
+ */
+int intfa_device_status(int clear, uint32_t *word);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INTFA_H_ */

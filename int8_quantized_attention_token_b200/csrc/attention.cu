@@ -1,0 +1,616 @@
+// attention.cu -- fused INT8 attention forward pass for sm_100a.
+//
+// Method (INT-FlashAttention: Enabling Flash Attention for INT8 Quantization,
+// abstract; IntAttention: A Fully Integer Attention Pipeline for Efficient
+// Edge Inference, section 2.1 eqs. 4-5, section 2.2 eq. 6, section 3.2;
+// FlashAttention-3, abstract, for the block-wise online softmax):
+//   S_ij  = sum_k Q_hat[i,k] K_hat[j,k]                   INT8 x INT8 -> INT32
+//   t_ij  = S_ij s_Q[i] s_K[j] / sqrt(d)                  (keys j > i masked if causal)
+//   per key block of 128:  m_new = max(m, max_j t_ij), alpha = exp(m - m_new)
+//                          p_ij = exp(t_ij - m_new),  P_hat = RNE(127 p_ij)
+//                          acc  = alpha acc + P_hat V_hat   (INT8 x INT8 -> INT32)
+//                          l    = alpha l + sum_j p_ij
+//   O_i   = s_V acc_i / (127 l_i)                          -> fp16
+// exp is evaluated as exp2 with log2(e) folded into the per-row constant.
+//
+// B200 design (one CTA per 128-query tile of one (b, h)):
+//   warp 8      TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
+//               block's s_K values into a 3-stage shared-memory ring.
+//   warp 9      tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
+//               kind::i8 into one of two TMEM S buffers; P V with the P codes
+//               read straight from TMEM (aliasing the first 32 columns of the
+//               S buffer they came from) into a TMEM O block; owns the TMEM
+//               allocation (512 columns: S0, S1, O).
+//   warps 0-3   softmax: one thread per query row; reads its S row from
+//               TMEM, runs the online max / sum, writes the row's 128 P codes
+//               back to TMEM as the A operand of P V, and hands alpha to the
+//               correction warps through shared memory.
+//   warps 4-7   correction: one thread per query row; keeps the fp32 output
+//               row in registers, folds each int32 P V block in with alpha,
+//               and writes the normalised fp16 row at the end.
+// Every wait is bounded (clock-based); a timeout records a status word,
+// raises a CTA-wide abort flag, drains in-flight copies and MMAs, frees TMEM
+// and returns.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace intfa {
+
+__device__ uint32_t g_status;  // 0 = fine; else 0x100 | wait site of the first timeout
+
+namespace {
+
+constexpr int BM = 128;                       // query rows per CTA
+constexpr int BN = 128;                       // keys per block
+constexpr int NS = 3;                         // K/V ring depth
+constexpr int kThreads = 320;                 // 10 warps
+constexpr int kTmemCols = 512;
+constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
+constexpr float kLog2e = 1.4426950408889634f;
+
+// -------------------------------------------------------- bounded waits ---
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         uint32_t site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            atomicCAS(&g_status, 0u, 0x100u | site);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Warp-uniform bounded wait: every lane polls, the warp agrees on the result.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t site) {
+    const bool ok = wait_bar(bar, parity, abort_flag, site);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitCycles) {
+            atomicCAS(&g_status, 0u, 0x1FFu);
+            return;
+        }
+    }
+}
+
+// ------------------------------------------------------- shared memory ---
+
+template <int D>
+struct alignas(1024) AttnSmem {
+    uint8_t q[BM * D];          // Q_hat tile, K-major, TMA-swizzled
+    uint8_t k[NS][BN * D];      // K_hat tiles
+    uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
+    float sk[NS][BN];           // s_K of each key block
+    float alpha[2][BM];         // softmax -> correction
+    float lsum[BM];             // final row sums
+    uint64_t q_full;
+    uint64_t k_full[NS], v_full[NS], kv_empty[NS];
+    uint64_t s_full[2], p_full[2];
+    uint64_t o_full, o_empty;
+    uint64_t a_full[2], a_empty[2];
+    uint64_t l_full, mma_drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D>
+constexpr size_t attn_smem_bytes() {
+    // 1024 for manual alignment; D = 64 is padded so that only one CTA (which
+    // holds all 512 TMEM columns) is resident per SM.
+    size_t s = sizeof(AttnSmem<D>) + 1024;
+    return s < 120 * 1024 ? 120 * 1024 : s;
+}
+
+template <int D>
+__device__ __forceinline__ AttnSmem<D> &get_smem() {
+    extern __shared__ uint8_t smem_raw[];
+    const uintptr_t p = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
+    return *reinterpret_cast<AttnSmem<D> *>(p);
+}
+
+// ---------------------------------------------------------------- kernel ---
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
+                    const float *__restrict__ sK, const float *__restrict__ sV,
+                    __half *__restrict__ O, int BH, int L, int causal) {
+    AttnSmem<D> &sm = get_smem<D>();
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    const int ntiles = (L + BM - 1) / BM;
+    const int t = blockIdx.x / BH;
+    const int bh = blockIdx.x - t * BH;
+    const int qt = causal ? (ntiles - 1 - t) : t;    // heaviest causal tiles first
+    const int q0 = qt * BM;
+    const int nb = causal ? (qt + 1) : (L + BN - 1) / BN;
+    volatile int *abort_flag = &sm.abort_flag;
+
+    if (tid == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sm.k_full[s], 32);
+            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1 + BM);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.p_full[b], BM);
+            mbar_init(&sm.a_full[b], BM);
+            mbar_init(&sm.a_empty[b], BM);
+        }
+        mbar_init(&sm.o_full, 1);
+        mbar_init(&sm.o_empty, BM);
+        mbar_init(&sm.l_full, BM);
+        mbar_init(&sm.mma_drain, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sm.tmem_base;
+    const uint32_t tS = tbase;          // S0 at column 0, S1 at column 128
+    const uint32_t tO = tbase + 256;    // O block, D columns
+
+    if (warp == 8) {
+        // ------------------------------------------------ TMA producer ---
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(&sm.q_full, BM * D);
+            tma_load_3d(&tmQ, &sm.q_full, sm.q, 0, q0, bh);
+        }
+        int issued = 0;
+        for (int j = 0; j < nb; ++j) {
+            const int st = j % NS;
+            if (j >= NS && !warp_wait(&sm.kv_empty[st], ((j / NS) - 1) & 1, abort_flag, 1)) break;
+            const int key = j * BN + 4 * lane;
+            const float *src = sK + static_cast<int64_t>(bh) * L;
+            float4 v4;
+            v4.x = key + 0 < L ? __ldg(src + key + 0) : 0.0f;
+            v4.y = key + 1 < L ? __ldg(src + key + 1) : 0.0f;
+            v4.z = key + 2 < L ? __ldg(src + key + 2) : 0.0f;
+            v4.w = key + 3 < L ? __ldg(src + key + 3) : 0.0f;
+            *reinterpret_cast<float4 *>(&sm.sk[st][4 * lane]) = v4;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.k_full[st], BN * D);
+                tma_load_3d(&tmK, &sm.k_full[st], sm.k[st], 0, j * BN, bh);
+                mbar_arrive_expect_tx(&sm.v_full[st], D * BN);
+                tma_load_3d(&tmV, &sm.v_full[st], sm.v[st], j * BN, 0, bh);
+            } else {
+                mbar_arrive(&sm.k_full[st]);
+            }
+            __syncwarp();
+            issued = j + 1;
+        }
+        // Drain: the last load issued into each stage (and Q) has landed.
+        drain_wait(&sm.q_full, 0);
+        for (int s = 0; s < NS && s < issued; ++s) {
+            const int last = s + ((issued - 1 - s) / NS) * NS;  // last block using stage s
+            drain_wait(&sm.k_full[s], (last / NS) & 1);
+            drain_wait(&sm.v_full[s], (last / NS) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ------------------------------------------------ MMA issuer ---
+        constexpr uint32_t kSwQK = (D == 128) ? kSwizzle128B : kSwizzle64B;
+        constexpr uint32_t kSboQK = 8 * D;      // 8 rows of D bytes
+        const uint32_t idesc_qk = make_idesc_i8(BM, BN);
+        const uint32_t idesc_pv = make_idesc_i8(BM, D);
+        const uint64_t qdesc = make_sdesc(smem_u32(sm.q), kSboQK, kSwQK);
+        bool ok = warp_wait(&sm.q_full, 0, abort_flag, 2);
+        tc_fence_after();
+
+        auto issue_pv = [&](int j) -> bool {
+            const int b = j & 1, st = j % NS;
+            if (!warp_wait(&sm.p_full[b], (j >> 1) & 1, abort_flag, 3)) return false;
+            if (!warp_wait(&sm.v_full[st], (j / NS) & 1, abort_flag, 4)) return false;
+            if (j >= 1 && !warp_wait(&sm.o_empty, (j - 1) & 1, abort_flag, 5)) return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
+#pragma unroll
+                for (int k = 0; k < BN / 32; ++k)
+                    mma_i8_ts(tO, tS + b * BN + 8 * k, vdesc + 2 * k, idesc_pv, k > 0);
+                mma_commit(&sm.o_full);
+                mma_commit(&sm.kv_empty[st]);
+            }
+            __syncwarp();
+            return true;
+        };
+
+        for (int j = 0; ok && j < nb; ++j) {
+            const int st = j % NS, b = j & 1;
+            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 6)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
+#pragma unroll
+                for (int k = 0; k < D / 32; ++k)
+                    mma_i8_ss(tS + b * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
+                mma_commit(&sm.s_full[b]);
+            }
+            __syncwarp();
+            if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        }
+        if (ok) issue_pv(nb - 1);
+        // Drain: every MMA this warp issued has completed before TMEM is freed.
+        if (lane == 0) mma_commit(&sm.mma_drain);
+        __syncwarp();
+        drain_wait(&sm.mma_drain, 0);
+        __syncwarp();
+    } else if (warp < 4) {
+        // --------------------------------------------------- softmax ---
+        const int row = tid;
+        const int qi = q0 + row;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+        const float c = (qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
+                        (kLog2e / sqrtf(static_cast<float>(D)));
+        float m_old = -INFINITY, l = 0.0f;
+        for (int j = 0; j < nb; ++j) {
+            const int b = j & 1, st = j % NS;
+            if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, abort_flag, 7)) break;
+            // s_K of this block: published by the producer's release-arrive
+            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 12)) break;
+            tc_fence_after();
+            uint32_t sr[BN];
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch)
+                tmem_ld32(tS + lane_off + b * BN + 32 * ch,
+                          *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * ch]));
+            tmem_wait_ld();
+            float v[BN];
+            const float *skp = sm.sk[st];
+#pragma unroll
+            for (int jj = 0; jj < BN; ++jj)
+                v[jj] = static_cast<float>(static_cast<int32_t>(sr[jj])) * skp[jj];
+            const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
+            if (need_mask) {
+#pragma unroll
+                for (int jj = 0; jj < BN; ++jj) {
+                    const int key = j * BN + jj;
+                    if (key >= L || (causal && key > qi)) v[jj] = -INFINITY;
+                }
+            }
+            mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
+            float bm = -INFINITY;
+#pragma unroll
+            for (int jj = 0; jj < BN; ++jj) bm = fmaxf(bm, v[jj]);
+            const float m_new = fmaxf(m_old, bm);
+            const float alpha = (m_old == -INFINITY) ? 0.0f : exp2f(c * (m_old - m_new));
+            const float cm = c * m_new;
+            float ps = 0.0f;
+            uint32_t pk[32];
+#pragma unroll
+            for (int w = 0; w < 32; ++w) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x = v[4 * w + e];
+                    const float p = (x == -INFINITY) ? 0.0f : exp2f(fmaf(x, c, -cm));
+                    ps += p;
+                    const uint32_t code = static_cast<uint32_t>(__float2int_rn(p * 127.0f));
+                    word |= code << (8 * e);
+                }
+                pk[w] = word;
+            }
+            l = l * alpha + ps;
+            tmem_st32(tS + lane_off + b * BN, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_full[b]);
+            if (j >= 2 && !warp_wait(&sm.a_empty[b], ((j >> 1) - 1) & 1, abort_flag, 8)) break;
+            sm.alpha[b][row] = alpha;
+            mbar_arrive(&sm.a_full[b]);
+            m_old = m_new;
+        }
+        sm.lsum[row] = l;
+        mbar_arrive(&sm.l_full);
+    } else {
+        // ------------------------------------------------ correction ---
+        const int row = tid - 128;
+        const int qi = q0 + row;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * (warp - 4)) << 16;
+        float o[D];
+#pragma unroll
+        for (int c = 0; c < D; ++c) o[c] = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < nb; ++j) {
+            const int b = j & 1;
+            if (!warp_wait(&sm.o_full, j & 1, abort_flag, 9)) { ok = false; break; }
+            if (!warp_wait(&sm.a_full[b], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
+            tc_fence_after();
+            const float alpha = sm.alpha[b][row];
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t r[32];
+                tmem_ld32(tO + lane_off + 32 * ch, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    o[32 * ch + c] = fmaf(o[32 * ch + c], alpha,
+                                          static_cast<float>(static_cast<int32_t>(r[c])));
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.o_empty);
+            mbar_arrive(&sm.a_empty[b]);
+        }
+        if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11) && qi < L) {
+            const float l = sm.lsum[row];
+            const float f = __ldg(sV + bh) / (127.0f * l);
+            uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(bh) * L + qi) * D);
+#pragma unroll
+            for (int c8 = 0; c8 < D / 8; ++c8) {
+                uint4 w;
+                __half2 *h = reinterpret_cast<__half2 *>(&w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    h[e] = __floats2half2_rn(o[8 * c8 + 2 * e] * f, o[8 * c8 + 2 * e + 1] * f);
+                dst[c8] = w;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------- debug Q K^T ---
+
+template <int D>
+struct alignas(1024) QKSmem {
+    uint8_t q[BM * D];
+    uint8_t k[BN * D];
+    uint64_t full, done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+    debug_qk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    int L, int32_t *__restrict__ S) {
+    extern __shared__ uint8_t smem_raw[];
+    QKSmem<D> &sm = *reinterpret_cast<QKSmem<D> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int q0 = blockIdx.x * BM, k0 = blockIdx.y * BN, bh = blockIdx.z;
+    volatile int *abort_flag = &sm.abort_flag;
+    if (tid == 0) {
+        mbar_init(&sm.full, 1);
+        mbar_init(&sm.done, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sm.tmem_base;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&sm.full, BM * D + BN * D);
+        tma_load_3d(&tmQ, &sm.full, sm.q, 0, q0, bh);
+        tma_load_3d(&tmK, &sm.full, sm.k, 0, k0, bh);
+    }
+    bool ok = warp_wait(&sm.full, 0, abort_flag, 20);
+    tc_fence_after();
+    if (tid == 0 && ok) {
+        constexpr uint32_t kSw = (D == 128) ? kSwizzle128B : kSwizzle64B;
+        const uint64_t qd = make_sdesc(smem_u32(sm.q), 8 * D, kSw);
+        const uint64_t kd = make_sdesc(smem_u32(sm.k), 8 * D, kSw);
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) mma_i8_ss(tbase, qd + 2 * k, kd + 2 * k, make_idesc_i8(BM, BN), k > 0);
+        mma_commit(&sm.done);
+    }
+    if (!ok) {
+        drain_wait(&sm.full, 0);
+    } else if (warp_wait(&sm.done, 0, abort_flag, 21)) {
+        tc_fence_after();
+        const int qi = q0 + tid;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(tbase + lane_off + 32 * ch, r);
+            tmem_wait_ld();
+            if (qi < L) {
+                int32_t *dst = S + (static_cast<int64_t>(bh) * L + qi) * L + k0 + 32 * ch;
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    if (k0 + 32 * ch + c < L) dst[c] = static_cast<int32_t>(r[c]);
+            }
+        }
+    } else if (tid == 0) {
+        // the MMA may still be in flight: wait for it before freeing TMEM
+        drain_wait(&sm.done, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, 128);
+    }
+}
+
+// ----------------------------------------------------------- host side ---
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            (void)cudaGetLastError();
+    }
+    return fn;
+}
+
+// 3-D uint8 tensor map: dims (x = inner, y, z), byte strides of y and z, box (bx, by, 1).
+int make_map(CUtensorMap *map, const void *base, uint64_t x, uint64_t y, uint64_t z,
+             uint64_t stride_y, uint64_t stride_z, uint32_t bx, uint32_t by,
+             CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return INTFA_ERR_CUDA;
+    const cuuint64_t dims[3] = {x, y, z};
+    const cuuint64_t strides[2] = {stride_y, stride_z};
+    const cuuint32_t box[3] = {bx, by, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? INTFA_OK : INTFA_ERR_CUDA;
+}
+
+template <int D>
+int launch_attn(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
+                const float *sK, const float *sV, int B, int H, int L, int causal, void *O,
+                cudaStream_t stream) {
+    const int BH = B * H;
+    const int64_t ld = intfa_vt_ld(L);
+    const CUtensorMapSwizzle swz = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUtensorMap mq, mk, mv;
+    int rc = make_map(&mq, Qq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BM, swz);
+    if (!rc) rc = make_map(&mk, Kq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BN, swz);
+    if (!rc) rc = make_map(&mv, Vt, ld, D, BH, ld, static_cast<uint64_t>(ld) * D, BN, D,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    const size_t smem = attn_smem_bytes<D>();
+    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(smem)));
+    if (rc) return rc;
+    const int ntiles = (L + BM - 1) / BM;
+    const unsigned grid = static_cast<unsigned>(ntiles) * static_cast<unsigned>(BH);
+    attn_fwd_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, sQ, sK, sV,
+                                                          static_cast<__half *>(O), BH, L, causal);
+    return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+int launch_debug_qk(const int8_t *Qq, const int8_t *Kq, int BH, int L, int32_t *S,
+                    cudaStream_t stream) {
+    const CUtensorMapSwizzle swz = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUtensorMap mq, mk;
+    int rc = make_map(&mq, Qq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BM, swz);
+    if (!rc) rc = make_map(&mk, Kq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BN, swz);
+    if (rc) return rc;
+    const size_t smem = sizeof(QKSmem<D>) + 1024;
+    rc = cuda_status(cudaFuncSetAttribute(debug_qk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(smem)));
+    if (rc) return rc;
+    const unsigned nt = static_cast<unsigned>((L + BM - 1) / BM);
+    debug_qk_kernel<D><<<dim3(nt, nt, BH), 128, smem, stream>>>(mq, mk, L, S);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
+                         const float *sK, const float *sV, int B, int H, int L, int d, int causal,
+                         void *O, cudaStream_t stream) {
+    if (d == 128) return launch_attn<128>(Qq, Kq, Vt, sQ, sK, sV, B, H, L, causal, O, stream);
+    if (d == 64) return launch_attn<64>(Qq, Kq, Vt, sQ, sK, sV, B, H, L, causal, O, stream);
+    return INTFA_ERR_UNSUPPORTED;
+}
+
+}  // namespace intfa
+
+// ------------------------------------------------------------------ C ABI ---
+
+namespace {
+int check_attn_shape(int B, int H, int L, int d) {
+    if (B <= 0 || H <= 0 || L <= 0) return INTFA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return INTFA_ERR_UNSUPPORTED;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    if (bh > (1 << 24)) return INTFA_ERR_UNSUPPORTED;
+    const int64_t tiles = (static_cast<int64_t>(L) + 127) / 128;
+    if (tiles * bh > 0x7FFFFFFF) return INTFA_ERR_UNSUPPORTED;
+    if (L > 131072) return INTFA_ERR_UNSUPPORTED;   // int32 P V accumulation bound: 127^2 L < 2^31
+    return INTFA_OK;
+}
+}  // namespace
+
+extern "C" int intfa_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                   const float *s_Q, const float *s_K, const float *s_V, int B,
+                                   int H, int L, int d, int causal, void *O_f16, void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    if (!Q_q || !K_q || !Vt_q || !s_Q || !s_K || !s_V || !O_f16) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(Vt_q) || !aligned16(O_f16) ||
+        (reinterpret_cast<uintptr_t>(s_Q) & 3u) || (reinterpret_cast<uintptr_t>(s_K) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_V) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    return launch_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
+                                static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int intfa_debug_qk(const int8_t *Q_q, const int8_t *K_q, int B, int H, int L, int d,
+                              int32_t *S, void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (!Q_q || !K_q || !S) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(S)) return INTFA_ERR_MISALIGNED;
+    const int BH = B * H;
+    if (static_cast<int64_t>((L + 127) / 128) > 65535 || BH > 65535) return INTFA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return d == 128 ? launch_debug_qk<128>(Q_q, K_q, BH, L, S, s) : launch_debug_qk<64>(Q_q, K_q, BH, L, S, s);
+}
+
+extern "C" int intfa_device_status(int clear, uint32_t *word) {
+    using namespace intfa;
+    int rc = cuda_status(cudaDeviceSynchronize());
+    if (rc) return rc;
+    uint32_t w = 0;
+    rc = cuda_status(cudaMemcpyFromSymbol(&w, g_status, sizeof(w)));
+    if (rc) return rc;
+    if (clear) {
+        const uint32_t z = 0;
+        rc = cuda_status(cudaMemcpyToSymbol(g_status, &z, sizeof(z)));
+        if (rc) return rc;
+    }
+    if (word) *word = w;
+    return w ? INTFA_ERR_DEVICE_TIMEOUT : INTFA_OK;
+}

@@ -1,0 +1,32 @@
+// internal.h -- host-side helpers shared by the libintfa translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/intfa.h"
+
+namespace intfa {
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return INTFA_OK;
+    (void)cudaGetLastError();  // clear the sticky-free error so later calls are not poisoned
+    return INTFA_ERR_CUDA;
+}
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Launchers implemented in quantize.cu / attention.cu (arguments already checked).
+int launch_quantize_per_token(const void *x, int64_t rows, int d, int8_t *xq, float *scale,
+                              cudaStream_t stream);
+int launch_quantize_per_tensor(const void *x, int64_t groups, int64_t rows, int cols,
+                               int transpose, int8_t *xq, float *scale, void *workspace,
+                               cudaStream_t stream);
+int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt,
+                         const float *sQ, const float *sK, const float *sV, int B, int H, int L,
+                         int d, int causal, void *O, cudaStream_t stream);
+
+}  // namespace intfa

@@ -1,0 +1,293 @@
+// quantize.cu -- symmetric INT8 quantisation kernels (IntAttention: A Fully
+// Integer Attention Pipeline for Efficient Edge Inference, section 2.1,
+// eq. 3: s = max|x| / 127, x ~= s x_hat, zero-point 0), per token row for Q
+// and K (INT-FlashAttention, abstract: token-level quantisation) and per
+// L x d tensor for V.
+//
+// Both are HBM-bound streaming kernels: 16-byte vector loads of 8 fp16
+// values per thread, warp-shuffle row reductions, 8-byte code stores.
+//
+// Rounding contract (bit-exact with the definition): s = fl32(amax / 127)
+// by an IEEE division; the code is RNE(fl32(x / s)) clamped to +-127.  The
+// per-element quotient is formed as y = x * fl32(1 / s) (IEEE reciprocal):
+// |y - x/s| <= |x/s| 2^-23 <= 1.6e-5 and |fl32(x/s) - x/s| <= 7.6e-6, so y
+// and fl32(x/s) round to the same integer unless x/s lies within ~2.4e-5 of
+// a half-integer; when y is within 1e-3 of one, the IEEE quotient
+// __fdiv_rn(x, s) is used instead.  The result is therefore identical to
+// rounding the IEEE quotient, at one multiply per element.
+#include <cuda_fp16.h>
+
+#include "internal.h"
+
+namespace intfa {
+namespace {
+
+__device__ __forceinline__ int quant_code(float x, float s, float r) {
+    float y = x * r;
+    const float f = y - floorf(y);
+    if (fabsf(f - 0.5f) < 1e-3f) y = __fdiv_rn(x, s);
+    int c = __float2int_rn(y);
+    c = c > 127 ? 127 : c;
+    c = c < -127 ? -127 : c;
+    return c;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
+    const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __half22float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ float absmax8(const float (&f)[8]) {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+    return m;
+}
+
+__device__ __forceinline__ uint2 codes8(const float (&f)[8], float s, float r) {
+    uint32_t w[2] = {0u, 0u};
+    if (s != 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t c = static_cast<uint32_t>(quant_code(f[i], s, r)) & 0xFFu;
+            w[i >> 2] |= c << (8 * (i & 3));
+        }
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+// ------------------------------------------------------------ per token ---
+
+// G lanes cover one row of d = 8 G values; a warp holds 32 / G rows.
+template <int G>
+__global__ void __launch_bounds__(256) quant_per_token_kernel(const uint4 *__restrict__ x,
+                                                              int64_t rows,
+                                                              uint2 *__restrict__ xq,
+                                                              float *__restrict__ scale) {
+    const int lane = threadIdx.x & 31;
+    const int sub = lane & (G - 1);
+    constexpr int kRowsPerWarp = 32 / G;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t r0 = warp * kRowsPerWarp; r0 < rows; r0 += nwarps * kRowsPerWarp) {
+        const int64_t r = r0 + lane / G;
+        const bool valid = r < rows;
+        float f[8];
+        if (valid) {
+            const uint4 v = __ldcs(x + r * G + sub);
+            unpack8(v, f);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = 0.0f;
+        }
+        float amax = absmax8(f);
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        const float s = __fdiv_rn(amax, 127.0f);
+        const float rcp = s != 0.0f ? __frcp_rn(s) : 0.0f;
+        if (valid) {
+            __stcs(xq + r * G + sub, codes8(f, s, rcp));
+            if (sub == 0) scale[r] = s;
+        }
+    }
+}
+
+// ----------------------------------------------------------- per tensor ---
+
+// Phase 1: max |x| per group into ws[g] (fp32 bit pattern; atomicMax on the
+// unsigned bits orders non-negative floats correctly).  ws zeroed before.
+__global__ void __launch_bounds__(256) group_amax_kernel(const uint4 *__restrict__ x,
+                                                         int64_t n8, unsigned *__restrict__ ws) {
+    const int g = blockIdx.y;
+    const uint4 *xg = x + static_cast<int64_t>(g) * n8;
+    float m = 0.0f;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float f[8];
+        unpack8(__ldg(xg + i), f);
+        m = fmaxf(m, absmax8(f));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ float part[8];
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (blockDim.x >> 5); ++w) m = fmaxf(m, part[w]);
+        atomicMax(ws + g, __float_as_uint(m));
+    }
+}
+
+// Phase 2, same layout as the input.
+__global__ void __launch_bounds__(256) group_convert_kernel(const uint4 *__restrict__ x,
+                                                            int64_t n8,
+                                                            const unsigned *__restrict__ ws,
+                                                            uint2 *__restrict__ xq,
+                                                            float *__restrict__ scale) {
+    const int g = blockIdx.y;
+    const float s = __fdiv_rn(__uint_as_float(ws[g]), 127.0f);
+    const float rcp = s != 0.0f ? __frcp_rn(s) : 0.0f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) scale[g] = s;
+    const uint4 *xg = x + static_cast<int64_t>(g) * n8;
+    uint2 *qg = xq + static_cast<int64_t>(g) * n8;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float f[8];
+        unpack8(__ldcs(xg + i), f);
+        __stcs(qg + i, codes8(f, s, rcp));
+    }
+}
+
+// Phase 2, transposed: group g of [rows][cols] -> [cols][ld], 64 rows per
+// block staged through shared memory; rows in [rows, ld) get code 0.
+constexpr int kTRows = 64;
+__global__ void __launch_bounds__(256) group_convert_t_kernel(const uint4 *__restrict__ x,
+                                                              int64_t rows, int cols, int64_t ld,
+                                                              const unsigned *__restrict__ ws,
+                                                              int8_t *__restrict__ xq,
+                                                              float *__restrict__ scale) {
+    __shared__ __align__(16) uint8_t tile[256 * kTRows];  // [col][row]
+    const int g = blockIdx.y;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTRows;
+    const float s = __fdiv_rn(__uint_as_float(ws[g]), 127.0f);
+    const float rcp = s != 0.0f ? __frcp_rn(s) : 0.0f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) scale[g] = s;
+    const int c8n = cols >> 3;
+    const uint4 *xg = x + static_cast<int64_t>(g) * rows * c8n;
+    for (int i = threadIdx.x; i < kTRows * c8n; i += blockDim.x) {
+        const int row = i / c8n, c8 = i - row * c8n;
+        uint2 w = make_uint2(0u, 0u);
+        if (r0 + row < rows) {
+            float f[8];
+            unpack8(__ldcs(xg + (r0 + row) * c8n + c8), f);
+            w = codes8(f, s, rcp);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t word = e < 4 ? w.x : w.y;
+            tile[(c8 * 8 + e) * kTRows + row] = static_cast<uint8_t>(word >> (8 * (e & 3)));
+        }
+    }
+    __syncthreads();
+    int8_t *qg = xq + static_cast<int64_t>(g) * cols * ld;
+    for (int j = threadIdx.x; j < cols * (kTRows / 16); j += blockDim.x) {
+        const int c = j >> 2, part = j & 3;
+        const int64_t rr = r0 + part * 16;
+        if (rr < ld) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(tile + c * kTRows + part * 16);
+            __stcs(reinterpret_cast<uint4 *>(qg + c * ld + rr), v);
+        }
+    }
+}
+
+int grid_for(int64_t work_items, int per_block) {
+    int64_t blocks = (work_items + per_block - 1) / per_block;
+    const int64_t cap = 148 * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return static_cast<int>(blocks);
+}
+
+}  // namespace
+
+int launch_quantize_per_token(const void *x, int64_t rows, int d, int8_t *xq, float *scale,
+                              cudaStream_t stream) {
+    if (rows == 0) return INTFA_OK;
+    const uint4 *xv = static_cast<const uint4 *>(x);
+    uint2 *qv = reinterpret_cast<uint2 *>(xq);
+    const int rows_per_block = 256 / (d / 8);
+    const int grid = grid_for(rows, rows_per_block);
+    switch (d) {
+        case 8: quant_per_token_kernel<1><<<grid, 256, 0, stream>>>(xv, rows, qv, scale); break;
+        case 16: quant_per_token_kernel<2><<<grid, 256, 0, stream>>>(xv, rows, qv, scale); break;
+        case 32: quant_per_token_kernel<4><<<grid, 256, 0, stream>>>(xv, rows, qv, scale); break;
+        case 64: quant_per_token_kernel<8><<<grid, 256, 0, stream>>>(xv, rows, qv, scale); break;
+        case 128: quant_per_token_kernel<16><<<grid, 256, 0, stream>>>(xv, rows, qv, scale); break;
+        case 256: quant_per_token_kernel<32><<<grid, 256, 0, stream>>>(xv, rows, qv, scale); break;
+        default: return INTFA_ERR_UNSUPPORTED;
+    }
+    return cuda_status(cudaGetLastError());
+}
+
+int launch_quantize_per_tensor(const void *x, int64_t groups, int64_t rows, int cols,
+                               int transpose, int8_t *xq, float *scale, void *workspace,
+                               cudaStream_t stream) {
+    if (groups == 0) return INTFA_OK;
+    unsigned *ws = static_cast<unsigned *>(workspace);
+    int rc = cuda_status(cudaMemsetAsync(ws, 0, static_cast<size_t>(groups) * sizeof(unsigned), stream));
+    if (rc) return rc;
+    const int64_t n8 = rows * cols / 8;
+    const uint4 *xv = static_cast<const uint4 *>(x);
+    int chunks = static_cast<int>((148 * 8 + groups - 1) / groups);
+    const int64_t max_chunks = (n8 + 255) / 256;
+    if (chunks > max_chunks) chunks = static_cast<int>(max_chunks);
+    if (chunks < 1) chunks = 1;
+    group_amax_kernel<<<dim3(chunks, static_cast<unsigned>(groups)), 256, 0, stream>>>(xv, n8, ws);
+    rc = cuda_status(cudaGetLastError());
+    if (rc) return rc;
+    if (!transpose) {
+        int cb = static_cast<int>((n8 + 255) / 256);
+        const int cap = static_cast<int>((148 * 16 + groups - 1) / groups);
+        if (cb > cap) cb = cap;
+        if (cb < 1) cb = 1;
+        group_convert_kernel<<<dim3(cb, static_cast<unsigned>(groups)), 256, 0, stream>>>(
+            xv, n8, ws, reinterpret_cast<uint2 *>(xq), scale);
+    } else {
+        const int64_t ld = intfa_vt_ld(rows);
+        const unsigned tiles = static_cast<unsigned>((ld + kTRows - 1) / kTRows);
+        group_convert_t_kernel<<<dim3(tiles, static_cast<unsigned>(groups)), 256, 0, stream>>>(
+            xv, rows, cols, ld, ws, xq, scale);
+    }
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace intfa
+
+// ------------------------------------------------------------------ C ABI ---
+
+extern "C" int intfa_quantize_per_token(const void *x_f16, int64_t rows, int d, int8_t *x_q,
+                                        float *scale, void *stream) {
+    using namespace intfa;
+    if (rows < 0) return INTFA_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_f16 || !x_q || !scale)) return INTFA_ERR_INVALID_ARG;
+    if (!(d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256)) return INTFA_ERR_UNSUPPORTED;
+    if (rows > (INT64_MAX / 2) / d) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(x_f16) || (reinterpret_cast<uintptr_t>(x_q) & 7u) != 0 ||
+        (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return INTFA_ERR_MISALIGNED;
+    if (d >= 16 && !aligned16(x_q)) return INTFA_ERR_MISALIGNED;
+    return launch_quantize_per_token(x_f16, rows, d, x_q, scale, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t intfa_quantize_per_tensor_workspace_size(int64_t groups) {
+    if (groups <= 0) return 0;
+    return intfa::round_up(static_cast<size_t>(groups) * sizeof(unsigned), 256);
+}
+
+extern "C" int64_t intfa_vt_ld(int64_t rows) { return rows <= 0 ? 0 : (rows + 15) / 16 * 16; }
+
+extern "C" int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int64_t rows, int cols,
+                                         int transpose, int8_t *x_q, float *scale,
+                                         void *workspace, size_t workspace_bytes, void *stream) {
+    using namespace intfa;
+    if (groups < 0 || rows < 0 || cols <= 0) return INTFA_ERR_INVALID_ARG;
+    if (transpose != 0 && transpose != 1) return INTFA_ERR_INVALID_ARG;
+    if (cols % 8 != 0) return INTFA_ERR_UNSUPPORTED;
+    if (transpose && cols > 256) return INTFA_ERR_UNSUPPORTED;
+    if (groups == 0 || rows == 0) return INTFA_OK;
+    if (groups > 65535) return INTFA_ERR_UNSUPPORTED;
+    if (rows > (INT64_MAX / 4) / cols / groups) return INTFA_ERR_INVALID_ARG;
+    if (!x_f16 || !x_q || !scale) return INTFA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < intfa_quantize_per_tensor_workspace_size(groups))
+        return INTFA_ERR_WORKSPACE;
+    if (!aligned16(x_f16) || !aligned16(x_q) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return INTFA_ERR_MISALIGNED;
+    return launch_quantize_per_tensor(x_f16, groups, rows, cols, transpose, x_q, scale, workspace,
+                                      static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,215 @@
+"""Thin ctypes binding of libintfa (include/intfa.h), same names as the C ABI.
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+kernels of libintfa.so.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libintfa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "intfa.h")
+
+STATUS = {0: "INTFA_OK", 1: "INTFA_ERR_INVALID_ARG", 2: "INTFA_ERR_UNSUPPORTED",
+          3: "INTFA_ERR_MISALIGNED", 4: "INTFA_ERR_CUDA", 5: "INTFA_ERR_DEVICE_TIMEOUT",
+          6: "INTFA_ERR_WORKSPACE"}
+
+
+class IntfaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({status_string(code)})")
+
+
+_lib = None
+
+
+def lib():
+    """Load libintfa.so (built in-tree by ``build.build()``); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libintfa.so not built ({LIB_PATH}); run "
+                           "python -m int8_quantized_attention_token_b200.build")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "intfa_status_string": ([I], ctypes.c_char_p),
+        "intfa_quantize_per_token": ([P, I64, I, P, P, P], I),
+        "intfa_quantize_per_tensor_workspace_size": ([I64], SZ),
+        "intfa_vt_ld": ([I64], I64),
+        "intfa_quantize_per_tensor": ([P, I64, I64, I, I, P, P, P, SZ, P], I),
+        "intfa_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
+        "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
+        "intfa_forward_workspace_size": ([I, I, I, I], SZ),
+        "intfa_forward_workspace_layout": ([I, I, I, I, ctypes.POINTER(SZ)], I),
+        "intfa_forward": ([P, P, P, I, I, I, I, I, P, P, SZ, P], I),
+        "intfa_forward_host_workspace_size": ([I, I, I, I], SZ),
+        "intfa_forward_host": ([P, P, P, I, I, I, I, I, P, P, SZ, P], I),
+        "intfa_device_status": ([I, ctypes.POINTER(ctypes.c_uint32)], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def declared_symbols() -> list[str]:
+    """Entry points declared in include/intfa.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(intfa_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(code: int) -> str:
+    return lib().intfa_status_string(int(code)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise IntfaError(rc, what)
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t) -> int:
+    return t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ------------------------------------------------------------- entry points ---
+
+def intfa_vt_ld(rows: int) -> int:
+    return int(lib().intfa_vt_ld(int(rows)))
+
+
+def intfa_quantize_per_token(x: torch.Tensor, x_q=None, scale=None, stream=None):
+    """fp16 [..., d] -> (int8 [..., d], fp32 [...]); one scale per row."""
+    _need(x, torch.float16, "x")
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    x_q = torch.empty(x.shape, dtype=torch.int8, device=x.device) if x_q is None else x_q
+    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if scale is None else scale
+    _check(lib().intfa_quantize_per_token(_ptr(x), rows, d, _ptr(x_q), _ptr(scale), _stream(stream)),
+           "intfa_quantize_per_token")
+    return x_q, scale
+
+
+def intfa_quantize_per_tensor(x: torch.Tensor, transpose: bool = False, x_q=None, scale=None,
+                              workspace=None, stream=None):
+    """fp16 [groups, rows, cols] -> codes and fp32 [groups] scales.
+
+    transpose=False: int8 [groups, rows, cols]; transpose=True: int8
+    [groups, cols, intfa_vt_ld(rows)] (the V_hat^T layout of the attention)."""
+    _need(x, torch.float16, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [groups, rows, cols]")
+    g, rows, cols = x.shape
+    if x_q is None:
+        shape = (g, cols, intfa_vt_ld(rows)) if transpose else (g, rows, cols)
+        x_q = torch.empty(shape, dtype=torch.int8, device=x.device)
+    scale = torch.empty((g,), dtype=torch.float32, device=x.device) if scale is None else scale
+    wsb = int(lib().intfa_quantize_per_tensor_workspace_size(g))
+    if workspace is None:
+        workspace = torch.empty((max(wsb, 1),), dtype=torch.uint8, device=x.device)
+    _check(lib().intfa_quantize_per_tensor(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
+                                           _ptr(scale), _ptr(workspace), workspace.numel(),
+                                           _stream(stream)), "intfa_quantize_per_tensor")
+    return x_q, scale
+
+
+def intfa_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, O=None, stream=None):
+    """Q_q, K_q int8 [B, H, L, d]; Vt_q int8 [B, H, d, intfa_vt_ld(L)];
+    s_Q, s_K fp32 [B, H, L]; s_V fp32 [B, H]  ->  O fp16 [B, H, L, d]."""
+    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
+        _need(t, torch.int8, n)
+    for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
+        _need(t, torch.float32, n)
+    B, H, L, d = Q_q.shape
+    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
+    _check(lib().intfa_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
+                                     _ptr(s_V), B, H, L, d, int(bool(causal)), _ptr(O),
+                                     _stream(stream)), "intfa_attention_fwd")
+    return O
+
+
+def intfa_debug_qk(Q_q, K_q, S=None, stream=None):
+    """int32 [B, H, L, L] = Q_hat K_hat^T through the tensor-core path."""
+    _need(Q_q, torch.int8, "Q_q")
+    _need(K_q, torch.int8, "K_q")
+    B, H, L, d = Q_q.shape
+    S = torch.empty((B, H, L, L), dtype=torch.int32, device=Q_q.device) if S is None else S
+    _check(lib().intfa_debug_qk(_ptr(Q_q), _ptr(K_q), B, H, L, d, _ptr(S), _stream(stream)),
+           "intfa_debug_qk")
+    return S
+
+
+def intfa_forward_workspace_size(B, H, L, d) -> int:
+    return int(lib().intfa_forward_workspace_size(B, H, L, d))
+
+
+def intfa_forward_host_workspace_size(B, H, L, d) -> int:
+    return int(lib().intfa_forward_host_workspace_size(B, H, L, d))
+
+
+def intfa_forward_workspace_layout(B, H, L, d) -> list[int]:
+    off = (ctypes.c_size_t * 6)()
+    _check(lib().intfa_forward_workspace_layout(B, H, L, d, off), "intfa_forward_workspace_layout")
+    return list(off)
+
+
+def intfa_forward(Q, K, V, causal: bool, O=None, workspace=None, stream=None):
+    """fp16 [B, H, L, d] device tensors -> O fp16; quantisation + attention."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.float16, n)
+    B, H, L, d = Q.shape
+    O = torch.empty_like(Q) if O is None else O
+    wsb = intfa_forward_workspace_size(B, H, L, d)
+    if workspace is None:
+        workspace = torch.empty((max(wsb, 1),), dtype=torch.uint8, device=Q.device)
+    _check(lib().intfa_forward(_ptr(Q), _ptr(K), _ptr(V), B, H, L, d, int(bool(causal)), _ptr(O),
+                               _ptr(workspace), workspace.numel(), _stream(stream)), "intfa_forward")
+    return O
+
+
+def intfa_forward_host(Q_host, K_host, V_host, causal: bool, O_host, workspace, stream=None):
+    """Host (pinned) fp16 tensors in and out; copies run inside the call."""
+    for t, n in ((Q_host, "Q"), (K_host, "K"), (V_host, "V"), (O_host, "O")):
+        if t.is_cuda or t.dtype != torch.float16 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous fp16 host tensor")
+    B, H, L, d = Q_host.shape
+    _check(lib().intfa_forward_host(_ptr(Q_host), _ptr(K_host), _ptr(V_host), B, H, L, d,
+                                    int(bool(causal)), _ptr(O_host), _ptr(workspace),
+                                    workspace.numel(), _stream(stream)), "intfa_forward_host")
+    return O_host
+
+
+def intfa_device_status(clear: bool = True) -> int:
+    """Synchronise and return the device status word (0 = no kernel timed out)."""
+    w = ctypes.c_uint32(0)
+    rc = lib().intfa_device_status(int(bool(clear)), ctypes.byref(w))
+    if rc not in (0, 5):
+        raise IntfaError(rc, "intfa_device_status")
+    return int(w.value)

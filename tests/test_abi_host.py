@@ -1,0 +1,86 @@
+"""The C-ABI library on the host (no GPU needed): it loads, exports every
+entry point include/intfa.h declares, and rejects bad arguments before
+launching anything."""
+import ctypes
+
+import pytest
+
+from int8_quantized_attention_token_b200 import build, intfa
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return intfa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = intfa.declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert intfa.status_string(code) not in ("", "unknown status")
+    assert intfa.status_string(99) == "unknown status"
+
+
+def test_vt_ld_and_workspace_sizes(L):
+    assert [intfa.intfa_vt_ld(n) for n in (1, 15, 16, 17, 4096)] == [16, 16, 16, 32, 4096]
+    assert L.intfa_quantize_per_tensor_workspace_size(128) == 512
+    assert L.intfa_quantize_per_tensor_workspace_size(0) == 0
+    B, H, Lq, d = 4, 32, 4096, 128
+    ws = intfa.intfa_forward_workspace_size(B, H, Lq, d)
+    n = B * H * Lq
+    assert ws >= 3 * n * d + 2 * 4 * n
+    assert intfa.intfa_forward_host_workspace_size(B, H, Lq, d) >= ws + 4 * 2 * n * d
+    off = intfa.intfa_forward_workspace_layout(B, H, Lq, d)
+    assert off[0] == 0 and all(o % 256 == 0 for o in off) and sorted(off) == off
+    assert intfa.intfa_forward_workspace_size(1, 1, 128, 96) == 0
+
+
+FAKE = 1 << 20   # a 16-byte aligned non-null address; never dereferenced: every call fails its checks
+
+
+def test_quantize_per_token_rejects(L):
+    assert L.intfa_quantize_per_token(None, 0, 64, None, None, None) == 0        # empty: no-op
+    assert L.intfa_quantize_per_token(FAKE, -1, 64, FAKE, FAKE, None) == 1
+    assert L.intfa_quantize_per_token(None, 4, 64, FAKE, FAKE, None) == 1
+    assert L.intfa_quantize_per_token(FAKE, 4, 96, FAKE, FAKE, None) == 2
+    assert L.intfa_quantize_per_token(FAKE + 2, 4, 64, FAKE, FAKE, None) == 3
+    assert L.intfa_quantize_per_token(FAKE, 4, 64, FAKE + 8, FAKE, None) == 3
+
+
+def test_quantize_per_tensor_rejects(L):
+    ws = L.intfa_quantize_per_tensor_workspace_size(4)
+    assert L.intfa_quantize_per_tensor(FAKE, 4, 10, 64, 2, FAKE, FAKE, FAKE, ws, None) == 1
+    assert L.intfa_quantize_per_tensor(FAKE, 4, 10, 60, 0, FAKE, FAKE, FAKE, ws, None) == 2
+    assert L.intfa_quantize_per_tensor(FAKE, 4, 10, 512, 1, FAKE, FAKE, FAKE, ws, None) == 2
+    assert L.intfa_quantize_per_tensor(FAKE, 4, 10, 64, 0, FAKE, FAKE, None, ws, None) == 6
+    assert L.intfa_quantize_per_tensor(FAKE, 4, 10, 64, 0, FAKE, FAKE, FAKE, ws - 1, None) == 6
+    assert L.intfa_quantize_per_tensor(FAKE + 4, 4, 10, 64, 0, FAKE, FAKE, FAKE, ws, None) == 3
+    assert L.intfa_quantize_per_tensor(FAKE, 0, 10, 64, 0, None, None, None, 0, None) == 0
+
+
+def test_attention_rejects(L):
+    a = [FAKE] * 6
+    assert L.intfa_attention_fwd(*a, 1, 1, 128, 96, 0, FAKE, None) == 2           # d
+    assert L.intfa_attention_fwd(*a, 0, 1, 128, 64, 0, FAKE, None) == 1           # B
+    assert L.intfa_attention_fwd(*a, 1, 1, 0, 64, 0, FAKE, None) == 1             # L
+    assert L.intfa_attention_fwd(*a, 1, 1, 128, 64, 2, FAKE, None) == 1           # causal flag
+    assert L.intfa_attention_fwd(None, *a[1:], 1, 1, 128, 64, 0, FAKE, None) == 1
+    assert L.intfa_attention_fwd(*a, 1, 1, 128, 64, 0, FAKE + 8, None) == 3       # O alignment
+    assert L.intfa_attention_fwd(FAKE + 1, *a[1:], 1, 1, 128, 64, 0, FAKE, None) == 3
+    assert L.intfa_attention_fwd(*a, 1, 1, 300000, 64, 0, FAKE, None) == 2        # int32 bound
+    assert L.intfa_debug_qk(FAKE, FAKE, 1, 1, 128, 32, FAKE, None) == 2
+    assert L.intfa_debug_qk(FAKE, None, 1, 1, 128, 64, FAKE, None) == 1
+
+
+def test_forward_rejects(L):
+    assert L.intfa_forward(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, None, 0, None) == 6
+    ws = intfa.intfa_forward_workspace_size(1, 1, 128, 64)
+    assert L.intfa_forward(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, FAKE + 16, ws, None) == 3
+    assert L.intfa_forward(FAKE, FAKE, FAKE, 1, 1, 128, 80, 0, FAKE, FAKE, ws, None) == 2
+    assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, FAKE, ws, None) == 6

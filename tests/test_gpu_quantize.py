@@ -1,0 +1,74 @@
+"""GPU quantisers vs the CPU oracle, bit-exact (codes and fp32 scales)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int8_quantized_attention_token_b200 import intfa
+from int8_quantized_attention_token_b200.workloads import WORKLOADS, make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def special_rows(d):
+    rows = [np.zeros(d), np.full(d, 1e-7)]                   # zero row, fp16 subnormals
+    r = np.zeros(d); r[0] = 127.0; r[1:5] = [2.5, -3.5, 0.5, 1.5]; rows.append(r)   # s = 1: ties
+    r = np.zeros(d); r[0] = 63.5; r[1:4] = [1.25, -0.75, 0.25]; rows.append(r)     # s = 0.5
+    rows.append(np.linspace(-60000, 60000, d))               # near the fp16 maximum
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("d", [8, 16, 32, 64, 128, 256])
+@pytest.mark.parametrize("rows", [1, 7, 1000, 4099])
+def test_per_token_bit_exact(rows, d):
+    g = torch.Generator().manual_seed(rows * 1000 + d)
+    x = (torch.randn(rows, d, generator=g) * torch.rand(rows, 1, generator=g) * 10).half()
+    sp = torch.from_numpy(special_rows(d)).half()
+    x[: min(rows, sp.shape[0])] = sp[: min(rows, sp.shape[0])]
+    q, s = intfa.intfa_quantize_per_token(x.cuda())
+    qo, so = oracle.quantize_per_token(x.float().numpy())
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+def test_per_token_empty():
+    x = torch.empty(0, 64, dtype=torch.float16, device="cuda")
+    q, s = intfa.intfa_quantize_per_token(x)
+    assert q.numel() == 0 and s.numel() == 0
+
+
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("groups,rows,cols", [(1, 1, 64), (3, 129, 64), (4, 1000, 128), (2, 77, 8),
+                                              (5, 4096, 128), (1, 33, 256)])
+def test_per_tensor_bit_exact(groups, rows, cols, transpose):
+    g = torch.Generator().manual_seed(groups * 7 + rows + cols)
+    x = (torch.randn(groups, rows, cols, generator=g) * 3).half()
+    x[0, 0, 0] = 0.0
+    if groups > 1:
+        x[1] = 0.0                                            # an all-zero group
+    q, s = intfa.intfa_quantize_per_tensor(x.cuda(), transpose=transpose)
+    qo, so = oracle.quantize_per_tensor(x.float().numpy(), groups)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    q = q.cpu().numpy()
+    if transpose:
+        ld = intfa.intfa_vt_ld(rows)
+        assert q.shape == (groups, cols, ld)
+        np.testing.assert_array_equal(q[:, :, :rows].transpose(0, 2, 1), qo)
+        assert not q[:, :, rows:].any()                       # padding codes are zero
+    else:
+        np.testing.assert_array_equal(q, qo)
+
+
+@pytest.mark.parametrize("w", [WORKLOADS[2], WORKLOADS[3]], ids=lambda w: w.name)
+def test_full_size_quantisation_bit_exact(w):
+    Q, K, V = make_workload(w)
+    for X in (Q, K):
+        q, s = intfa.intfa_quantize_per_token(X.cuda())
+        qo, so = oracle.quantize_per_token(X.float().numpy())
+        np.testing.assert_array_equal(q.cpu().numpy(), qo)
+        np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    Vg = V.reshape(w.B * w.H, w.L, w.d)
+    q, s = intfa.intfa_quantize_per_tensor(Vg.cuda(), transpose=True)
+    qo, so = oracle.quantize_per_tensor(Vg.float().numpy(), w.B * w.H)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy()[:, :, : w.L].transpose(0, 2, 1), qo)
