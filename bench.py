@@ -1,0 +1,402 @@
+"""Benchmark of the INT8 attention forward hot path on B200.
+
+One step = the whole path on one batch of synthetic fp16 input already in HBM:
+per-token quantisation of Q and K, per-head quantisation of V (transposed),
+and the fused INT8 attention kernel.  The metric is INT8 attention TOPS:
+4 B H L^2 d ops (halved when causal) per step / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...    # the CPU oracle, timed on host cores
+
+N > 1 runs under torchrun, one rank per GPU, each rank the full workload on
+its own GPU (independent replicas: the path has no exchange step); the time
+is the max over ranks and the value the ops of all ranks over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "INT8 attention fwd TOPS and % of B200 dense INT8 tensor peak"
+UNIT = "TOPS"
+DEFAULT_WORKLOAD = "attn_B4_H32_L4096_d128_causal"
+# Nominal dense ratio INT8 : BF16 on B200 (4.5 POPS : 2.25 PFLOP/s).
+I8_PER_BF16 = 2.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "int8_quantized_attention_token_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            m = json.load(f)
+        return {"bf16_burst": float(m["bf16_tflops"]), "bf16_sustained": float(m["bf16_tflops_sustained"]),
+                "hbm_gbs": float(m["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"bf16_burst": FALLBACK_BF16_TFLOPS, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0,
+                "source": "fallback"}
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        e = t.get(workload)
+        if e and e.get("kernel_sha") == kernel_sources_sha():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms; only the
+    samples that arrive inside the timed window are kept."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.perf_counter(), line.strip()))
+
+    def stop(self, t_begin=None, t_end=None):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, ln in self.lines:
+            if t_begin is not None and not (t_begin <= ts <= t_end + 0.1):
+                continue
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- GPU arm ---
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from int8_quantized_attention_token_b200 import intfa
+    from int8_quantized_attention_token_b200.workloads import by_name, make_workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = by_name(args.workload)
+    B, H, L, d = w.B, w.H, w.L, w.d
+    Qh, Kh, Vh = make_workload(w)
+    Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
+    BH = B * H
+    ld = intfa.intfa_vt_ld(L)
+    Qq = torch.empty(B, H, L, d, dtype=torch.int8, device=dev)
+    Kq = torch.empty_like(Qq)
+    Vt = torch.empty(BH, d, ld, dtype=torch.int8, device=dev)
+    sQ = torch.empty(B, H, L, dtype=torch.float32, device=dev)
+    sK = torch.empty_like(sQ)
+    sV = torch.empty(BH, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, intfa.lib().intfa_quantize_per_tensor_workspace_size(BH)), dtype=torch.uint8, device=dev)
+    O = torch.empty(B, H, L, d, dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    V3 = V.reshape(BH, L, d)
+
+    def step(ev=None):
+        intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
+        intfa.intfa_quantize_per_token(K, Kq, sK, stream=stream)
+        intfa.intfa_quantize_per_tensor(V3, True, Vt, sV, ws, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        intfa.intfa_attention_fwd(Qq, Kq, Vt.reshape(B, H, d, ld), sQ, sK, sV.reshape(B, H), w.causal, O,
+                                  stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    kernels_per_step = 5  # quantise Q, quantise K, V abs-max, V convert, attention
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if intfa.intfa_device_status(clear=True) != 0:
+        raise RuntimeError("a kernel timed out during warm-up")
+
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    h0 = time.perf_counter()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(attn_ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    h1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.1)
+    clk = clocks.stop(h0, h1)
+    elapsed_ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
+    if intfa.intfa_device_status(clear=True) != 0:
+        raise RuntimeError("a kernel timed out during the timed region")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    ms_per_step = elapsed_ms / args.steps
+    value = w.ops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
+    attn_mean = sum(attn_ms) / len(attn_ms)
+    achieved = w.ops / (attn_mean * 1e-3) / 1e12
+    pk = peaks()
+    peak = pk["bf16_burst"] * I8_PER_BF16
+
+    # End to end through the host-buffer entry point: pinned fp16 in, fp16 out.
+    e2e = None
+    if not args.no_e2e:
+        Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
+        Op = torch.empty(B, H, L, d, dtype=torch.float16).pin_memory()
+        wsh = torch.empty(intfa.intfa_forward_host_workspace_size(B, H, L, d), dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            intfa.intfa_forward_host(Qp, Kp, Vp, w.causal, Op, wsh, stream=stream)
+        torch.cuda.synchronize(dev)
+        e_steps = max(3, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            intfa.intfa_forward_host(Qp, Kp, Vp, w.causal, Op, wsh, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        nbytes = B * H * L * d * 2
+        e2e = {"value": w.ops * world * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "steps": e_steps, "ms_per_step": e_ms / e_steps,
+               "api": "intfa_forward_host (pinned host fp16 Q/K/V in, O out)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+            "data": "synthetic (seeded N(0,1) fp16 Q/K/V)",
+            "config": {**w.as_dict(), "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (fp16 Q/K/V 3x128 MiB read per step)"},
+            "pct_of_int8_peak": round(100.0 * value / world / peak, 2),
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": round(achieved, 2),
+                         "peak": round(peak, 1), "unit": UNIT, "frac": round(achieved / peak, 4),
+                         "traffic": traffic_for(w.name),
+                         "peak_note": f"{pk['source']} bf16 burst {pk['bf16_burst']} TFLOP/s x {I8_PER_BF16} "
+                                      "(nominal dense INT8:BF16 ratio)",
+                         "frac_of_sustained": round(achieved / (pk["bf16_sustained"] * I8_PER_BF16), 4),
+                         "attn_ms": round(attn_mean, 5), "ops_per_launch": w.ops},
+            "kernels_ms_per_step": {"attention": round(attn_mean, 5),
+                                    "quantisation": round(ms_per_step - attn_mean, 5)},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
+            "clocks": clk, "kernel_sha": kernel_sources_sha(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------- CPU arm ---
+
+def oracle_sample(w, heads, threads=None):
+    """Run the oracle's whole path (quantise, block-wise online attention) on
+    `heads` full (b, h) heads of the workload; returns (seconds, ops, cores)."""
+    import numpy as np
+
+    import oracle
+    from int8_quantized_attention_token_b200.workloads import make_workload
+
+    cores = len(os.sched_getaffinity(0)) if threads is None else threads
+    oracle.set_threads(cores)
+    Q, K, V = make_workload(w)
+    t = 0.0
+    for (b, h) in heads:
+        q, k, v = (X[b, h].float().numpy() for X in (Q, K, V))
+        t0 = time.perf_counter()
+        Qq, sQ = oracle.quantize_per_token(q)
+        Kq, sK = oracle.quantize_per_token(k)
+        Vq, sV = oracle.quantize_per_tensor(v, 1)
+        oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), w.causal, 128)
+        t += time.perf_counter() - t0
+    ops = w.ops / (w.B * w.H) * len(heads)
+    return t, ops, oracle.get_threads()
+
+
+def cpu_baseline(w, budget_s=15.0):
+    t1, ops1, cores = oracle_sample(w, [(0, 0)])
+    n = max(1, min(w.B * w.H - 1, int(budget_s / max(t1, 1e-3)) - 1))
+    heads = [((i + 1) // w.H % w.B, (i + 1) % w.H) for i in range(n)]
+    t, ops, cores = oracle_sample(w, heads)
+    t += t1
+    ops += ops1
+    return {"value": round(ops / t / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n + 1} of {w.B * w.H} heads at full L={w.L} (quantise + online attention), "
+                      f"{t:.1f} s on {cores} threads"}
+
+
+def oracle_rows_step(w, head, rows, data):
+    """One reference step: the oracle's whole path for one head (quantise Q, K,
+    V; block-wise online attention) on a contiguous run of query rows.  Returns
+    (seconds, ops): ops = 4 d per visible (query, key) pair."""
+    import numpy as np
+
+    import oracle
+
+    Q, K, V = data
+    b, h = head
+    q, k, v = (X[b, h].float().numpy() for X in (Q, K, V))
+    t0 = time.perf_counter()
+    Qq, sQ = oracle.quantize_per_token(q)
+    Kq, sK = oracle.quantize_per_token(k)
+    Vq, sV = oracle.quantize_per_tensor(v, 1)
+    oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), w.causal, 128,
+                                 int(rows[0]), int(rows[-1]) + 1)
+    t = time.perf_counter() - t0
+    visible = (np.asarray(rows) + 1) if w.causal else np.full(len(rows), w.L)
+    return t, 4.0 * w.d * float(visible.sum())
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from int8_quantized_attention_token_b200.workloads import by_name, make_workload
+    w = by_name(args.workload)
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    data = make_workload(w)
+    heads = [(i // w.H % w.B, i % w.H) for i in range(w.B * w.H)]
+    rng = np.random.default_rng(0)
+    # size each step so that the whole run takes about args.ref_seconds
+    cal = min(w.L, 256)
+    t_cal, _ = oracle_rows_step(w, heads[0], np.arange(w.L - cal, w.L), data)
+    per_row = t_cal / cal
+    n_rows = int(max(1, min(w.L, args.ref_seconds / max(args.steps, 1) / max(per_row, 1e-6))))
+    tt, ops_total = 0.0, 0.0
+    for i in range(args.steps):
+        r0 = int(rng.integers(0, w.L - n_rows + 1))
+        rows = np.arange(r0, r0 + n_rows)
+        t, ops = oracle_rows_step(w, heads[i % len(heads)], rows, data)
+        tt += t
+        ops_total += ops
+    value = ops_total / tt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tt / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) fp16 Q/K/V)", "config": w.as_dict(),
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle.get_threads(),
+                             "kind": "oracle",
+                             "sample": f"per step: one head of the workload quantised, {n_rows} consecutive query "
+                                       f"rows (random start) of it through the block-wise online attention; {args.steps} steps, "
+                                       f"{tt:.1f} s"},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="libintfa", choices=["libintfa", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl != "reference":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

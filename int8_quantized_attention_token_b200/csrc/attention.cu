@@ -51,6 +51,12 @@ constexpr int kThreads = 320;                 // 10 warps
 constexpr int kTmemCols = 512;
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
+// 1.5 * 2^23: for an integer |n| < 2^22, the fp32 bit pattern 0x4B400000 + n
+// is exactly the value 1.5 * 2^23 + n, so n -> float is one integer add and one
+// float subtract; and for 0 <= y < 2^22, fl(y + 1.5 * 2^23) holds RNE(y) in its
+// low mantissa bits.
+constexpr float kMagic = 12582912.0f;
+constexpr uint32_t kMagicBits = 0x4B400000u;
 
 // -------------------------------------------------------- bounded waits ---
 
@@ -136,9 +142,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = tid & 31;
 
     const int ntiles = (L + BM - 1) / BM;
-    const int t = blockIdx.x / BH;
-    const int bh = blockIdx.x - t * BH;
-    const int qt = causal ? (ntiles - 1 - t) : t;    // heaviest causal tiles first
+    // Head-major order: the CTAs resident together mostly share one head's
+    // K_hat / V_hat, which then stay in L2; within a head the heaviest causal
+    // tiles go first.
+    const int bh = blockIdx.x / ntiles;
+    const int t = blockIdx.x - bh * ntiles;
+    const int qt = causal ? (ntiles - 1 - t) : t;
     const int q0 = qt * BM;
     const int nb = causal ? (qt + 1) : (L + BN - 1) / BN;
     volatile int *abort_flag = &sm.abort_flag;
@@ -267,8 +276,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = tid;
         const int qi = q0 + row;
         const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
-        const float c = (qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
-                        (kLog2e / sqrtf(static_cast<float>(D)));
+        // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c * (S_ij s_K[j]).
+        // Clamped to a tiny positive value: a zero Q row then still maps masked
+        // keys (v = -inf) to p = 0 and visible keys to p = 1.
+        const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
+                                  (kLog2e / sqrtf(static_cast<float>(D))),
+                              1e-30f);
+        const uint64_t c2 = f2_pack(c, c);
+        const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
+        const uint64_t k127 = f2_pack(127.0f, 127.0f);
+        const uint64_t mag2 = f2_pack(kMagic, kMagic);
         float m_old = -INFINITY, l = 0.0f;
         for (int j = 0; j < nb; ++j) {
             const int b = j & 1, st = j % NS;
@@ -276,17 +293,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             // s_K of this block: published by the producer's release-arrive
             if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 12)) break;
             tc_fence_after();
-            uint32_t sr[BN];
-#pragma unroll
-            for (int ch = 0; ch < BN / 32; ++ch)
-                tmem_ld32(tS + lane_off + b * BN + 32 * ch,
-                          *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * ch]));
-            tmem_wait_ld();
+            // v_j = fl(S_ij s_K[j]) exactly as an fp32 product: the int32 S is
+            // turned into fp32 by the magic-number add (|S| <= 127^2 d < 2^22).
             float v[BN];
-            const float *skp = sm.sk[st];
+            {
+                uint32_t sr[BN];
 #pragma unroll
-            for (int jj = 0; jj < BN; ++jj)
-                v[jj] = static_cast<float>(static_cast<int32_t>(sr[jj])) * skp[jj];
+                for (int ch = 0; ch < BN / 32; ++ch)
+                    tmem_ld32(tS + lane_off + b * BN + 32 * ch,
+                              *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * ch]));
+                tmem_wait_ld();
+                const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
+#pragma unroll
+                for (int q = 0; q < BN / 4; ++q) {
+                    const float4 k4 = sk4[q];
+                    uint64_t a = f2_pack(__uint_as_float(sr[4 * q] + kMagicBits),
+                                         __uint_as_float(sr[4 * q + 1] + kMagicBits));
+                    uint64_t e = f2_pack(__uint_as_float(sr[4 * q + 2] + kMagicBits),
+                                         __uint_as_float(sr[4 * q + 3] + kMagicBits));
+                    a = fmul2(fadd2(a, negC2), f2_pack(k4.x, k4.y));
+                    e = fmul2(fadd2(e, negC2), f2_pack(k4.z, k4.w));
+                    f2_unpack(a, v[4 * q], v[4 * q + 1]);
+                    f2_unpack(e, v[4 * q + 2], v[4 * q + 3]);
+                }
+            }
             const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
             if (need_mask) {
 #pragma unroll
@@ -296,27 +326,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
-            float bm = -INFINITY;
+            float mx[8];
 #pragma unroll
-            for (int jj = 0; jj < BN; ++jj) bm = fmaxf(bm, v[jj]);
+            for (int i = 0; i < 8; ++i) mx[i] = v[i];
+#pragma unroll
+            for (int jj = 8; jj < BN; jj += 16) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], v[jj + i], v[jj + 8 + i]);
+            }
+            const float bm = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             const float m_new = fmaxf(m_old, bm);
-            const float alpha = (m_old == -INFINITY) ? 0.0f : exp2f(c * (m_old - m_new));
-            const float cm = c * m_new;
-            float ps = 0.0f;
+            const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
+            const uint64_t ncm2 = f2_pack(-c * m_new, -c * m_new);
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[32];
 #pragma unroll
-            for (int w = 0; w < 32; ++w) {
-                uint32_t word = 0;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x = v[4 * w + e];
-                    const float p = (x == -INFINITY) ? 0.0f : exp2f(fmaf(x, c, -cm));
-                    ps += p;
-                    const uint32_t code = static_cast<uint32_t>(__float2int_rn(p * 127.0f));
-                    word |= code << (8 * e);
-                }
-                pk[w] = word;
+            for (int q = 0; q < 32; ++q) {
+                const uint64_t x01 = ffma2(f2_pack(v[4 * q], v[4 * q + 1]), c2, ncm2);
+                const uint64_t x23 = ffma2(f2_pack(v[4 * q + 2], v[4 * q + 3]), c2, ncm2);
+                float x0, x1, x2, x3;
+                f2_unpack(x01, x0, x1);
+                f2_unpack(x23, x2, x3);
+                const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
+                const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
+                acc[q & 3] = fadd2(acc[q & 3], fadd2(p01, p23));
+                // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
+                float t0, t1, t2, t3;
+                f2_unpack(ffma2(p01, k127, mag2), t0, t1);
+                f2_unpack(ffma2(p23, k127, mag2), t2, t3);
+                pk[q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
+                             prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
             }
+            float s0, s1, s2, s3, s4, s5, s6, s7;
+            f2_unpack(acc[0], s0, s1);
+            f2_unpack(acc[1], s2, s3);
+            f2_unpack(acc[2], s4, s5);
+            f2_unpack(acc[3], s6, s7);
+            const float ps = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
             l = l * alpha + ps;
             tmem_st32(tS + lane_off + b * BN, pk);
             tmem_wait_st();
@@ -334,9 +380,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = tid - 128;
         const int qi = q0 + row;
         const uint32_t lane_off = static_cast<uint32_t>(32 * (warp - 4)) << 16;
-        float o[D];
+        const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
+        uint64_t o2[D / 2];   // the output row as fp32 pairs
 #pragma unroll
-        for (int c = 0; c < D; ++c) o[c] = 0.0f;
+        for (int c = 0; c < D / 2; ++c) o2[c] = 0ull;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
             const int b = j & 1;
@@ -344,15 +391,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&sm.a_full[b], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
             tc_fence_after();
             const float alpha = sm.alpha[b][row];
+            const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t r[32];
                 tmem_ld32(tO + lane_off + 32 * ch, r);
                 tmem_wait_ld();
+                // int32 P V block -> fp32 exactly (|x| <= 127^2 128 < 2^22), then
+                // o = alpha o + x on pairs.
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    o[32 * ch + c] = fmaf(o[32 * ch + c], alpha,
-                                          static_cast<float>(static_cast<int32_t>(r[c])));
+                for (int i = 0; i < 16; ++i) {
+                    const uint64_t x = fadd2(f2_pack(__uint_as_float(r[2 * i] + kMagicBits),
+                                                     __uint_as_float(r[2 * i + 1] + kMagicBits)),
+                                             negC2);
+                    o2[16 * ch + i] = ffma2(o2[16 * ch + i], a2, x);
+                }
             }
             tc_fence_before();
             mbar_arrive(&sm.o_empty);
@@ -367,8 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint4 w;
                 __half2 *h = reinterpret_cast<__half2 *>(&w);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    h[e] = __floats2half2_rn(o[8 * c8 + 2 * e] * f, o[8 * c8 + 2 * e + 1] * f);
+                for (int e = 0; e < 4; ++e) {
+                    float lo, hi;
+                    f2_unpack(o2[4 * c8 + e], lo, hi);
+                    h[e] = __floats2half2_rn(lo * f, hi * f);
+                }
                 dst[c8] = w;
             }
         }
