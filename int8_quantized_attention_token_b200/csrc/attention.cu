@@ -13,21 +13,32 @@
 //   O_i   = s_V acc_i / (127 l_i)                          -> fp16
 // exp is evaluated as exp2 with log2(e) folded into the per-row constant.
 //
-// B200 design (one CTA per 128-query tile of one (b, h)):
+// B200 design (one CTA per 128-query tile of one (b, h); 12 warps):
 //   warp 8      TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
 //               block's s_K values into a 3-stage shared-memory ring.
 //   warp 9      tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
 //               kind::i8 into one of two TMEM S buffers; P V with the P codes
 //               read straight from TMEM (aliasing the first 32 columns of the
 //               S buffer they came from) into a TMEM O block; owns the TMEM
-//               allocation (512 columns: S0, S1, O).
-//   warps 0-3   softmax: one thread per query row; reads its S row from
-//               TMEM, runs the online max / sum, writes the row's 128 P codes
-//               back to TMEM as the A operand of P V, and hands alpha to the
-//               correction warps through shared memory.
-//   warps 4-7   correction: one thread per query row; keeps the fp32 output
-//               row in registers, folds each int32 P V block in with alpha,
-//               and writes the normalised fp16 row at the end.
+//               allocation (512 columns: S0, S1, the int32 P V block and
+//               the fp32 output accumulator).
+//   warps 4-7   "prep" (one thread per query row): S row -> v = S s_K in
+//               fp32 (written back over S in TMEM), causal / ragged mask,
+//               running max m and alpha; then the output side: folds each
+//               int32 P V block into the row's fp32 accumulator in TMEM
+//               (o = alpha o + block) and writes the normalised fp16 row at
+//               the end.
+//   warps 0-3   "exp" (one thread per query row, same TMEM lanes as the prep
+//               warp on its SM sub-partition): reads v in 32-column chunks,
+//               p = 2^(c v - c m), the row sum, and the P codes, which it
+//               writes back to TMEM as the A operand of P V.
+//   warps 10-11 idle.
+// All per-row loops walk the row in 32-column chunks (one TMEM load each) and
+// are not unrolled across chunks, which keeps the three code paths that share
+// an SM sub-partition small enough for its instruction cache.
+// The exp warps are bound by the special-function unit (one exp2 per score);
+// the prep warps' integer/FMA work for block j+1 and the output update for
+// block j-1 run beside it on the same sub-partitions.
 // Every wait is bounded (clock-based); a timeout records a status word,
 // raises a CTA-wide abort flag, drains in-flight copies and MMAs, frees TMEM
 // and returns.
@@ -47,7 +58,10 @@ namespace {
 constexpr int BM = 128;                       // query rows per CTA
 constexpr int BN = 128;                       // keys per block
 constexpr int NS = 3;                         // K/V ring depth
-constexpr int kThreads = 320;                 // 10 warps
+constexpr int kThreads = 384;                 // 12 warps = 3 warpgroups
+// Warp roles inside the third warpgroup (warps 8-11).
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kTmemCols = 512;
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
@@ -60,11 +74,14 @@ constexpr uint32_t kMagicBits = 0x4B400000u;
 
 // -------------------------------------------------------- bounded waits ---
 
+// A waiting thread sleeps inside try_wait (suspend-time hint) between probes.
+constexpr uint32_t kSleepNs = 1000000;
+
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                          uint32_t site) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, kSleepNs)) {
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitCycles) {
             *abort_flag = 1;
@@ -85,7 +102,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, kSleepNs)) {
         if (clock64() - t0 > kWaitCycles) {
             atomicCAS(&g_status, 0u, 0x1FFu);
             return;
@@ -101,13 +118,13 @@ struct alignas(1024) AttnSmem {
     uint8_t k[NS][BN * D];      // K_hat tiles
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
-    float alpha[2][BM];         // softmax -> correction
-    float lsum[BM];             // final row sums
+    float2 cm_alpha[2][BM];     // prep -> exp: (c m_new, alpha) per row and S buffer
+    float lsum[BM];             // exp -> prep: final row sums
     uint64_t q_full;
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
     uint64_t s_full[2], p_full[2];
+    uint64_t x_full[2][4];      // prep warp k -> exp warp k (same TMEM lane quadrant)
     uint64_t o_full, o_empty;
-    uint64_t a_full[2], a_empty[2];
     uint64_t l_full, mma_drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -121,11 +138,18 @@ constexpr size_t attn_smem_bytes() {
     return s < 120 * 1024 ? 120 * 1024 : s;
 }
 
+// Dynamic shared memory rounded up to 1024 B by pointer arithmetic on the
+// __shared__ array itself, so that the compiler keeps every access in the
+// shared state space (an integer round trip would make them generic).
+__device__ __forceinline__ uint8_t *smem_aligned_1024() {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t off = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    return smem_raw + off;
+}
+
 template <int D>
 __device__ __forceinline__ AttnSmem<D> &get_smem() {
-    extern __shared__ uint8_t smem_raw[];
-    const uintptr_t p = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
-    return *reinterpret_cast<AttnSmem<D> *>(p);
+    return *reinterpret_cast<AttnSmem<D> *>(smem_aligned_1024());
 }
 
 // ---------------------------------------------------------------- kernel ---
@@ -161,9 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
+            for (int k = 0; k < 4; ++k) mbar_init(&sm.x_full[b][k], 32);
             mbar_init(&sm.p_full[b], BM);
-            mbar_init(&sm.a_full[b], BM);
-            mbar_init(&sm.a_empty[b], BM);
         }
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.o_empty, BM);
@@ -172,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -181,9 +204,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
     const uint32_t tS = tbase;          // S0 at column 0, S1 at column 128
-    const uint32_t tO = tbase + 256;    // O block, D columns
+    const uint32_t tO = tbase + 256;    // int32 P V block, D columns
+    const uint32_t tA = tO + D;         // fp32 output accumulator, D columns
 
-    if (warp == 8) {
+    if (warp >= 8) {
+      if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ---
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -223,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             drain_wait(&sm.v_full[s], (last / NS) & 1);
         }
         __syncwarp();
-    } else if (warp == 9) {
+      } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer ---
         constexpr uint32_t kSwQK = (D == 128) ? kSwizzle128B : kSwizzle64B;
         constexpr uint32_t kSboQK = 8 * D;      // 8 rows of D bytes
@@ -271,91 +296,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         drain_wait(&sm.mma_drain, 0);
         __syncwarp();
+      }
+      // the other two warps of this warpgroup have no role
     } else if (warp < 4) {
-        // --------------------------------------------------- softmax ---
+        // ------------------------------------------------------- exp ---
         const int row = tid;
-        const int qi = q0 + row;
         const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
-        // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c * (S_ij s_K[j]).
-        // Clamped to a tiny positive value: a zero Q row then still maps masked
-        // keys (v = -inf) to p = 0 and visible keys to p = 1.
+        const int qi = q0 + row;
+        // c = s_Q[i] log2(e) / sqrt(d) (see the prep warps for the clamp)
         const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
                                   (kLog2e / sqrtf(static_cast<float>(D))),
                               1e-30f);
         const uint64_t c2 = f2_pack(c, c);
-        const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
         const uint64_t k127 = f2_pack(127.0f, 127.0f);
         const uint64_t mag2 = f2_pack(kMagic, kMagic);
-        float m_old = -INFINITY, l = 0.0f;
+        float l = 0.0f;
         for (int j = 0; j < nb; ++j) {
-            const int b = j & 1, st = j % NS;
-            if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, abort_flag, 7)) break;
-            // s_K of this block: published by the producer's release-arrive
-            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 12)) break;
+            const int b = j & 1;
+            if (!warp_wait(&sm.x_full[b][warp], (j >> 1) & 1, abort_flag, 7)) break;
             tc_fence_after();
-            // v_j = fl(S_ij s_K[j]) exactly as an fp32 product: the int32 S is
-            // turned into fp32 by the magic-number add (|S| <= 127^2 d < 2^22).
-            float v[BN];
-            {
-                uint32_t sr[BN];
-#pragma unroll
-                for (int ch = 0; ch < BN / 32; ++ch)
-                    tmem_ld32(tS + lane_off + b * BN + 32 * ch,
-                              *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * ch]));
-                tmem_wait_ld();
-                const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
-#pragma unroll
-                for (int q = 0; q < BN / 4; ++q) {
-                    const float4 k4 = sk4[q];
-                    uint64_t a = f2_pack(__uint_as_float(sr[4 * q] + kMagicBits),
-                                         __uint_as_float(sr[4 * q + 1] + kMagicBits));
-                    uint64_t e = f2_pack(__uint_as_float(sr[4 * q + 2] + kMagicBits),
-                                         __uint_as_float(sr[4 * q + 3] + kMagicBits));
-                    a = fmul2(fadd2(a, negC2), f2_pack(k4.x, k4.y));
-                    e = fmul2(fadd2(e, negC2), f2_pack(k4.z, k4.w));
-                    f2_unpack(a, v[4 * q], v[4 * q + 1]);
-                    f2_unpack(e, v[4 * q + 2], v[4 * q + 3]);
-                }
-            }
-            const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
-            if (need_mask) {
-#pragma unroll
-                for (int jj = 0; jj < BN; ++jj) {
-                    const int key = j * BN + jj;
-                    if (key >= L || (causal && key > qi)) v[jj] = -INFINITY;
-                }
-            }
-            mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
-            float mx[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = v[i];
-#pragma unroll
-            for (int jj = 8; jj < BN; jj += 16) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], v[jj + i], v[jj + 8 + i]);
-            }
-            const float bm = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-            const float m_new = fmaxf(m_old, bm);
-            const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
-            const uint64_t ncm2 = f2_pack(-c * m_new, -c * m_new);
+            const float2 ca = sm.cm_alpha[b][row];
+            const uint64_t ncm2 = f2_pack(-ca.x, -ca.x);
+            const uint32_t tv = tS + lane_off + b * BN;
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-            uint32_t pk[32];
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t w[32];
+                tmem_ld32(tv + 32 * ch, w);
+                tmem_wait_ld();
+                uint32_t pk[8];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const uint64_t x01 = ffma2(f2_pack(v[4 * q], v[4 * q + 1]), c2, ncm2);
-                const uint64_t x23 = ffma2(f2_pack(v[4 * q + 2], v[4 * q + 3]), c2, ncm2);
-                float x0, x1, x2, x3;
-                f2_unpack(x01, x0, x1);
-                f2_unpack(x23, x2, x3);
-                const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
-                const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
-                acc[q & 3] = fadd2(acc[q & 3], fadd2(p01, p23));
-                // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
-                float t0, t1, t2, t3;
-                f2_unpack(ffma2(p01, k127, mag2), t0, t1);
-                f2_unpack(ffma2(p23, k127, mag2), t2, t3);
-                pk[q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
-                             prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
+                for (int q = 0; q < 8; ++q) {
+                    // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
+                    float x0, x1, x2, x3;
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), c2, ncm2), x0, x1);
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2, ncm2), x2, x3);
+                    const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
+                    const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
+                    acc[q & 3] = fadd2(acc[q & 3], fadd2(p01, p23));
+                    // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
+                    float t0, t1, t2, t3;
+                    f2_unpack(ffma2(p01, k127, mag2), t0, t1);
+                    f2_unpack(ffma2(p23, k127, mag2), t2, t3);
+                    pk[q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
+                                 prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
+                }
+                // codes of keys 32 ch .. 32 ch + 31 -> columns 8 ch .. 8 ch + 7,
+                // which this thread has already read (chunk 0 is columns 0..31)
+                tmem_st8(tv + 8 * ch, pk);
             }
             float s0, s1, s2, s3, s4, s5, s6, s7;
             f2_unpack(acc[0], s0, s1);
@@ -363,76 +351,159 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_unpack(acc[2], s4, s5);
             f2_unpack(acc[3], s6, s7);
             const float ps = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-            l = l * alpha + ps;
-            tmem_st32(tS + lane_off + b * BN, pk);
+            l = l * ca.y + ps;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
-            if (j >= 2 && !warp_wait(&sm.a_empty[b], ((j >> 1) - 1) & 1, abort_flag, 8)) break;
-            sm.alpha[b][row] = alpha;
-            mbar_arrive(&sm.a_full[b]);
-            m_old = m_new;
         }
         sm.lsum[row] = l;
         mbar_arrive(&sm.l_full);
     } else {
-        // ------------------------------------------------ correction ---
+        // ------------------------------------------------------ prep ---
         const int row = tid - 128;
         const int qi = q0 + row;
         const uint32_t lane_off = static_cast<uint32_t>(32 * (warp - 4)) << 16;
+        // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c (S_ij s_K[j]).
+        // Clamped to a tiny positive value: a zero Q row then still maps masked
+        // keys (v = -inf) to p = 0 and visible keys to p = 1.
+        const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
+                                  (kLog2e / sqrtf(static_cast<float>(D))),
+                              1e-30f);
         const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
-        uint64_t o2[D / 2];   // the output row as fp32 pairs
+        {
+            // the fp32 output accumulator starts at zero
+            uint32_t z[32];
 #pragma unroll
-        for (int c = 0; c < D / 2; ++c) o2[c] = 0ull;
-        bool ok = true;
-        for (int j = 0; j < nb; ++j) {
-            const int b = j & 1;
-            if (!warp_wait(&sm.o_full, j & 1, abort_flag, 9)) { ok = false; break; }
-            if (!warp_wait(&sm.a_full[b], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
-            tc_fence_after();
-            const float alpha = sm.alpha[b][row];
-            const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(tO + lane_off + 32 * ch, r);
-                tmem_wait_ld();
-                // int32 P V block -> fp32 exactly (|x| <= 127^2 128 < 2^22), then
-                // o = alpha o + x on pairs.
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = fadd2(f2_pack(__uint_as_float(r[2 * i] + kMagicBits),
-                                                     __uint_as_float(r[2 * i + 1] + kMagicBits)),
-                                             negC2);
-                    o2[16 * ch + i] = ffma2(o2[16 * ch + i], a2, x);
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&sm.o_empty);
-            mbar_arrive(&sm.a_empty[b]);
+            for (int i = 0; i < 32; ++i) z[i] = 0u;
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) tmem_st32(tA + lane_off + 32 * ch, z);
+            tmem_wait_st();
         }
-        if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11) && qi < L) {
+        float m_old = -INFINITY;
+        float alpha_prev = 0.0f;   // alpha of the block whose P V is folded next
+        bool ok = true;
+        for (int j = 0; ok && j <= nb; ++j) {
+            float alpha_cur = 0.0f;
+            if (j < nb) {
+                // -- block j: v = fl(S s_K) (exact int32 -> fp32 by the
+                // magic-number add, |S| <= 127^2 d < 2^22), mask, row max.
+                const int b = j & 1, st = j % NS;
+                if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, abort_flag, 12)) { ok = false; break; }
+                // s_K of this block: published by the producer's release-arrive
+                if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 13)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t ts = tS + lane_off + b * BN;
+                const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
+                const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    uint32_t w[32];
+                    tmem_ld32(ts + 32 * ch, w);
+                    tmem_wait_ld();
+                    float vv[32];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 k4 = sk4[8 * ch + q];
+                        const uint64_t a = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q] + kMagicBits),
+                                                               __uint_as_float(w[4 * q + 1] + kMagicBits)),
+                                                       negC2),
+                                                 f2_pack(k4.x, k4.y));
+                        const uint64_t e = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q + 2] + kMagicBits),
+                                                               __uint_as_float(w[4 * q + 3] + kMagicBits)),
+                                                       negC2),
+                                                 f2_pack(k4.z, k4.w));
+                        f2_unpack(a, vv[4 * q], vv[4 * q + 1]);
+                        f2_unpack(e, vv[4 * q + 2], vv[4 * q + 3]);
+                    }
+                    if (need_mask) {
+                        // keys past the end of the sequence, or after the query
+                        // (causal), get v = -inf (p = 0)
+                        const int lim = causal ? min(L, qi + 1) : L;
+                        const int key0 = j * BN + 32 * ch;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (key0 + e >= lim) vv[e] = -INFINITY;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        mx[q & 3] = fmax3(mx[q & 3], fmaxf(vv[4 * q], vv[4 * q + 1]), fmaxf(vv[4 * q + 2], vv[4 * q + 3]));
+                        w[4 * q] = __float_as_uint(vv[4 * q]);
+                        w[4 * q + 1] = __float_as_uint(vv[4 * q + 1]);
+                        w[4 * q + 2] = __float_as_uint(vv[4 * q + 2]);
+                        w[4 * q + 3] = __float_as_uint(vv[4 * q + 3]);
+                    }
+                    tmem_st32(ts + 32 * ch, w);
+                }
+                mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
+                const float m_new = fmaxf(m_old, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
+                alpha_cur = ex2(c * (m_old - m_new));   // 0 for the first block
+                m_old = m_new;
+                sm.cm_alpha[b][row] = make_float2(c * m_new, alpha_cur);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.x_full[b][warp - 4]);
+            }
+            if (j >= 1) {
+                // -- output side of block j - 1: acc = alpha acc + (P V block),
+                // the int32 block turned into fp32 exactly (|x| <= 127^2 128 < 2^22).
+                if (!warp_wait(&sm.o_full, (j - 1) & 1, abort_flag, 9)) { ok = false; break; }
+                tc_fence_after();
+                const uint64_t a2 = f2_pack(alpha_prev, alpha_prev);
+#pragma unroll 1
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t w[32], o[32];
+                    tmem_ld32(tO + lane_off + 32 * ch, w);
+                    tmem_ld32(tA + lane_off + 32 * ch, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const uint64_t x = fadd2(f2_pack(__uint_as_float(w[2 * i] + kMagicBits),
+                                                         __uint_as_float(w[2 * i + 1] + kMagicBits)),
+                                                 negC2);
+                        float lo, hi;
+                        f2_unpack(ffma2(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2, x),
+                                  lo, hi);
+                        o[2 * i] = __float_as_uint(lo);
+                        o[2 * i + 1] = __float_as_uint(hi);
+                    }
+                    tmem_st32(tA + lane_off + 32 * ch, o);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.o_empty);
+            }
+            alpha_prev = alpha_cur;
+        }
+        if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11)) {
+            tc_fence_after();
             const float l = sm.lsum[row];
             const float f = __ldg(sV + bh) / (127.0f * l);
             uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(bh) * L + qi) * D);
+#pragma unroll 1
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(tA + lane_off + 32 * ch, o);
+                tmem_wait_ld();
+                if (qi < L) {
 #pragma unroll
-            for (int c8 = 0; c8 < D / 8; ++c8) {
-                uint4 w;
-                __half2 *h = reinterpret_cast<__half2 *>(&w);
+                    for (int c8 = 0; c8 < 4; ++c8) {
+                        uint4 w;
+                        __half2 *h = reinterpret_cast<__half2 *>(&w);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float lo, hi;
-                    f2_unpack(o2[4 * c8 + e], lo, hi);
-                    h[e] = __floats2half2_rn(lo * f, hi * f);
+                        for (int e = 0; e < 4; ++e)
+                            h[e] = __floats2half2_rn(__uint_as_float(o[8 * c8 + 2 * e]) * f,
+                                                     __uint_as_float(o[8 * c8 + 2 * e + 1]) * f);
+                        dst[4 * ch + c8] = w;
+                    }
                 }
-                dst[c8] = w;
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
     }
@@ -453,9 +524,7 @@ template <int D>
 __global__ void __launch_bounds__(128, 1)
     debug_qk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     int L, int32_t *__restrict__ S) {
-    extern __shared__ uint8_t smem_raw[];
-    QKSmem<D> &sm = *reinterpret_cast<QKSmem<D> *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    QKSmem<D> &sm = *reinterpret_cast<QKSmem<D> *>(smem_aligned_1024());
     const int tid = threadIdx.x, warp = tid >> 5;
     const int q0 = blockIdx.x * BM, k0 = blockIdx.y * BN, bh = blockIdx.z;
     volatile int *abort_flag = &sm.abort_flag;
