@@ -13,10 +13,10 @@
 //   O_i   = s_V acc_i / (127 l_i)                          -> fp16
 // exp is evaluated as exp2 with log2(e) folded into the per-row constant.
 //
-// B200 design (one CTA per 128-query tile of one (b, h); 12 warps):
-//   warp 8      TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
+// B200 design (one CTA per 128-query tile of one (b, h); 16 warps):
+//   warp 12     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
 //               block's s_K values into a 3-stage shared-memory ring.
-//   warp 9      tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
+//   warp 13     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
 //               kind::i8 into one of two TMEM S buffers; P V with the P codes
 //               read straight from TMEM (aliasing the first 32 columns of the
 //               S buffer they came from) into a TMEM O block; owns the TMEM
@@ -24,21 +24,22 @@
 //               the fp32 output accumulator).
 //   warps 4-7   "prep" (one thread per query row): S row -> v = S s_K in
 //               fp32 (written back over S in TMEM), causal / ragged mask,
-//               running max m and alpha; then the output side: folds each
-//               int32 P V block into the row's fp32 accumulator in TMEM
+//               running max m and alpha.
+//   warps 8-11  output side (one thread per query row): folds each int32
+//               P V block into the row's fp32 accumulator in TMEM
 //               (o = alpha o + block) and writes the normalised fp16 row at
 //               the end.
 //   warps 0-3   "exp" (one thread per query row, same TMEM lanes as the prep
 //               warp on its SM sub-partition): reads v in 32-column chunks,
 //               p = 2^(c v - c m), the row sum, and the P codes, which it
 //               writes back to TMEM as the A operand of P V.
-//   warps 10-11 idle.
+//   warps 14-15 idle.
 // All per-row loops walk the row in 32-column chunks (one TMEM load each) and
 // are not unrolled across chunks, which keeps the three code paths that share
 // an SM sub-partition small enough for its instruction cache.
 // The exp warps are bound by the special-function unit (one exp2 per score);
-// the prep warps' integer/FMA work for block j+1 and the output update for
-// block j-1 run beside it on the same sub-partitions.
+// the prep warps' integer/FMA work for block j+1 and the output warps'
+// update for block j-1 run beside it on the same sub-partitions.
 // Every wait is bounded (clock-based); a timeout records a status word,
 // raises a CTA-wide abort flag, drains in-flight copies and MMAs, frees TMEM
 // and returns.
@@ -58,10 +59,10 @@ namespace {
 constexpr int BM = 128;                       // query rows per CTA
 constexpr int BN = 128;                       // keys per block
 constexpr int NS = 3;                         // K/V ring depth
-constexpr int kThreads = 384;                 // 12 warps = 3 warpgroups
-// Warp roles inside the third warpgroup (warps 8-11).
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 512;                 // 16 warps = 4 warpgroups
+// Warp roles inside the fourth warpgroup (warps 12-15).
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr int kTmemCols = 512;
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
@@ -119,11 +120,14 @@ struct alignas(1024) AttnSmem {
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
     float2 cm_alpha[2][BM];     // prep -> exp: (c m_new, alpha) per row and S buffer
-    float lsum[BM];             // exp -> prep: final row sums
+    float alpha_o[2][BM];       // prep -> output: alpha per row and S buffer
+    float lsum[BM];             // exp -> output: final row sums
     uint64_t q_full;
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
     uint64_t s_full[2], p_full[2];
     uint64_t x_full[2][4];      // prep warp k -> exp warp k (same TMEM lane quadrant)
+    uint64_t a_full[2][4];      // prep warp k -> output warp k
+    uint64_t a_empty[2][4];     // output warp k -> prep warp k
     uint64_t o_full, o_empty;
     uint64_t l_full, mma_drain;
     uint32_t tmem_base;
@@ -185,7 +189,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            for (int k = 0; k < 4; ++k) mbar_init(&sm.x_full[b][k], 32);
+            for (int k = 0; k < 4; ++k) {
+                mbar_init(&sm.x_full[b][k], 32);
+                mbar_init(&sm.a_full[b][k], 32);
+                mbar_init(&sm.a_empty[b][k], 32);
+            }
             mbar_init(&sm.p_full[b], BM);
         }
         mbar_init(&sm.o_full, 1);
@@ -207,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tbase + 256;    // int32 P V block, D columns
     const uint32_t tA = tO + D;         // fp32 output accumulator, D columns
 
-    if (warp >= 8) {
+    if (warp >= 12) {
       if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ---
         if (lane == 0) {
@@ -358,17 +366,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sm.lsum[row] = l;
         mbar_arrive(&sm.l_full);
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------------ prep ---
         const int row = tid - 128;
         const int qi = q0 + row;
-        const uint32_t lane_off = static_cast<uint32_t>(32 * (warp - 4)) << 16;
+        const int quad = warp - 4;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c (S_ij s_K[j]).
         // Clamped to a tiny positive value: a zero Q row then still maps masked
         // keys (v = -inf) to p = 0 and visible keys to p = 1.
         const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
                                   (kLog2e / sqrtf(static_cast<float>(D))),
                               1e-30f);
+        const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
+        float m_old = -INFINITY;
+        for (int j = 0; j < nb; ++j) {
+            // -- block j: v = fl(S s_K) (exact int32 -> fp32 by the
+            // magic-number add, |S| <= 127^2 d < 2^22), mask, row max.
+            const int b = j & 1, st = j % NS;
+            if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, abort_flag, 12)) break;
+            // s_K of this block: published by the producer's release-arrive
+            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 13)) break;
+            tc_fence_after();
+            const uint32_t ts = tS + lane_off + b * BN;
+            const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
+            const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t w[32];
+                tmem_ld32(ts + 32 * ch, w);
+                tmem_wait_ld();
+                float vv[32];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 k4 = sk4[8 * ch + q];
+                    const uint64_t a = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q] + kMagicBits),
+                                                           __uint_as_float(w[4 * q + 1] + kMagicBits)),
+                                                   negC2),
+                                             f2_pack(k4.x, k4.y));
+                    const uint64_t e = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q + 2] + kMagicBits),
+                                                           __uint_as_float(w[4 * q + 3] + kMagicBits)),
+                                                   negC2),
+                                             f2_pack(k4.z, k4.w));
+                    f2_unpack(a, vv[4 * q], vv[4 * q + 1]);
+                    f2_unpack(e, vv[4 * q + 2], vv[4 * q + 3]);
+                }
+                if (need_mask) {
+                    // keys past the end of the sequence, or after the query
+                    // (causal), get v = -inf (p = 0)
+                    const int lim = causal ? min(L, qi + 1) : L;
+                    const int key0 = j * BN + 32 * ch;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (key0 + e >= lim) vv[e] = -INFINITY;
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    mx[q & 3] = fmax3(mx[q & 3], fmaxf(vv[4 * q], vv[4 * q + 1]), fmaxf(vv[4 * q + 2], vv[4 * q + 3]));
+                    w[4 * q] = __float_as_uint(vv[4 * q]);
+                    w[4 * q + 1] = __float_as_uint(vv[4 * q + 1]);
+                    w[4 * q + 2] = __float_as_uint(vv[4 * q + 2]);
+                    w[4 * q + 3] = __float_as_uint(vv[4 * q + 3]);
+                }
+                tmem_st32(ts + 32 * ch, w);
+            }
+            mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
+            const float m_new = fmaxf(m_old, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
+            const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
+            m_old = m_new;
+            sm.cm_alpha[b][row] = make_float2(c * m_new, alpha);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.x_full[b][quad]);
+            // alpha of block j -> the output warp of this quadrant
+            if (j >= 2 && !warp_wait(&sm.a_empty[b][quad], ((j >> 1) - 1) & 1, abort_flag, 14)) break;
+            sm.alpha_o[b][row] = alpha;
+            mbar_arrive(&sm.a_full[b][quad]);
+        }
+    } else {
+        // ------------------------------------------------ output side ---
+        const int row = tid - 256;
+        const int qi = q0 + row;
+        const int quad = warp - 8;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
         {
             // the fp32 output accumulator starts at zero
@@ -379,101 +460,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ch = 0; ch < D / 32; ++ch) tmem_st32(tA + lane_off + 32 * ch, z);
             tmem_wait_st();
         }
-        float m_old = -INFINITY;
-        float alpha_prev = 0.0f;   // alpha of the block whose P V is folded next
         bool ok = true;
-        for (int j = 0; ok && j <= nb; ++j) {
-            float alpha_cur = 0.0f;
-            if (j < nb) {
-                // -- block j: v = fl(S s_K) (exact int32 -> fp32 by the
-                // magic-number add, |S| <= 127^2 d < 2^22), mask, row max.
-                const int b = j & 1, st = j % NS;
-                if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, abort_flag, 12)) { ok = false; break; }
-                // s_K of this block: published by the producer's release-arrive
-                if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 13)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t ts = tS + lane_off + b * BN;
-                const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
-                const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int j = 0; j < nb; ++j) {
+            const int b = j & 1;
+            // acc = alpha acc + (P V block), the int32 block turned into fp32
+            // exactly (|x| <= 127^2 128 < 2^22)
+            if (!warp_wait(&sm.o_full, j & 1, abort_flag, 9)) { ok = false; break; }
+            if (!warp_wait(&sm.a_full[b][quad], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
+            tc_fence_after();
+            const float alpha = sm.alpha_o[b][row];
+            mbar_arrive(&sm.a_empty[b][quad]);
+            const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll 1
-                for (int ch = 0; ch < BN / 32; ++ch) {
-                    uint32_t w[32];
-                    tmem_ld32(ts + 32 * ch, w);
-                    tmem_wait_ld();
-                    float vv[32];
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t w[32], o[32];
+                tmem_ld32(tO + lane_off + 32 * ch, w);
+                tmem_ld32(tA + lane_off + 32 * ch, o);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 k4 = sk4[8 * ch + q];
-                        const uint64_t a = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q] + kMagicBits),
-                                                               __uint_as_float(w[4 * q + 1] + kMagicBits)),
-                                                       negC2),
-                                                 f2_pack(k4.x, k4.y));
-                        const uint64_t e = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q + 2] + kMagicBits),
-                                                               __uint_as_float(w[4 * q + 3] + kMagicBits)),
-                                                       negC2),
-                                                 f2_pack(k4.z, k4.w));
-                        f2_unpack(a, vv[4 * q], vv[4 * q + 1]);
-                        f2_unpack(e, vv[4 * q + 2], vv[4 * q + 3]);
-                    }
-                    if (need_mask) {
-                        // keys past the end of the sequence, or after the query
-                        // (causal), get v = -inf (p = 0)
-                        const int lim = causal ? min(L, qi + 1) : L;
-                        const int key0 = j * BN + 32 * ch;
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (key0 + e >= lim) vv[e] = -INFINITY;
-                    }
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        mx[q & 3] = fmax3(mx[q & 3], fmaxf(vv[4 * q], vv[4 * q + 1]), fmaxf(vv[4 * q + 2], vv[4 * q + 3]));
-                        w[4 * q] = __float_as_uint(vv[4 * q]);
-                        w[4 * q + 1] = __float_as_uint(vv[4 * q + 1]);
-                        w[4 * q + 2] = __float_as_uint(vv[4 * q + 2]);
-                        w[4 * q + 3] = __float_as_uint(vv[4 * q + 3]);
-                    }
-                    tmem_st32(ts + 32 * ch, w);
+                for (int i = 0; i < 16; ++i) {
+                    const uint64_t x = fadd2(f2_pack(__uint_as_float(w[2 * i] + kMagicBits),
+                                                     __uint_as_float(w[2 * i + 1] + kMagicBits)),
+                                             negC2);
+                    float lo, hi;
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2, x),
+                              lo, hi);
+                    o[2 * i] = __float_as_uint(lo);
+                    o[2 * i + 1] = __float_as_uint(hi);
                 }
-                mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
-                const float m_new = fmaxf(m_old, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
-                alpha_cur = ex2(c * (m_old - m_new));   // 0 for the first block
-                m_old = m_new;
-                sm.cm_alpha[b][row] = make_float2(c * m_new, alpha_cur);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sm.x_full[b][warp - 4]);
+                tmem_st32(tA + lane_off + 32 * ch, o);
             }
-            if (j >= 1) {
-                // -- output side of block j - 1: acc = alpha acc + (P V block),
-                // the int32 block turned into fp32 exactly (|x| <= 127^2 128 < 2^22).
-                if (!warp_wait(&sm.o_full, (j - 1) & 1, abort_flag, 9)) { ok = false; break; }
-                tc_fence_after();
-                const uint64_t a2 = f2_pack(alpha_prev, alpha_prev);
-#pragma unroll 1
-                for (int ch = 0; ch < D / 32; ++ch) {
-                    uint32_t w[32], o[32];
-                    tmem_ld32(tO + lane_off + 32 * ch, w);
-                    tmem_ld32(tA + lane_off + 32 * ch, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const uint64_t x = fadd2(f2_pack(__uint_as_float(w[2 * i] + kMagicBits),
-                                                         __uint_as_float(w[2 * i + 1] + kMagicBits)),
-                                                 negC2);
-                        float lo, hi;
-                        f2_unpack(ffma2(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2, x),
-                                  lo, hi);
-                        o[2 * i] = __float_as_uint(lo);
-                        o[2 * i + 1] = __float_as_uint(hi);
-                    }
-                    tmem_st32(tA + lane_off + 32 * ch, o);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sm.o_empty);
-            }
-            alpha_prev = alpha_cur;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.o_empty);
         }
         if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11)) {
             tc_fence_after();
