@@ -15,19 +15,19 @@
 //
 // B200 design (one CTA per 128-query tile of one (b, h); 16 warps):
 //   warp 12     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
-//               block's s_K values into a 3-stage shared-memory ring.
+//               block's s_K values into a 5-stage shared-memory ring.
 //   warp 13     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
-//               kind::i8 into one of two TMEM S buffers; P V with the P codes
-//               read straight from TMEM (aliasing the first 32 columns of the
-//               S buffer they came from) into a TMEM O block; owns the TMEM
-//               allocation (512 columns: S0, S1, the int32 P V block and
-//               the fp32 output accumulator).
+//               kind::i8 into one of three TMEM S buffers, running three key
+//               blocks ahead of P V; P V with the P codes read straight from
+//               TMEM (aliasing the first 32 columns of the S buffer they came
+//               from) into a TMEM int32 block; owns the TMEM allocation
+//               (S0..S2: 3 x 128 columns, P V block: d columns).
 //   warps 4-7   "prep" (one thread per query row): S row -> v = S s_K in
 //               fp32 (written back over S in TMEM), causal / ragged mask,
 //               running max m and alpha.
 //   warps 8-11  output side (one thread per query row): folds each int32
-//               P V block into the row's fp32 accumulator in TMEM
-//               (o = alpha o + block) and writes the normalised fp16 row at
+//               P V block into the row's fp32 accumulator, held in registers
+//               (o = alpha o + block), and writes the normalised fp16 row at
 //               the end.
 //   warps 0-3   "exp" (one thread per query row, same TMEM lanes as the prep
 //               warp on its SM sub-partition): reads v in 32-column chunks,
@@ -58,12 +58,33 @@ namespace {
 
 constexpr int BM = 128;                       // query rows per CTA
 constexpr int BN = 128;                       // keys per block
-constexpr int NS = 3;                         // K/V ring depth
+constexpr int NS = 5;                         // K/V ring depth
 constexpr int kThreads = 512;                 // 16 warps = 4 warpgroups
+constexpr int SB = 3;                         // TMEM S buffers
+// Register split (setmaxnreg): launched with kLaunchRegs per thread (checked
+// on the host before every launch); the output warpgroup, which holds a
+// d-column fp32 row, takes registers from the other three.  The shares add up
+// to at most the launch total.
+constexpr int kLaunchRegs = 128;
+constexpr uint32_t kRegsExp = 104;
+constexpr uint32_t kRegsPrep = 104;
+constexpr uint32_t kRegsOutput = 216;
+constexpr uint32_t kRegsOther = 40;
+static_assert(128 * (kRegsExp + kRegsPrep + kRegsOutput + kRegsOther) <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 // Warp roles inside the fourth warpgroup (warps 12-15).
 constexpr int kProducerWarp = 12;
 constexpr int kMmaWarp = 13;
 constexpr int kTmemCols = 512;
+
+// Moves this warpgroup from kLaunchRegs to R registers per thread with the
+// matching setmaxnreg direction (chosen at compile time).
+template <uint32_t R>
+__device__ __forceinline__ void regs_to() {
+    static_assert(R % 8 == 0 && R >= 24 && R <= 256, "setmaxnreg range");
+    if constexpr (R > static_cast<uint32_t>(kLaunchRegs)) regs_inc<R>();
+    else if constexpr (R < static_cast<uint32_t>(kLaunchRegs)) regs_dec<R>();
+}
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
 // 1.5 * 2^23: for an integer |n| < 2^22, the fp32 bit pattern 0x4B400000 + n
@@ -119,13 +140,13 @@ struct alignas(1024) AttnSmem {
     uint8_t k[NS][BN * D];      // K_hat tiles
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
-    float2 cm_alpha[2][BM];     // prep -> exp: (c m_new, alpha) per row and S buffer
+    float2 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha) per row and S buffer
     float alpha_o[2][BM];       // prep -> output: alpha per row and S buffer
     float lsum[BM];             // exp -> output: final row sums
     uint64_t q_full;
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
-    uint64_t s_full[2], p_full[2];
-    uint64_t x_full[2][4];      // prep warp k -> exp warp k (same TMEM lane quadrant)
+    uint64_t s_full[SB], p_full[SB];
+    uint64_t x_full[SB][4];     // prep warp k -> exp warp k (same TMEM lane quadrant)
     uint64_t a_full[2][4];      // prep warp k -> output warp k
     uint64_t a_empty[2][4];     // output warp k -> prep warp k
     uint64_t o_full, o_empty;
@@ -187,15 +208,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1 + BM);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < SB; ++b) {
             mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.p_full[b], BM);
+            for (int k = 0; k < 4; ++k) mbar_init(&sm.x_full[b][k], 32);
+        }
+        for (int b = 0; b < 2; ++b)
             for (int k = 0; k < 4; ++k) {
-                mbar_init(&sm.x_full[b][k], 32);
                 mbar_init(&sm.a_full[b][k], 32);
                 mbar_init(&sm.a_empty[b][k], 32);
             }
-            mbar_init(&sm.p_full[b], BM);
-        }
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.o_empty, BM);
         mbar_init(&sm.l_full, BM);
@@ -211,11 +233,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
-    const uint32_t tS = tbase;          // S0 at column 0, S1 at column 128
-    const uint32_t tO = tbase + 256;    // int32 P V block, D columns
-    const uint32_t tA = tO + D;         // fp32 output accumulator, D columns
+    const uint32_t tS = tbase;              // S buffer s at column 128 s
+    const uint32_t tO = tbase + 128 * SB;   // int32 P V block, D columns
 
     if (warp >= 12) {
+      regs_to<kRegsOther>();
       if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ---
         if (lane == 0) {
@@ -266,9 +288,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = warp_wait(&sm.q_full, 0, abort_flag, 2);
         tc_fence_after();
 
+        auto issue_qk = [&](int j) -> bool {
+            const int st = j % NS, sb = j % SB;
+            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 6)) return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
+#pragma unroll
+                for (int k = 0; k < D / 32; ++k)
+                    mma_i8_ss(tS + sb * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
+                mma_commit(&sm.s_full[sb]);
+            }
+            __syncwarp();
+            return true;
+        };
         auto issue_pv = [&](int j) -> bool {
-            const int b = j & 1, st = j % NS;
-            if (!warp_wait(&sm.p_full[b], (j >> 1) & 1, abort_flag, 3)) return false;
+            const int sb = j % SB, st = j % NS;
+            if (!warp_wait(&sm.p_full[sb], (j / SB) & 1, abort_flag, 3)) return false;
             if (!warp_wait(&sm.v_full[st], (j / NS) & 1, abort_flag, 4)) return false;
             if (j >= 1 && !warp_wait(&sm.o_empty, (j - 1) & 1, abort_flag, 5)) return false;
             tc_fence_after();
@@ -276,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
 #pragma unroll
                 for (int k = 0; k < BN / 32; ++k)
-                    mma_i8_ts(tO, tS + b * BN + 8 * k, vdesc + 2 * k, idesc_pv, k > 0);
+                    mma_i8_ts(tO, tS + sb * BN + 8 * k, vdesc + 2 * k, idesc_pv, k > 0);
                 mma_commit(&sm.o_full);
                 mma_commit(&sm.kv_empty[st]);
             }
@@ -284,21 +320,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
         };
 
+        // Q K^T runs SB blocks ahead of P V: Q K^T of block j + SB reuses the
+        // S buffer of block j and is issued after P V of block j, which the
+        // tensor pipe executes first.
+        for (int j = 0; ok && j < SB && j < nb; ++j) ok = issue_qk(j);
         for (int j = 0; ok && j < nb; ++j) {
-            const int st = j % NS, b = j & 1;
-            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 6)) { ok = false; break; }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
-#pragma unroll
-                for (int k = 0; k < D / 32; ++k)
-                    mma_i8_ss(tS + b * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
-                mma_commit(&sm.s_full[b]);
-            }
-            __syncwarp();
-            if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+            if (!issue_pv(j)) { ok = false; break; }
+            if (j + SB < nb && !issue_qk(j + SB)) { ok = false; break; }
         }
-        if (ok) issue_pv(nb - 1);
         // Drain: every MMA this warp issued has completed before TMEM is freed.
         if (lane == 0) mma_commit(&sm.mma_drain);
         __syncwarp();
@@ -307,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the other two warps of this warpgroup have no role
     } else if (warp < 4) {
+        regs_to<kRegsExp>();
         // ------------------------------------------------------- exp ---
         const int row = tid;
         const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
@@ -320,8 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t mag2 = f2_pack(kMagic, kMagic);
         float l = 0.0f;
         for (int j = 0; j < nb; ++j) {
-            const int b = j & 1;
-            if (!warp_wait(&sm.x_full[b][warp], (j >> 1) & 1, abort_flag, 7)) break;
+            const int b = j % SB;
+            if (!warp_wait(&sm.x_full[b][warp], (j / SB) & 1, abort_flag, 7)) break;
             tc_fence_after();
             const float2 ca = sm.cm_alpha[b][row];
             const uint64_t ncm2 = f2_pack(-ca.x, -ca.x);
@@ -367,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.lsum[row] = l;
         mbar_arrive(&sm.l_full);
     } else if (warp < 8) {
+        regs_to<kRegsPrep>();
         // ------------------------------------------------------ prep ---
         const int row = tid - 128;
         const int qi = q0 + row;
@@ -383,8 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nb; ++j) {
             // -- block j: v = fl(S s_K) (exact int32 -> fp32 by the
             // magic-number add, |S| <= 127^2 d < 2^22), mask, row max.
-            const int b = j & 1, st = j % NS;
-            if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, abort_flag, 12)) break;
+            const int b = j % SB, ab = j & 1, st = j % NS;
+            if (!warp_wait(&sm.s_full[b], (j / SB) & 1, abort_flag, 12)) break;
             // s_K of this block: published by the producer's release-arrive
             if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 13)) break;
             tc_fence_after();
@@ -440,82 +471,65 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&sm.x_full[b][quad]);
             // alpha of block j -> the output warp of this quadrant
-            if (j >= 2 && !warp_wait(&sm.a_empty[b][quad], ((j >> 1) - 1) & 1, abort_flag, 14)) break;
-            sm.alpha_o[b][row] = alpha;
-            mbar_arrive(&sm.a_full[b][quad]);
+            if (j >= 2 && !warp_wait(&sm.a_empty[ab][quad], ((j >> 1) - 1) & 1, abort_flag, 14)) break;
+            sm.alpha_o[ab][row] = alpha;
+            mbar_arrive(&sm.a_full[ab][quad]);
         }
     } else {
+        regs_to<kRegsOutput>();
         // ------------------------------------------------ output side ---
         const int row = tid - 256;
         const int qi = q0 + row;
         const int quad = warp - 8;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
-        {
-            // the fp32 output accumulator starts at zero
-            uint32_t z[32];
+        uint64_t o2[D / 2];   // the output row as fp32 pairs
 #pragma unroll
-            for (int i = 0; i < 32; ++i) z[i] = 0u;
-#pragma unroll 1
-            for (int ch = 0; ch < D / 32; ++ch) tmem_st32(tA + lane_off + 32 * ch, z);
-            tmem_wait_st();
-        }
+        for (int i = 0; i < D / 2; ++i) o2[i] = 0ull;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
-            const int b = j & 1;
-            // acc = alpha acc + (P V block), the int32 block turned into fp32
+            const int ab = j & 1;
+            // o = alpha o + (P V block), the int32 block turned into fp32
             // exactly (|x| <= 127^2 128 < 2^22)
             if (!warp_wait(&sm.o_full, j & 1, abort_flag, 9)) { ok = false; break; }
-            if (!warp_wait(&sm.a_full[b][quad], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
+            if (!warp_wait(&sm.a_full[ab][quad], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
             tc_fence_after();
-            const float alpha = sm.alpha_o[b][row];
-            mbar_arrive(&sm.a_empty[b][quad]);
+            const float alpha = sm.alpha_o[ab][row];
+            mbar_arrive(&sm.a_empty[ab][quad]);
             const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll 1
+            uint32_t w[2][32];
+            tmem_ld32(tO + lane_off, w[0]);
+            tmem_wait_ld();
+#pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t w[32], o[32];
-                tmem_ld32(tO + lane_off + 32 * ch, w);
-                tmem_ld32(tA + lane_off + 32 * ch, o);
-                tmem_wait_ld();
+                if (ch + 1 < D / 32) tmem_ld32(tO + lane_off + 32 * (ch + 1), w[(ch + 1) & 1]);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = fadd2(f2_pack(__uint_as_float(w[2 * i] + kMagicBits),
-                                                     __uint_as_float(w[2 * i + 1] + kMagicBits)),
+                    const uint64_t x = fadd2(f2_pack(__uint_as_float(w[ch & 1][2 * i] + kMagicBits),
+                                                     __uint_as_float(w[ch & 1][2 * i + 1] + kMagicBits)),
                                              negC2);
-                    float lo, hi;
-                    f2_unpack(ffma2(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2, x),
-                              lo, hi);
-                    o[2 * i] = __float_as_uint(lo);
-                    o[2 * i + 1] = __float_as_uint(hi);
+                    o2[16 * ch + i] = ffma2(o2[16 * ch + i], a2, x);
                 }
-                tmem_st32(tA + lane_off + 32 * ch, o);
+                if (ch + 1 < D / 32) tmem_wait_ld();
             }
-            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.o_empty);
         }
-        if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11)) {
-            tc_fence_after();
+        if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11) && qi < L) {
             const float l = sm.lsum[row];
             const float f = __ldg(sV + bh) / (127.0f * l);
             uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(bh) * L + qi) * D);
-#pragma unroll 1
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t o[32];
-                tmem_ld32(tA + lane_off + 32 * ch, o);
-                tmem_wait_ld();
-                if (qi < L) {
 #pragma unroll
-                    for (int c8 = 0; c8 < 4; ++c8) {
-                        uint4 w;
-                        __half2 *h = reinterpret_cast<__half2 *>(&w);
+            for (int c8 = 0; c8 < D / 8; ++c8) {
+                uint4 wv;
+                __half2 *h = reinterpret_cast<__half2 *>(&wv);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            h[e] = __floats2half2_rn(__uint_as_float(o[8 * c8 + 2 * e]) * f,
-                                                     __uint_as_float(o[8 * c8 + 2 * e + 1]) * f);
-                        dst[4 * ch + c8] = w;
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    float lo, hi;
+                    f2_unpack(o2[4 * c8 + e], lo, hi);
+                    h[e] = __floats2half2_rn(lo * f, hi * f);
                 }
+                dst[c8] = wv;
             }
         }
     }
@@ -663,6 +677,12 @@ int launch_attn(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const floa
     rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(smem)));
     if (rc) return rc;
+    // The in-kernel register split assumes exactly kLaunchRegs per thread at
+    // launch; a different count could leave setmaxnreg.inc waiting forever.
+    cudaFuncAttributes fa;
+    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>));
+    if (rc) return rc;
+    if (fa.numRegs != kLaunchRegs) return INTFA_ERR_UNSUPPORTED;
     const int ntiles = (L + BM - 1) / BM;
     const unsigned grid = static_cast<unsigned>(ntiles) * static_cast<unsigned>(BH);
     attn_fwd_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, sQ, sK, sV,
