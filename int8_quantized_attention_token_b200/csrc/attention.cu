@@ -87,12 +87,9 @@ __device__ __forceinline__ void regs_to() {
 }
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
-// 1.5 * 2^23: for an integer |n| < 2^22, the fp32 bit pattern 0x4B400000 + n
-// is exactly the value 1.5 * 2^23 + n, so n -> float is one integer add and one
-// float subtract; and for 0 <= y < 2^22, fl(y + 1.5 * 2^23) holds RNE(y) in its
-// low mantissa bits.
+// 1.5 * 2^23: for 0 <= y < 2^22, fl(y + 1.5 * 2^23) is 1.5 * 2^23 + RNE(y),
+// so RNE(y) sits in the low mantissa bits of that float.
 constexpr float kMagic = 12582912.0f;
-constexpr uint32_t kMagicBits = 0x4B400000u;
 
 // -------------------------------------------------------- bounded waits ---
 
@@ -345,50 +342,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
                                   (kLog2e / sqrtf(static_cast<float>(D))),
                               1e-30f);
-        const uint64_t c2 = f2_pack(c, c);
-        const uint64_t k127 = f2_pack(127.0f, 127.0f);
-        const uint64_t mag2 = f2_pack(kMagic, kMagic);
         float l = 0.0f;
         for (int j = 0; j < nb; ++j) {
             const int b = j % SB;
             if (!warp_wait(&sm.x_full[b][warp], (j / SB) & 1, abort_flag, 7)) break;
             tc_fence_after();
             const float2 ca = sm.cm_alpha[b][row];
-            const uint64_t ncm2 = f2_pack(-ca.x, -ca.x);
             const uint32_t tv = tS + lane_off + b * BN;
-            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+            const float ncm = -ca.x;
+            float ps0 = 0.0f, ps1 = 0.0f, ps2 = 0.0f, ps3 = 0.0f;
+            // two 32-column chunks per step: the next pair's TMEM load is in
+            // flight while this pair is processed
+            uint32_t w[2][32];
+            tmem_ld32(tv, w[0]);
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                uint32_t w[32];
-                tmem_ld32(tv + 32 * ch, w);
+            for (int ch = 0; ch < BN / 32; ch += 2) {
+                tmem_ld32(tv + 32 * (ch + 1), w[1]);
                 tmem_wait_ld();
-                uint32_t pk[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
-                    float x0, x1, x2, x3;
-                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), c2, ncm2), x0, x1);
-                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2, ncm2), x2, x3);
-                    const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
-                    const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
-                    acc[q & 3] = fadd2(acc[q & 3], fadd2(p01, p23));
-                    // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
-                    float t0, t1, t2, t3;
-                    f2_unpack(ffma2(p01, k127, mag2), t0, t1);
-                    f2_unpack(ffma2(p23, k127, mag2), t2, t3);
-                    pk[q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
-                                 prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 1 && ch + 2 < BN / 32) {
+                        // w[0] is consumed: start loading the next even chunk
+                        tmem_ld32(tv + 32 * (ch + 2), w[0]);
+                    }
+                    const uint32_t *wv = w[h];
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
+                        const float p0 = ex2(fmaf(__uint_as_float(wv[4 * q]), c, ncm));
+                        const float p1 = ex2(fmaf(__uint_as_float(wv[4 * q + 1]), c, ncm));
+                        const float p2 = ex2(fmaf(__uint_as_float(wv[4 * q + 2]), c, ncm));
+                        const float p3 = ex2(fmaf(__uint_as_float(wv[4 * q + 3]), c, ncm));
+                        ps0 += p0;
+                        ps1 += p1;
+                        ps2 += p2;
+                        ps3 += p3;
+                        // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
+                        const uint32_t t0 = __float_as_uint(fmaf(p0, 127.0f, kMagic));
+                        const uint32_t t1 = __float_as_uint(fmaf(p1, 127.0f, kMagic));
+                        const uint32_t t2 = __float_as_uint(fmaf(p2, 127.0f, kMagic));
+                        const uint32_t t3 = __float_as_uint(fmaf(p3, 127.0f, kMagic));
+                        pk[q] = prmt(prmt(t0, t1, 0x0040u), prmt(t2, t3, 0x0040u), 0x5410u);
+                    }
+                    // codes of keys 32 c .. 32 c + 31 -> columns 8 c .. 8 c + 7,
+                    // which this thread has already read (chunk 0 is columns 0..31)
+                    tmem_st8(tv + 8 * (ch + h), pk);
                 }
-                // codes of keys 32 ch .. 32 ch + 31 -> columns 8 ch .. 8 ch + 7,
-                // which this thread has already read (chunk 0 is columns 0..31)
-                tmem_st8(tv + 8 * ch, pk);
             }
-            float s0, s1, s2, s3, s4, s5, s6, s7;
-            f2_unpack(acc[0], s0, s1);
-            f2_unpack(acc[1], s2, s3);
-            f2_unpack(acc[2], s4, s5);
-            f2_unpack(acc[3], s6, s7);
-            const float ps = ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            const float ps = (ps0 + ps1) + (ps2 + ps3);
             l = l * ca.y + ps;
             tmem_wait_st();
             tc_fence_before();
@@ -409,11 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
                                   (kLog2e / sqrtf(static_cast<float>(D))),
                               1e-30f);
-        const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
         float m_old = -INFINITY;
         for (int j = 0; j < nb; ++j) {
-            // -- block j: v = fl(S s_K) (exact int32 -> fp32 by the
-            // magic-number add, |S| <= 127^2 d < 2^22), mask, row max.
+            // -- block j: v = fl(S s_K) (int32 -> fp32 exact, |S| <= 127^2 d
+            // < 2^24), mask, row max.
             const int b = j % SB, ab = j & 1, st = j % NS;
             if (!warp_wait(&sm.s_full[b], (j / SB) & 1, abort_flag, 12)) break;
             // s_K of this block: published by the producer's release-arrive
@@ -432,13 +433,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const float4 k4 = sk4[8 * ch + q];
-                    const uint64_t a = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q] + kMagicBits),
-                                                           __uint_as_float(w[4 * q + 1] + kMagicBits)),
-                                                   negC2),
+                    const uint64_t a = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q])),
+                                                     __int2float_rn(static_cast<int32_t>(w[4 * q + 1]))),
                                              f2_pack(k4.x, k4.y));
-                    const uint64_t e = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q + 2] + kMagicBits),
-                                                           __uint_as_float(w[4 * q + 3] + kMagicBits)),
-                                                   negC2),
+                    const uint64_t e = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q + 2])),
+                                                     __int2float_rn(static_cast<int32_t>(w[4 * q + 3]))),
                                              f2_pack(k4.z, k4.w));
                     f2_unpack(a, vv[4 * q], vv[4 * q + 1]);
                     f2_unpack(e, vv[4 * q + 2], vv[4 * q + 3]);
@@ -454,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    mx[q & 3] = fmax3(mx[q & 3], fmaxf(vv[4 * q], vv[4 * q + 1]), fmaxf(vv[4 * q + 2], vv[4 * q + 3]));
+                    mx[q & 3] = fmax3(mx[q & 3], vv[4 * q], vv[4 * q + 1]);
+                    mx[(q + 2) & 3] = fmax3(mx[(q + 2) & 3], vv[4 * q + 2], vv[4 * q + 3]);
                     w[4 * q] = __float_as_uint(vv[4 * q]);
                     w[4 * q + 1] = __float_as_uint(vv[4 * q + 1]);
                     w[4 * q + 2] = __float_as_uint(vv[4 * q + 2]);
@@ -482,7 +482,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qi = q0 + row;
         const int quad = warp - 8;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        const uint64_t negC2 = f2_pack(-kMagic, -kMagic);
         uint64_t o2[D / 2];   // the output row as fp32 pairs
 #pragma unroll
         for (int i = 0; i < D / 2; ++i) o2[i] = 0ull;
@@ -490,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nb; ++j) {
             const int ab = j & 1;
             // o = alpha o + (P V block), the int32 block turned into fp32
-            // exactly (|x| <= 127^2 128 < 2^22)
+            // exactly (|x| <= 127^2 128 < 2^24)
             if (!warp_wait(&sm.o_full, j & 1, abort_flag, 9)) { ok = false; break; }
             if (!warp_wait(&sm.a_full[ab][quad], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
             tc_fence_after();
@@ -505,9 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ch + 1 < D / 32) tmem_ld32(tO + lane_off + 32 * (ch + 1), w[(ch + 1) & 1]);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = fadd2(f2_pack(__uint_as_float(w[ch & 1][2 * i] + kMagicBits),
-                                                     __uint_as_float(w[ch & 1][2 * i + 1] + kMagicBits)),
-                                             negC2);
+                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w[ch & 1][2 * i])),
+                                               __int2float_rn(static_cast<int32_t>(w[ch & 1][2 * i + 1])));
                     o2[16 * ch + i] = ffma2(o2[16 * ch + i], a2, x);
                 }
                 if (ch + 1 < D / 32) tmem_wait_ld();
