@@ -13,27 +13,27 @@
 //   O_i   = s_V acc_i / (127 l_i)                          -> fp16
 // exp is evaluated as exp2 with log2(e) folded into the per-row constant.
 //
-// B200 design (one CTA per 128-query tile of one (b, h); 16 warps):
-//   warp 12     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
+// B200 design (one CTA per 128-query tile of one (b, h); 20 warps):
+//   warp 16     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
 //               block's s_K values into a 5-stage shared-memory ring.
-//   warp 13     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
+//   warp 17     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
 //               kind::i8 into one of three TMEM S buffers, running three key
 //               blocks ahead of P V; P V with the P codes read straight from
 //               TMEM (aliasing the first 32 columns of the S buffer they came
 //               from) into a TMEM int32 block; owns the TMEM allocation
 //               (S0..S2: 3 x 128 columns, P V block: d columns).
-//   warps 4-7   "prep" (one thread per query row): S row -> v = S s_K in
+//   warps 8-11  "prep" (one thread per query row): S row -> v = S s_K in
 //               fp32 (written back over S in TMEM), causal / ragged mask,
 //               running max m and alpha.
-//   warps 8-11  output side (one thread per query row): folds each int32
+//   warps 12-15 output side (one thread per query row): folds each int32
 //               P V block into the row's fp32 accumulator, held in registers
 //               (o = alpha o + block), and writes the normalised fp16 row at
 //               the end.
-//   warps 0-3   "exp" (one thread per query row, same TMEM lanes as the prep
-//               warp on its SM sub-partition): reads v in 32-column chunks,
-//               p = 2^(c v - c m), the row sum, and the P codes, which it
-//               writes back to TMEM as the A operand of P V.
-//   warps 14-15 idle.
+//   warps 0-7   "exp" (two warps per TMEM lane quadrant, each one thread per
+//               query row and half of the 128 keys): reads v in 32-column
+//               chunks, p = 2^(c v - c m), the row sum, and the P codes,
+//               which it writes back to TMEM as the A operand of P V.
+//   warps 18-19 idle.
 // All per-row loops walk the row in 32-column chunks (one TMEM load each) and
 // are not unrolled across chunks, which keeps the three code paths that share
 // an SM sub-partition small enough for its instruction cache.
@@ -59,22 +59,22 @@ namespace {
 constexpr int BM = 128;                       // query rows per CTA
 constexpr int BN = 128;                       // keys per block
 constexpr int NS = 5;                         // K/V ring depth
-constexpr int kThreads = 512;                 // 16 warps = 4 warpgroups
+constexpr int kThreads = 640;                 // 20 warps = 5 warpgroups
 constexpr int SB = 3;                         // TMEM S buffers
 // Register split (setmaxnreg): launched with kLaunchRegs per thread (checked
 // on the host before every launch); the output warpgroup, which holds a
 // d-column fp32 row, takes registers from the other three.  The shares add up
 // to at most the launch total.
-constexpr int kLaunchRegs = 128;
-constexpr uint32_t kRegsExp = 104;
-constexpr uint32_t kRegsPrep = 104;
-constexpr uint32_t kRegsOutput = 216;
-constexpr uint32_t kRegsOther = 40;
-static_assert(128 * (kRegsExp + kRegsPrep + kRegsOutput + kRegsOther) <= kThreads * kLaunchRegs,
+constexpr int kLaunchRegs = 96;
+constexpr uint32_t kRegsExp = 72;      // each of the two exp warpgroups
+constexpr uint32_t kRegsPrep = 96;
+constexpr uint32_t kRegsOutput = 192;
+constexpr uint32_t kRegsOther = 48;
+static_assert(128 * (2 * kRegsExp + kRegsPrep + kRegsOutput + kRegsOther) <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-// Warp roles inside the fourth warpgroup (warps 12-15).
-constexpr int kProducerWarp = 12;
-constexpr int kMmaWarp = 13;
+// Warp roles inside the fifth warpgroup (warps 16-19).
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr int kTmemCols = 512;
 
 // Moves this warpgroup from kLaunchRegs to R registers per thread with the
@@ -139,7 +139,7 @@ struct alignas(1024) AttnSmem {
     float sk[NS][BN];           // s_K of each key block
     float2 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha) per row and S buffer
     float alpha_o[2][BM];       // prep -> output: alpha per row and S buffer
-    float lsum[BM];             // exp -> output: final row sums
+    float lsum[2][BM];          // exp -> output: final row sums of each column half
     uint64_t q_full;
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
     uint64_t s_full[SB], p_full[SB];
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < SB; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.p_full[b], BM);
+            mbar_init(&sm.p_full[b], 2 * BM);
             for (int k = 0; k < 4; ++k) mbar_init(&sm.x_full[b][k], 32);
         }
         for (int b = 0; b < 2; ++b)
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.o_empty, BM);
-        mbar_init(&sm.l_full, BM);
+        mbar_init(&sm.l_full, 2 * BM);
         mbar_init(&sm.mma_drain, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tbase;              // S buffer s at column 128 s
     const uint32_t tO = tbase + 128 * SB;   // int32 P V block, D columns
 
-    if (warp >= 12) {
+    if (warp >= 16) {
       regs_to<kRegsOther>();
       if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ---
@@ -308,8 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
 #pragma unroll
-                for (int k = 0; k < BN / 32; ++k)
-                    mma_i8_ts(tO, tS + sb * BN + 8 * k, vdesc + 2 * k, idesc_pv, k > 0);
+                for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k..: see the exp warps
+                    mma_i8_ts(tO, tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k, idesc_pv, k > 0);
                 mma_commit(&sm.o_full);
                 mma_commit(&sm.kv_empty[st]);
             }
@@ -332,11 +332,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       // the other two warps of this warpgroup have no role
-    } else if (warp < 4) {
+    } else if (warp < 8) {
         regs_to<kRegsExp>();
         // ------------------------------------------------------- exp ---
-        const int row = tid;
-        const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+        // Two warps per TMEM lane quadrant: half hf takes keys 64 hf .. 64 hf
+        // + 63 of each block (chunks 2 hf, 2 hf + 1) and writes their 16 code
+        // words into columns 64 hf .. 64 hf + 15, which only it reads.
+        const int hf = warp >> 2, quad = warp & 3;
+        const int row = 32 * quad + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         const int qi = q0 + row;
         // c = s_Q[i] log2(e) / sqrt(d) (see the prep warps for the clamp)
         const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
@@ -345,65 +349,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         float l = 0.0f;
         for (int j = 0; j < nb; ++j) {
             const int b = j % SB;
-            if (!warp_wait(&sm.x_full[b][warp], (j / SB) & 1, abort_flag, 7)) break;
+            if (!warp_wait(&sm.x_full[b][quad], (j / SB) & 1, abort_flag, 7)) break;
             tc_fence_after();
             const float2 ca = sm.cm_alpha[b][row];
-            const uint32_t tv = tS + lane_off + b * BN;
             const float ncm = -ca.x;
+            const uint32_t tv = tS + lane_off + b * BN + 64 * hf;
             float ps0 = 0.0f, ps1 = 0.0f, ps2 = 0.0f, ps3 = 0.0f;
-            // two 32-column chunks per step: the next pair's TMEM load is in
-            // flight while this pair is processed
-            uint32_t w[2][32];
-            tmem_ld32(tv, w[0]);
-#pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ch += 2) {
-                tmem_ld32(tv + 32 * (ch + 1), w[1]);
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                uint32_t w[32];
+                tmem_ld32(tv + 32 * e, w);
                 tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (h == 1 && ch + 2 < BN / 32) {
-                        // w[0] is consumed: start loading the next even chunk
-                        tmem_ld32(tv + 32 * (ch + 2), w[0]);
-                    }
-                    const uint32_t *wv = w[h];
-                    uint32_t pk[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
-                        const float p0 = ex2(fmaf(__uint_as_float(wv[4 * q]), c, ncm));
-                        const float p1 = ex2(fmaf(__uint_as_float(wv[4 * q + 1]), c, ncm));
-                        const float p2 = ex2(fmaf(__uint_as_float(wv[4 * q + 2]), c, ncm));
-                        const float p3 = ex2(fmaf(__uint_as_float(wv[4 * q + 3]), c, ncm));
-                        ps0 += p0;
-                        ps1 += p1;
-                        ps2 += p2;
-                        ps3 += p3;
-                        // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
-                        const uint32_t t0 = __float_as_uint(fmaf(p0, 127.0f, kMagic));
-                        const uint32_t t1 = __float_as_uint(fmaf(p1, 127.0f, kMagic));
-                        const uint32_t t2 = __float_as_uint(fmaf(p2, 127.0f, kMagic));
-                        const uint32_t t3 = __float_as_uint(fmaf(p3, 127.0f, kMagic));
-                        pk[q] = prmt(prmt(t0, t1, 0x0040u), prmt(t2, t3, 0x0040u), 0x5410u);
-                    }
-                    // codes of keys 32 c .. 32 c + 31 -> columns 8 c .. 8 c + 7,
-                    // which this thread has already read (chunk 0 is columns 0..31)
-                    tmem_st8(tv + 8 * (ch + h), pk);
+                for (int q = 0; q < 8; ++q) {
+                    // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
+                    const float p0 = ex2(fmaf(__uint_as_float(w[4 * q]), c, ncm));
+                    const float p1 = ex2(fmaf(__uint_as_float(w[4 * q + 1]), c, ncm));
+                    const float p2 = ex2(fmaf(__uint_as_float(w[4 * q + 2]), c, ncm));
+                    const float p3 = ex2(fmaf(__uint_as_float(w[4 * q + 3]), c, ncm));
+                    ps0 += p0;
+                    ps1 += p1;
+                    ps2 += p2;
+                    ps3 += p3;
+                    // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
+                    const uint32_t t0 = __float_as_uint(fmaf(p0, 127.0f, kMagic));
+                    const uint32_t t1 = __float_as_uint(fmaf(p1, 127.0f, kMagic));
+                    const uint32_t t2 = __float_as_uint(fmaf(p2, 127.0f, kMagic));
+                    const uint32_t t3 = __float_as_uint(fmaf(p3, 127.0f, kMagic));
+                    pk[8 * e + q] = prmt(prmt(t0, t1, 0x0040u), prmt(t2, t3, 0x0040u), 0x5410u);
                 }
             }
+            // both chunks are in registers: their columns now take the codes
+            tmem_st8(tv, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
+            tmem_st8(tv + 8, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
             const float ps = (ps0 + ps1) + (ps2 + ps3);
             l = l * ca.y + ps;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
         }
-        sm.lsum[row] = l;
+        sm.lsum[hf][row] = l;
         mbar_arrive(&sm.l_full);
-    } else if (warp < 8) {
+    } else if (warp < 12) {
         regs_to<kRegsPrep>();
         // ------------------------------------------------------ prep ---
-        const int row = tid - 128;
+        const int row = tid - 256;
         const int qi = q0 + row;
-        const int quad = warp - 4;
+        const int quad = warp - 8;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c (S_ij s_K[j]).
         // Clamped to a tiny positive value: a zero Q row then still maps masked
@@ -478,9 +471,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         regs_to<kRegsOutput>();
         // ------------------------------------------------ output side ---
-        const int row = tid - 256;
+        const int row = tid - 384;
         const int qi = q0 + row;
-        const int quad = warp - 8;
+        const int quad = warp - 12;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         uint64_t o2[D / 2];   // the output row as fp32 pairs
 #pragma unroll
@@ -496,25 +489,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float alpha = sm.alpha_o[ab][row];
             mbar_arrive(&sm.a_empty[ab][quad]);
             const uint64_t a2 = f2_pack(alpha, alpha);
-            uint32_t w[2][32];
-            tmem_ld32(tO + lane_off, w[0]);
-            tmem_wait_ld();
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
-                if (ch + 1 < D / 32) tmem_ld32(tO + lane_off + 32 * (ch + 1), w[(ch + 1) & 1]);
+                uint32_t w[32];
+                tmem_ld32(tO + lane_off + 32 * ch, w);
+                tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w[ch & 1][2 * i])),
-                                               __int2float_rn(static_cast<int32_t>(w[ch & 1][2 * i + 1])));
+                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w[2 * i])),
+                                               __int2float_rn(static_cast<int32_t>(w[2 * i + 1])));
                     o2[16 * ch + i] = ffma2(o2[16 * ch + i], a2, x);
                 }
-                if (ch + 1 < D / 32) tmem_wait_ld();
             }
             tc_fence_before();
             mbar_arrive(&sm.o_empty);
         }
         if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11) && qi < L) {
-            const float l = sm.lsum[row];
+            const float l = sm.lsum[0][row] + sm.lsum[1][row];
             const float f = __ldg(sV + bh) / (127.0f * l);
             uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(bh) * L + qi) * D);
 #pragma unroll
