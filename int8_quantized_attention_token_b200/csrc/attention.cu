@@ -17,11 +17,11 @@
 //   warp 16     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
 //               block's s_K values into a 5-stage shared-memory ring.
 //   warp 17     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
-//               kind::i8 into one of three TMEM S buffers, running three key
+//               kind::i8 into one of two TMEM S buffers, running two key
 //               blocks ahead of P V; P V with the P codes read straight from
-//               TMEM (aliasing the first 32 columns of the S buffer they came
-//               from) into a TMEM int32 block; owns the TMEM allocation
-//               (S0..S2: 3 x 128 columns, P V block: d columns).
+//               TMEM (aliasing columns of the S buffer they came from) into
+//               one of two TMEM int32 blocks; owns the TMEM allocation
+//               (S0, S1: 2 x 128 columns; P V blocks: 2 x 128 columns).
 //   warps 8-11  "prep" (one thread per query row): S row -> v = S s_K in
 //               fp32 (written back over S in TMEM), causal / ragged mask,
 //               running max m and alpha.
@@ -60,7 +60,8 @@ constexpr int BM = 128;                       // query rows per CTA
 constexpr int BN = 128;                       // keys per block
 constexpr int NS = 5;                         // K/V ring depth
 constexpr int kThreads = 640;                 // 20 warps = 5 warpgroups
-constexpr int SB = 3;                         // TMEM S buffers
+constexpr int SB = 2;                         // TMEM S buffers
+constexpr int OB = 2;                         // TMEM P V blocks
 // Register split (setmaxnreg): launched with kLaunchRegs per thread (checked
 // on the host before every launch); the output warpgroup, which holds a
 // d-column fp32 row, takes registers from the other three.  The shares add up
@@ -146,7 +147,7 @@ struct alignas(1024) AttnSmem {
     uint64_t x_full[SB][4];     // prep warp k -> exp warp k (same TMEM lane quadrant)
     uint64_t a_full[2][4];      // prep warp k -> output warp k
     uint64_t a_empty[2][4];     // output warp k -> prep warp k
-    uint64_t o_full, o_empty;
+    uint64_t o_full[OB], o_empty[OB];
     uint64_t l_full, mma_drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -215,8 +216,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_init(&sm.a_full[b][k], 32);
                 mbar_init(&sm.a_empty[b][k], 32);
             }
-        mbar_init(&sm.o_full, 1);
-        mbar_init(&sm.o_empty, BM);
+        for (int b = 0; b < OB; ++b) {
+            mbar_init(&sm.o_full[b], 1);
+            mbar_init(&sm.o_empty[b], BM);
+        }
         mbar_init(&sm.l_full, 2 * BM);
         mbar_init(&sm.mma_drain, 1);
         sm.abort_flag = 0;
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
     const uint32_t tS = tbase;              // S buffer s at column 128 s
-    const uint32_t tO = tbase + 128 * SB;   // int32 P V block, D columns
+    const uint32_t tO = tbase + 128 * SB;   // int32 P V block o at column tO + 128 o
 
     if (warp >= 16) {
       regs_to<kRegsOther>();
@@ -303,14 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int sb = j % SB, st = j % NS;
             if (!warp_wait(&sm.p_full[sb], (j / SB) & 1, abort_flag, 3)) return false;
             if (!warp_wait(&sm.v_full[st], (j / NS) & 1, abort_flag, 4)) return false;
-            if (j >= 1 && !warp_wait(&sm.o_empty, (j - 1) & 1, abort_flag, 5)) return false;
+            // P V block j & 1 held block j - 2: its output fold is done
+            if (j >= OB && !warp_wait(&sm.o_empty[j % OB], ((j / OB) - 1) & 1, abort_flag, 5)) return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
 #pragma unroll
                 for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k..: see the exp warps
-                    mma_i8_ts(tO, tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k, idesc_pv, k > 0);
-                mma_commit(&sm.o_full);
+                    mma_i8_ts(tO + 128 * (j % OB), tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k,
+                              idesc_pv, k > 0);
+                mma_commit(&sm.o_full[j % OB]);
                 mma_commit(&sm.kv_empty[st]);
             }
             __syncwarp();
@@ -319,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // Q K^T runs SB blocks ahead of P V: Q K^T of block j + SB reuses the
         // S buffer of block j and is issued after P V of block j, which the
-        // tensor pipe executes first.
+        // tensor pipe executes first.  P V alternates between OB blocks, so
+        // the output fold of block j overlaps P V of block j + 1.
         for (int j = 0; ok && j < SB && j < nb; ++j) ok = issue_qk(j);
         for (int j = 0; ok && j < nb; ++j) {
             if (!issue_pv(j)) { ok = false; break; }
@@ -483,7 +489,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int ab = j & 1;
             // o = alpha o + (P V block), the int32 block turned into fp32
             // exactly (|x| <= 127^2 128 < 2^24)
-            if (!warp_wait(&sm.o_full, j & 1, abort_flag, 9)) { ok = false; break; }
+            const uint32_t to = tO + 128 * (j % OB);
+            if (!warp_wait(&sm.o_full[j % OB], (j / OB) & 1, abort_flag, 9)) { ok = false; break; }
             if (!warp_wait(&sm.a_full[ab][quad], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
             tc_fence_after();
             const float alpha = sm.alpha_o[ab][row];
@@ -492,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t w[32];
-                tmem_ld32(tO + lane_off + 32 * ch, w);
+                tmem_ld32(to + lane_off + 32 * ch, w);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -502,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&sm.o_empty);
+            mbar_arrive(&sm.o_empty[j % OB]);
         }
         if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11) && qi < L) {
             const float l = sm.lsum[0][row] + sm.lsum[1][row];
