@@ -14,9 +14,9 @@
 // exp is evaluated as exp2 with log2(e) folded into the per-row constant.
 //
 // B200 design (one CTA per 128-query tile of one (b, h); 20 warps):
-//   warp 16     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
+//   role 16     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
 //               block's s_K values into a 5-stage shared-memory ring.
-//   warp 17     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
+//   role 17     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
 //               kind::i8 into one of two TMEM S buffers, running two key
 //               blocks ahead of P V; P V with the P codes read straight from
 //               TMEM (aliasing columns of the S buffer they came from) into
@@ -33,7 +33,8 @@
 //               query row and half of the 128 keys): reads v in 32-column
 //               chunks, p = 2^(c v - c m), the row sum, and the P codes,
 //               which it writes back to TMEM as the A operand of P V.
-//   warps 18-19 idle.
+//   roles 18-19 idle.
+// Roles 16-19 run on hardware warps 0-3, roles 0-15 on hardware warps 4-19.
 // All per-row loops walk the row in 32-column chunks (one TMEM load each) and
 // are not unrolled across chunks, which keeps the three code paths that share
 // an SM sub-partition small enough for its instruction cache.
@@ -185,8 +186,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __half *__restrict__ O, int BH, int L, int causal) {
     AttnSmem<D> &sm = get_smem<D>();
     const int tid = threadIdx.x;
-    const int warp = tid >> 5;
     const int lane = tid & 31;
+    // Role numbering: the producer / MMA warpgroup (roles 16-19) runs on the
+    // lowest hardware warps 0-3, which the warp schedulers favour, so that the
+    // issue of tensor-core work is not queued behind the compute warps.  A
+    // role keeps its hardware warp's TMEM lane quadrant (role = warp - 4 mod 4).
+    const int hw_warp = tid >> 5;
+    const int warp = hw_warp < 4 ? hw_warp + 16 : hw_warp - 4;
+    const int rtid = 32 * warp + lane;
 
     const int ntiles = (L + BM - 1) / BM;
     // Head-major order: the CTAs resident together mostly share one head's
@@ -288,48 +295,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = warp_wait(&sm.q_full, 0, abort_flag, 2);
         tc_fence_after();
 
-        auto issue_qk = [&](int j) -> bool {
+        auto mma_qk = [&](int j) {   // lane 0 only; K tile of block j has landed
             const int st = j % NS, sb = j % SB;
-            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 6)) return false;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
+            const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
 #pragma unroll
-                for (int k = 0; k < D / 32; ++k)
-                    mma_i8_ss(tS + sb * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
-                mma_commit(&sm.s_full[sb]);
-            }
-            __syncwarp();
-            return true;
+            for (int k = 0; k < D / 32; ++k)
+                mma_i8_ss(tS + sb * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
+            mma_commit(&sm.s_full[sb]);
         };
-        auto issue_pv = [&](int j) -> bool {
+        auto mma_pv = [&](int j) {   // lane 0 only; P codes and V tile of block j ready
             const int sb = j % SB, st = j % NS;
-            if (!warp_wait(&sm.p_full[sb], (j / SB) & 1, abort_flag, 3)) return false;
-            if (!warp_wait(&sm.v_full[st], (j / NS) & 1, abort_flag, 4)) return false;
-            // P V block j & 1 held block j - 2: its output fold is done
-            if (j >= OB && !warp_wait(&sm.o_empty[j % OB], ((j / OB) - 1) & 1, abort_flag, 5)) return false;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
+            const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
 #pragma unroll
-                for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k..: see the exp warps
-                    mma_i8_ts(tO + 128 * (j % OB), tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k,
-                              idesc_pv, k > 0);
-                mma_commit(&sm.o_full[j % OB]);
-                mma_commit(&sm.kv_empty[st]);
-            }
-            __syncwarp();
-            return true;
+            for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k..: see the exp warps
+                mma_i8_ts(tO + 128 * (j % OB), tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k,
+                          idesc_pv, k > 0);
+            mma_commit(&sm.o_full[j % OB]);
+            mma_commit(&sm.kv_empty[st]);
         };
 
         // Q K^T runs SB blocks ahead of P V: Q K^T of block j + SB reuses the
-        // S buffer of block j and is issued after P V of block j, which the
-        // tensor pipe executes first.  P V alternates between OB blocks, so
-        // the output fold of block j overlaps P V of block j + 1.
-        for (int j = 0; ok && j < SB && j < nb; ++j) ok = issue_qk(j);
+        // S buffer of block j and is issued right after P V of block j, which
+        // the tensor pipe executes first.  P V alternates between OB blocks, so
+        // the output fold of block j overlaps P V of block j + 1.  Waits that
+        // are normally already satisfied come before the one that gates P V
+        // (the P codes), so that only the MMA issue follows it.
+        for (int j = 0; ok && j < SB && j < nb; ++j) {
+            if (!warp_wait(&sm.k_full[j % NS], (j / NS) & 1, abort_flag, 6)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) mma_qk(j);
+            __syncwarp();
+        }
         for (int j = 0; ok && j < nb; ++j) {
-            if (!issue_pv(j)) { ok = false; break; }
-            if (j + SB < nb && !issue_qk(j + SB)) { ok = false; break; }
+            const int jq = j + SB;
+            if (!warp_wait(&sm.v_full[j % NS], (j / NS) & 1, abort_flag, 4)) { ok = false; break; }
+            // P V block j % OB held block j - OB: its output fold is done
+            if (j >= OB && !warp_wait(&sm.o_empty[j % OB], ((j / OB) - 1) & 1, abort_flag, 5)) { ok = false; break; }
+            if (jq < nb && !warp_wait(&sm.k_full[jq % NS], (jq / NS) & 1, abort_flag, 6)) { ok = false; break; }
+            if (!warp_wait(&sm.p_full[j % SB], (j / SB) & 1, abort_flag, 3)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                mma_pv(j);
+                if (jq < nb) mma_qk(jq);
+            }
+            __syncwarp();
         }
         // Drain: every MMA this warp issued has completed before TMEM is freed.
         if (lane == 0) mma_commit(&sm.mma_drain);
@@ -400,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < 12) {
         regs_to<kRegsPrep>();
         // ------------------------------------------------------ prep ---
-        const int row = tid - 256;
+        const int row = rtid - 256;
         const int qi = q0 + row;
         const int quad = warp - 8;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
@@ -477,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         regs_to<kRegsOutput>();
         // ------------------------------------------------ output side ---
-        const int row = tid - 384;
+        const int row = rtid - 384;
         const int qi = q0 + row;
         const int quad = warp - 12;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
