@@ -36,9 +36,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def kernel_sources_sha() -> str:
+    """Hash of the attention kernel's sources (the dominant kernel)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_quantized_attention_token_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in ("attention.cu", "ptx.cuh"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -126,6 +127,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The max of x over all ranks of the default process group (x itself
+    when there is none): every timing is reported as the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # --------------------------------------------------------------- GPU arm ---
 
 def run_gpu(args):
@@ -206,10 +219,7 @@ def run_gpu(args):
     attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
     if intfa.intfa_device_status(clear=True) != 0:
         raise RuntimeError("a kernel timed out during the timed region")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
     ms_per_step = elapsed_ms / args.steps
     value = w.ops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
@@ -237,10 +247,7 @@ def run_gpu(args):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, dev)
         nbytes = B * H * L * d * 2
         e2e = {"value": w.ops * world * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
