@@ -92,6 +92,32 @@ int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int64_t rows, i
                               size_t workspace_bytes, void *stream);
 
 /*
+ * Per-tensor quantisation without any device allocation.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory themselves and therefore cannot supply the workspace that
+ * intfa_quantize_per_tensor needs -- for instance a plug-in running inside a
+ * host application whose memory pool owns all device memory, or a
+ * latency-critical caller that must not take the device-wide synchronisation
+ * of cudaMalloc / cudaFree.
+ *
+ * Same arguments, results and layout rules as intfa_quantize_per_tensor
+ * (bit-identical output), minus the workspace.  The per-group scratch is a
+ * fixed array of INTFA_NOALLOC_MAX_GROUPS 32-bit words (16 KiB) compiled into
+ * the library; every GPU that loads the library holds it until the process
+ * exits.  groups > INTFA_NOALLOC_MAX_GROUPS returns INTFA_ERR_UNSUPPORTED
+ * before touching the device.  The first call on each device looks up the
+ * array's device address (a one-time set-up, which may load the module); make
+ * that first call before any stream capture.  All calls share the one array:
+ * the call clears what it needs before use, but calls that overlap on the GPU
+ * (on different streams, or from several threads without ordering) race on it
+ * and give wrong results -- serialise them.  Nothing here calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ */
+#define INTFA_NOALLOC_MAX_GROUPS 4096
+int intfa_quantize_per_tensor_noalloc(const void *x_f16, int64_t groups, int64_t rows, int cols,
+                                      int transpose, int8_t *x_q, float *scale, void *stream);
+
+/*
  * Fused INT8 attention forward pass (INT-FlashAttention abstract; IntAttention
  * eqs. 4-6, section 3.2 and eq. 5; FlashAttention-3's block-wise online
  * softmax), one kernel:

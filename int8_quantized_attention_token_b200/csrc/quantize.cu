@@ -17,6 +17,8 @@
 // rounding the IEEE quotient, at one multiply per element.
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "internal.h"
 
 namespace intfa {
@@ -289,5 +291,63 @@ extern "C" int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int6
         (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
         return INTFA_ERR_MISALIGNED;
     return launch_quantize_per_tensor(x_f16, groups, rows, cols, transpose, x_q, scale, workspace,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------- per tensor, no allocation ---
+//
+// For callers that cannot allocate device memory themselves (see
+// intfa_quantize_per_tensor_noalloc in include/intfa.h): the per-group abs-max
+// scratch of the per-tensor quantiser lives in this file-scope device array
+// instead of a caller workspace.  Every GPU that loads the library holds it
+// until the process exits.  Host code must not pass the symbol itself to a
+// kernel (on the host it only names a stand-in); its device address is looked
+// up once per device with cudaGetSymbolAddress and cached.
+
+static __device__ __align__(256) unsigned g_noalloc_amax[INTFA_NOALLOC_MAX_GROUPS];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_amax on the current device (set-up on first use).
+int noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return intfa::cuda_status(cudaErrorInvalidDevice);
+    if (dev < 0 || dev >= kMaxDevices) return INTFA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_amax);
+        if (e != cudaSuccess || p == nullptr) return intfa::cuda_status(e == cudaSuccess ? cudaErrorUnknown : e);
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return INTFA_OK;
+}
+
+}  // namespace
+
+extern "C" int intfa_quantize_per_tensor_noalloc(const void *x_f16, int64_t groups, int64_t rows,
+                                                 int cols, int transpose, int8_t *x_q, float *scale,
+                                                 void *stream) {
+    using namespace intfa;
+    if (groups < 0 || rows < 0 || cols <= 0) return INTFA_ERR_INVALID_ARG;
+    if (transpose != 0 && transpose != 1) return INTFA_ERR_INVALID_ARG;
+    if (cols % 8 != 0) return INTFA_ERR_UNSUPPORTED;
+    if (transpose && cols > 256) return INTFA_ERR_UNSUPPORTED;
+    if (groups > INTFA_NOALLOC_MAX_GROUPS) return INTFA_ERR_UNSUPPORTED;   // beyond the built-in scratch
+    if (groups == 0 || rows == 0) return INTFA_OK;
+    if (rows > (INT64_MAX / 4) / cols / groups) return INTFA_ERR_INVALID_ARG;
+    if (!x_f16 || !x_q || !scale) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(x_f16) || !aligned16(x_q) || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return INTFA_ERR_MISALIGNED;
+    void *scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    // The launcher clears the scratch (cudaMemsetAsync) before the abs-max pass.
+    return launch_quantize_per_tensor(x_f16, groups, rows, cols, transpose, x_q, scale, scratch,
                                       static_cast<cudaStream_t>(stream));
 }

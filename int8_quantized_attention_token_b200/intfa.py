@@ -47,6 +47,7 @@ def lib():
         "intfa_quantize_per_tensor_workspace_size": ([I64], SZ),
         "intfa_vt_ld": ([I64], I64),
         "intfa_quantize_per_tensor": ([P, I64, I64, I, I, P, P, P, SZ, P], I),
+        "intfa_quantize_per_tensor_noalloc": ([P, I64, I64, I, I, P, P, P], I),
         "intfa_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
         "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
         "intfa_forward_workspace_size": ([I, I, I, I], SZ),
@@ -137,6 +138,28 @@ def intfa_quantize_per_tensor(x: torch.Tensor, transpose: bool = False, x_q=None
     _check(lib().intfa_quantize_per_tensor(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
                                            _ptr(scale), _ptr(workspace), workspace.numel(),
                                            _stream(stream)), "intfa_quantize_per_tensor")
+    return x_q, scale
+
+
+def intfa_quantize_per_tensor_noalloc(x: torch.Tensor, transpose: bool = False, x_q=None, scale=None,
+                                      stream=None):
+    """intfa_quantize_per_tensor without a workspace, for callers that cannot
+    allocate device memory: the scratch is a fixed array inside the library
+    (at most INTFA_NOALLOC_MAX_GROUPS = 4096 groups).  Calls that overlap on
+    the GPU race on that array; the first call on a device does a one-time
+    set-up and should come before any stream capture.  (This wrapper itself
+    allocates outputs with torch when x_q / scale are not given.)"""
+    _need(x, torch.float16, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [groups, rows, cols]")
+    g, rows, cols = x.shape
+    if x_q is None:
+        shape = (g, cols, intfa_vt_ld(rows)) if transpose else (g, rows, cols)
+        x_q = torch.empty(shape, dtype=torch.int8, device=x.device)
+    scale = torch.empty((g,), dtype=torch.float32, device=x.device) if scale is None else scale
+    _check(lib().intfa_quantize_per_tensor_noalloc(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
+                                                   _ptr(scale), _stream(stream)),
+           "intfa_quantize_per_tensor_noalloc")
     return x_q, scale
 
 
