@@ -9,12 +9,22 @@
 //
 // Rounding contract (bit-exact with the definition): s = fl32(amax / 127)
 // by an IEEE division; the code is RNE(fl32(x / s)) clamped to +-127.  The
-// per-element quotient is formed as y = x * fl32(1 / s) (IEEE reciprocal):
-// |y - x/s| <= |x/s| 2^-23 <= 1.6e-5 and |fl32(x/s) - x/s| <= 7.6e-6, so y
-// and fl32(x/s) round to the same integer unless x/s lies within ~2.4e-5 of
-// a half-integer; when y is within 1e-3 of one, the IEEE quotient
-// __fdiv_rn(x, s) is used instead.  The result is therefore identical to
-// rounding the IEEE quotient, at one multiply per element.
+// per-element quotient is formed as y = x * r with r = rcp.approx(s)
+// (relative error <= 2^-23): |y - x/s| <= 127 (2^-23 + 2^-24) <= 2.3e-5 and
+// |fl32(x/s) - x/s| <= 7.6e-6, so y and fl32(x/s) round to the same integer
+// unless x/s lies within ~3.1e-5 of a half-integer; when y is within 1e-3 of
+// one, the IEEE quotient __fdiv_rn(x, s) is used instead.  The result is
+// therefore identical to rounding the IEEE quotient, at one multiply per
+// element.
+// The scale fl32(amax / 127) is formed with Markstein's correction (P.
+// Markstein, "IA-64 and Elementary Functions", 2000): q0 = amax * c with
+// c = fl32(1/127), residual r = fma(-q0, 127, amax) (exact), q = fma(r, c, q0).
+// amax is always an fp16 magnitude; the GPU tests check q against the IEEE
+// quotient for every finite fp16 value.
+// RNE itself is fl(y + 1.5 * 2^23): for |y| < 2^22 that float is
+// 1.5 * 2^23 + RNE(y) exactly, so its low byte is the code in two's complement
+// and y - (t - 1.5 * 2^23) is the exact rounding residual.  |fl32(x/s)| never
+// exceeds 127.00002, so the +-127 clamp never binds.
 #include <cuda_fp16.h>
 
 #include <mutex>
@@ -24,14 +34,37 @@
 namespace intfa {
 namespace {
 
-__device__ __forceinline__ int quant_code(float x, float s, float r) {
-    float y = x * r;
-    const float f = y - floorf(y);
-    if (fabsf(f - 0.5f) < 1e-3f) y = __fdiv_rn(x, s);
-    int c = __float2int_rn(y);
-    c = c > 127 ? 127 : c;
-    c = c < -127 ? -127 : c;
-    return c;
+constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+
+// fl32(a / 127) for fp16 magnitudes a (see the header comment).
+__device__ __forceinline__ float div127(float a) {
+    const float c = 1.0f / 127.0f;
+    const float q0 = a * c;
+    const float r = fmaf(-q0, 127.0f, a);
+    return fmaf(r, c, q0);
+}
+
+// Approximate 1 / s (relative error <= 2^-23); 0 for s == 0.
+__device__ __forceinline__ float rcp_or_zero(float s) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return s != 0.0f ? r : 0.0f;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// The code of x as the low byte of a float's bit pattern (see above); s == 0
+// (r == 0) gives code 0.
+__device__ __forceinline__ uint32_t code_bits(float x, float s, float r) {
+    const float y = x * r;
+    float t = y + kRound;
+    const float res = y - (t - kRound);
+    if (fabsf(res) > 0.499f) t = __fdiv_rn(x, s) + kRound;
+    return __float_as_uint(t);
 }
 
 __device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
@@ -51,21 +84,21 @@ __device__ __forceinline__ float absmax8(const float (&f)[8]) {
     return m;
 }
 
+// 8 codes packed little-endian into two words.
 __device__ __forceinline__ uint2 codes8(const float (&f)[8], float s, float r) {
-    uint32_t w[2] = {0u, 0u};
-    if (s != 0.0f) {
+    uint32_t t[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t c = static_cast<uint32_t>(quant_code(f[i], s, r)) & 0xFFu;
-            w[i >> 2] |= c << (8 * (i & 3));
-        }
-    }
-    return make_uint2(w[0], w[1]);
+    for (int i = 0; i < 8; ++i) t[i] = code_bits(f[i], s, r);
+    return make_uint2(prmt(prmt(t[0], t[1], 0x0040u), prmt(t[2], t[3], 0x0040u), 0x5410u),
+                      prmt(prmt(t[4], t[5], 0x0040u), prmt(t[6], t[7], 0x0040u), 0x5410u));
 }
 
 // ------------------------------------------------------------ per token ---
 
-// G lanes cover one row of d = 8 G values; a warp holds 32 / G rows.
+// G lanes cover one row of d = 8 G values; a warp holds 32 / G rows per
+// slice and handles kSlices slices per iteration, issuing all their 16-byte
+// loads before any arithmetic (more bytes in flight per thread).
+constexpr int kSlices = 4;
 template <int G>
 __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint4 *__restrict__ x,
                                                               int64_t rows,
@@ -76,25 +109,28 @@ __global__ void __launch_bounds__(256) quant_per_token_kernel(const uint4 *__res
     constexpr int kRowsPerWarp = 32 / G;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-    for (int64_t r0 = warp * kRowsPerWarp; r0 < rows; r0 += nwarps * kRowsPerWarp) {
-        const int64_t r = r0 + lane / G;
-        const bool valid = r < rows;
-        float f[8];
-        if (valid) {
-            const uint4 v = __ldcs(x + r * G + sub);
-            unpack8(v, f);
-        } else {
+    const int64_t step = nwarps * kRowsPerWarp;
+    for (int64_t r0 = warp * kRowsPerWarp; r0 < rows; r0 += kSlices * step) {
+        uint4 v[kSlices];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = 0.0f;
+        for (int k = 0; k < kSlices; ++k) {
+            const int64_t r = r0 + k * step + lane / G;
+            v[k] = r < rows ? __ldcs(x + r * G + sub) : make_uint4(0u, 0u, 0u, 0u);
         }
-        float amax = absmax8(f);
 #pragma unroll
-        for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        const float s = __fdiv_rn(amax, 127.0f);
-        const float rcp = s != 0.0f ? __frcp_rn(s) : 0.0f;
-        if (valid) {
-            __stcs(xq + r * G + sub, codes8(f, s, rcp));
-            if (sub == 0) scale[r] = s;
+        for (int k = 0; k < kSlices; ++k) {
+            const int64_t r = r0 + k * step + lane / G;
+            float f[8];
+            unpack8(v[k], f);
+            float amax = absmax8(f);
+#pragma unroll
+            for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+            const float s = div127(amax);
+            const float rcp = rcp_or_zero(s);
+            if (r < rows) {
+                __stcs(xq + r * G + sub, codes8(f, s, rcp));
+                if (sub == 0) scale[r] = s;
+            }
         }
     }
 }
@@ -132,8 +168,8 @@ __global__ void __launch_bounds__(256) group_convert_kernel(const uint4 *__restr
                                                             uint2 *__restrict__ xq,
                                                             float *__restrict__ scale) {
     const int g = blockIdx.y;
-    const float s = __fdiv_rn(__uint_as_float(ws[g]), 127.0f);
-    const float rcp = s != 0.0f ? __frcp_rn(s) : 0.0f;
+    const float s = div127(__uint_as_float(ws[g]));
+    const float rcp = rcp_or_zero(s);
     if (blockIdx.x == 0 && threadIdx.x == 0) scale[g] = s;
     const uint4 *xg = x + static_cast<int64_t>(g) * n8;
     uint2 *qg = xq + static_cast<int64_t>(g) * n8;
@@ -145,44 +181,65 @@ __global__ void __launch_bounds__(256) group_convert_kernel(const uint4 *__restr
     }
 }
 
-// Phase 2, transposed: group g of [rows][cols] -> [cols][ld], 64 rows per
-// block staged through shared memory; rows in [rows, ld) get code 0.
-constexpr int kTRows = 64;
+// Phase 2, transposed: group g of [rows][cols] -> [cols][ld]; rows in
+// [rows, ld) get code 0.  A block covers kTRG row groups of 4 rows: thread
+// (rg, c8) loads rows 4 rg .. 4 rg + 3 of columns 8 c8 .. 8 c8 + 7 (16-byte
+// coalesced loads), packs the 4 codes of each column into one 32-bit word and
+// stores the 8 words to shared memory, column-major with a one-word pad and a
+// per-thread rotation of the column order (bank-conflict-light); the block then
+// writes each column's 4 kTRG bytes with 16-byte stores.
+constexpr int kTRG = 16;              // row groups of 4 per block (64 rows)
+constexpr int kTRows = 4 * kTRG;
 __global__ void __launch_bounds__(256) group_convert_t_kernel(const uint4 *__restrict__ x,
                                                               int64_t rows, int cols, int64_t ld,
                                                               const unsigned *__restrict__ ws,
                                                               int8_t *__restrict__ xq,
                                                               float *__restrict__ scale) {
-    __shared__ __align__(16) uint8_t tile[256 * kTRows];  // [col][row]
+    __shared__ uint32_t tile[256 * (kTRG + 1)];   // [col][row group], padded
     const int g = blockIdx.y;
     const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kTRows;
-    const float s = __fdiv_rn(__uint_as_float(ws[g]), 127.0f);
-    const float rcp = s != 0.0f ? __frcp_rn(s) : 0.0f;
+    const float s = div127(__uint_as_float(ws[g]));
+    const float rcp = rcp_or_zero(s);
     if (blockIdx.x == 0 && threadIdx.x == 0) scale[g] = s;
     const int c8n = cols >> 3;
     const uint4 *xg = x + static_cast<int64_t>(g) * rows * c8n;
-    for (int i = threadIdx.x; i < kTRows * c8n; i += blockDim.x) {
-        const int row = i / c8n, c8 = i - row * c8n;
-        uint2 w = make_uint2(0u, 0u);
-        if (r0 + row < rows) {
-            float f[8];
-            unpack8(__ldcs(xg + (r0 + row) * c8n + c8), f);
-            w = codes8(f, s, rcp);
-        }
+    for (int t = threadIdx.x; t < kTRG * c8n; t += blockDim.x) {
+        const int c8 = t % c8n, rg = t / c8n;
+        uint2 w[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const uint32_t word = e < 4 ? w.x : w.y;
-            tile[(c8 * 8 + e) * kTRows + row] = static_cast<uint8_t>(word >> (8 * (e & 3)));
+        for (int k = 0; k < 4; ++k) {
+            const int64_t r = r0 + 4 * rg + k;
+            w[k] = make_uint2(0u, 0u);
+            if (r < rows) {
+                float f[8];
+                unpack8(__ldcs(xg + r * c8n + c8), f);
+                w[k] = codes8(f, s, rcp);
+            }
+        }
+        // column e's word = byte e of rows 0..3 (PRMT selects byte e of
+        // the first and byte e of the second source, then interleaves)
+        uint32_t col[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t sel = static_cast<uint32_t>(e | ((e + 4) << 4));
+            col[e] = prmt(prmt(w[0].x, w[1].x, sel), prmt(w[2].x, w[3].x, sel), 0x5410u);
+            col[e + 4] = prmt(prmt(w[0].y, w[1].y, sel), prmt(w[2].y, w[3].y, sel), 0x5410u);
+        }
+        const int rot = (c8 >> 2) & 7;
+#pragma unroll
+        for (int e0 = 0; e0 < 8; ++e0) {
+            const int e = (e0 + rot) & 7;
+            tile[(8 * c8 + e) * (kTRG + 1) + rg] = col[e];
         }
     }
     __syncthreads();
     int8_t *qg = xq + static_cast<int64_t>(g) * cols * ld;
-    for (int j = threadIdx.x; j < cols * (kTRows / 16); j += blockDim.x) {
-        const int c = j >> 2, part = j & 3;
-        const int64_t rr = r0 + part * 16;
+    for (int j = threadIdx.x; j < cols * (kTRG / 4); j += blockDim.x) {
+        const int c = j / (kTRG / 4), part = j % (kTRG / 4);
+        const int64_t rr = r0 + 16 * part;
         if (rr < ld) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(tile + c * kTRows + part * 16);
-            __stcs(reinterpret_cast<uint4 *>(qg + c * ld + rr), v);
+            const uint32_t *src = &tile[c * (kTRG + 1) + 4 * part];
+            __stcs(reinterpret_cast<uint4 *>(qg + c * ld + rr), make_uint4(src[0], src[1], src[2], src[3]));
         }
     }
 }

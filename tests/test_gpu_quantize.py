@@ -72,3 +72,24 @@ def test_full_size_quantisation_bit_exact(w):
     qo, so = oracle.quantize_per_tensor(Vg.float().numpy(), w.B * w.H)
     np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
     np.testing.assert_array_equal(q.cpu().numpy()[:, :, : w.L].transpose(0, 2, 1), qo)
+
+
+def test_scale_of_every_fp16_magnitude():
+    """Rows whose abs-max runs over every finite fp16 magnitude: scales and
+    codes equal the oracle's IEEE fp32 results bit for bit."""
+    mags = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    n = mags.size
+    rng = np.random.default_rng(9)
+    frac = rng.uniform(-1, 1, (n, 7)).astype(np.float32)
+    x = np.concatenate([mags[:, None], (frac * mags[:, None])], axis=1).astype(np.float16)
+    xt = torch.from_numpy(x)
+    q, s = intfa.intfa_quantize_per_token(xt.cuda())
+    qo, so = oracle.quantize_per_token(x.astype(np.float32))
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    # the same magnitudes as per-tensor abs-maxes
+    g = x[:, None, :8].repeat(1, axis=1).reshape(n, 1, 8)
+    q2, s2 = intfa.intfa_quantize_per_tensor(torch.from_numpy(np.ascontiguousarray(g)).cuda(), transpose=True)
+    qo2, so2 = oracle.quantize_per_tensor(g.astype(np.float32), n)
+    np.testing.assert_array_equal(s2.cpu().numpy().view(np.uint32), so2.view(np.uint32))
+    np.testing.assert_array_equal(q2.cpu().numpy()[:, :, :1].transpose(0, 2, 1), qo2)
