@@ -96,42 +96,38 @@ __device__ __forceinline__ uint2 codes8(const float (&f)[8], float s, float r) {
 // ------------------------------------------------------------ per token ---
 
 // G lanes cover one row of d = 8 G values; a warp holds 32 / G rows per
-// slice and handles kSlices slices per iteration, issuing all their 16-byte
-// loads before any arithmetic (more bytes in flight per thread).
-constexpr int kSlices = 4;
+// slice and strides over the rows by the whole grid.  Each thread issues the
+// 16-byte load of its next slice before the arithmetic on the current one, so
+// two loads per thread are in flight (six 256-thread blocks per SM).
 template <int G>
-__global__ void __launch_bounds__(256) quant_per_token_kernel(const uint4 *__restrict__ x,
-                                                              int64_t rows,
-                                                              uint2 *__restrict__ xq,
-                                                              float *__restrict__ scale) {
+__global__ void __launch_bounds__(256, 6) quant_per_token_kernel(const uint4 *__restrict__ x,
+                                                                 int64_t rows,
+                                                                 uint2 *__restrict__ xq,
+                                                                 float *__restrict__ scale) {
     const int lane = threadIdx.x & 31;
     const int sub = lane & (G - 1);
     constexpr int kRowsPerWarp = 32 / G;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int64_t step = nwarps * kRowsPerWarp;
-    for (int64_t r0 = warp * kRowsPerWarp; r0 < rows; r0 += kSlices * step) {
-        uint4 v[kSlices];
+    int64_t r = warp * kRowsPerWarp + lane / G;
+    uint4 v = r < rows ? __ldcs(x + r * G + sub) : make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t r0 = warp * kRowsPerWarp; r0 < rows; r0 += step) {
+        const int64_t rn = r + step;
+        const uint4 vn = rn < rows ? __ldcs(x + rn * G + sub) : make_uint4(0u, 0u, 0u, 0u);
+        float f[8];
+        unpack8(v, f);
+        float amax = absmax8(f);
 #pragma unroll
-        for (int k = 0; k < kSlices; ++k) {
-            const int64_t r = r0 + k * step + lane / G;
-            v[k] = r < rows ? __ldcs(x + r * G + sub) : make_uint4(0u, 0u, 0u, 0u);
+        for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        const float s = div127(amax);
+        const float rcp = rcp_or_zero(s);
+        if (r < rows) {
+            __stcs(xq + r * G + sub, codes8(f, s, rcp));
+            if (sub == 0) scale[r] = s;
         }
-#pragma unroll
-        for (int k = 0; k < kSlices; ++k) {
-            const int64_t r = r0 + k * step + lane / G;
-            float f[8];
-            unpack8(v[k], f);
-            float amax = absmax8(f);
-#pragma unroll
-            for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-            const float s = div127(amax);
-            const float rcp = rcp_or_zero(s);
-            if (r < rows) {
-                __stcs(xq + r * G + sub, codes8(f, s, rcp));
-                if (sub == 0) scale[r] = s;
-            }
-        }
+        r = rn;
+        v = vn;
     }
 }
 
@@ -190,7 +186,7 @@ __global__ void __launch_bounds__(256) group_convert_kernel(const uint4 *__restr
 // writes each column's 4 kTRG bytes with 16-byte stores.
 constexpr int kTRG = 16;              // row groups of 4 per block (64 rows)
 constexpr int kTRows = 4 * kTRG;
-__global__ void __launch_bounds__(256) group_convert_t_kernel(const uint4 *__restrict__ x,
+__global__ void __launch_bounds__(256, 6) group_convert_t_kernel(const uint4 *__restrict__ x,
                                                               int64_t rows, int cols, int64_t ld,
                                                               const unsigned *__restrict__ ws,
                                                               int8_t *__restrict__ xq,
