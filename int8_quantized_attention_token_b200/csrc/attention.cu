@@ -61,8 +61,9 @@ constexpr int BM = 128;                       // query rows per CTA
 constexpr int BN = 128;                       // keys per block
 constexpr int NS = 5;                         // K/V ring depth
 constexpr int kThreads = 640;                 // 20 warps = 5 warpgroups
-constexpr int SB = 2;                         // TMEM S buffers
-constexpr int OB = 2;                         // TMEM P V blocks
+constexpr int SB = 3;                         // TMEM S buffers
+constexpr int OB = 1;                         // TMEM P V blocks
+constexpr int AB = 4;                         // alpha ring depth (prep -> output side)
 // Register split (setmaxnreg): launched with kLaunchRegs per thread (checked
 // on the host before every launch); the output warpgroup, which holds a
 // d-column fp32 row, takes registers from the other three.  The shares add up
@@ -120,6 +121,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// A non-blocking probe issued ahead of time (its latency then overlaps other
+// work); settle() only waits if some lane's probe found the phase incomplete.
+__device__ __forceinline__ bool settle(bool probed, uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                       uint32_t site) {
+    if (__all_sync(0xFFFFFFFFu, probed)) return true;
+    return warp_wait(bar, parity, abort_flag, site);
+}
+
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     const long long t0 = clock64();
@@ -140,14 +149,14 @@ struct alignas(1024) AttnSmem {
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
     float2 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha) per row and S buffer
-    float alpha_o[2][BM];       // prep -> output: alpha per row and S buffer
+    float alpha_o[AB][BM];      // prep -> output: alpha of block j (slot j mod AB)
     float lsum[2][BM];          // exp -> output: final row sums of each column half
     uint64_t q_full;
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
     uint64_t s_full[SB], p_full[SB];
     uint64_t x_full[SB][4];     // prep warp k -> exp warp k (same TMEM lane quadrant)
-    uint64_t a_full[2][4];      // prep warp k -> output warp k
-    uint64_t a_empty[2][4];     // output warp k -> prep warp k
+    uint64_t a_full[AB][4];     // prep warp k -> output warp k
+    uint64_t a_empty[AB][4];    // output warp k -> prep warp k
     uint64_t o_full[OB], o_empty[OB];
     uint64_t l_full, mma_drain;
     uint32_t tmem_base;
@@ -174,6 +183,45 @@ __device__ __forceinline__ uint8_t *smem_aligned_1024() {
 template <int D>
 __device__ __forceinline__ AttnSmem<D> &get_smem() {
     return *reinterpret_cast<AttnSmem<D> *>(smem_aligned_1024());
+}
+
+// ------------------------------------------------------- prep pieces ---
+
+// v = fl(S s_K) in place (int32 -> fp32 is exact: |S| <= 127^2 d < 2^24).
+__device__ __forceinline__ void scores_to_v(uint32_t (&w)[32], const float4 *sk4) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 k4 = sk4[q];
+        const uint64_t a = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q])),
+                                         __int2float_rn(static_cast<int32_t>(w[4 * q + 1]))),
+                                 f2_pack(k4.x, k4.y));
+        const uint64_t e = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q + 2])),
+                                         __int2float_rn(static_cast<int32_t>(w[4 * q + 3]))),
+                                 f2_pack(k4.z, k4.w));
+        float v0, v1, v2, v3;
+        f2_unpack(a, v0, v1);
+        f2_unpack(e, v2, v3);
+        w[4 * q] = __float_as_uint(v0);
+        w[4 * q + 1] = __float_as_uint(v1);
+        w[4 * q + 2] = __float_as_uint(v2);
+        w[4 * q + 3] = __float_as_uint(v3);
+    }
+}
+
+// Keys at or past lim get v = -inf.
+__device__ __forceinline__ void mask_v(uint32_t (&w)[32], int key0, int lim) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+        if (key0 + e >= lim) w[e] = __float_as_uint(-INFINITY);
+}
+
+__device__ __forceinline__ void max_v(const uint32_t (&w)[32], float (&mx)[4]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        mx[q & 3] = fmax3(mx[q & 3], __uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1]));
+        mx[(q + 2) & 3] =
+            fmax3(mx[(q + 2) & 3], __uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3]));
+    }
 }
 
 // ---------------------------------------------------------------- kernel ---
@@ -218,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.p_full[b], 2 * BM);
             for (int k = 0; k < 4; ++k) mbar_init(&sm.x_full[b][k], 32);
         }
-        for (int b = 0; b < 2; ++b)
+        for (int b = 0; b < AB; ++b)
             for (int k = 0; k < 4; ++k) {
                 mbar_init(&sm.a_full[b][k], 32);
                 mbar_init(&sm.a_empty[b][k], 32);
@@ -362,14 +410,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   (kLog2e / sqrtf(static_cast<float>(D))),
                               1e-30f);
         float l = 0.0f;
+        bool pre_x = false;   // probe of this block's x_full, taken one block early
         for (int j = 0; j < nb; ++j) {
             const int b = j % SB;
-            if (!warp_wait(&sm.x_full[b][quad], (j / SB) & 1, abort_flag, 7)) break;
+            if (!settle(pre_x, &sm.x_full[b][quad], (j / SB) & 1, abort_flag, 7)) break;
             tc_fence_after();
+            pre_x = j + 1 < nb && mbar_test_wait(&sm.x_full[(j + 1) % SB][quad], ((j + 1) / SB) & 1);
             const float2 ca = sm.cm_alpha[b][row];
             const float ncm = -ca.x;
             const uint32_t tv = tS + lane_off + b * BN + 64 * hf;
-            float ps0 = 0.0f, ps1 = 0.0f, ps2 = 0.0f, ps3 = 0.0f;
+            const uint64_t c2 = f2_pack(c, c), ncm2 = f2_pack(ncm, ncm);
+            const uint64_t k127 = f2_pack(127.0f, 127.0f), magic = f2_pack(kMagic, kMagic);
+            uint64_t ps01 = 0ull, ps23 = 0ull;
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -379,22 +431,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
-                    const float p0 = ex2(fmaf(__uint_as_float(w[4 * q]), c, ncm));
-                    const float p1 = ex2(fmaf(__uint_as_float(w[4 * q + 1]), c, ncm));
-                    const float p2 = ex2(fmaf(__uint_as_float(w[4 * q + 2]), c, ncm));
-                    const float p3 = ex2(fmaf(__uint_as_float(w[4 * q + 3]), c, ncm));
-                    ps0 += p0;
-                    ps1 += p1;
-                    ps2 += p2;
-                    ps3 += p3;
+                    float x0, x1, x2, x3;
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), c2, ncm2), x0, x1);
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2, ncm2), x2, x3);
+                    const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
+                    const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
+                    ps01 = fadd2(ps01, p01);
+                    ps23 = fadd2(ps23, p23);
                     // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
-                    const uint32_t t0 = __float_as_uint(fmaf(p0, 127.0f, kMagic));
-                    const uint32_t t1 = __float_as_uint(fmaf(p1, 127.0f, kMagic));
-                    const uint32_t t2 = __float_as_uint(fmaf(p2, 127.0f, kMagic));
-                    const uint32_t t3 = __float_as_uint(fmaf(p3, 127.0f, kMagic));
-                    pk[8 * e + q] = prmt(prmt(t0, t1, 0x0040u), prmt(t2, t3, 0x0040u), 0x5410u);
+                    float t0, t1, t2, t3;
+                    f2_unpack(ffma2(p01, k127, magic), t0, t1);
+                    f2_unpack(ffma2(p23, k127, magic), t2, t3);
+                    pk[8 * e + q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
+                                         prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
                 }
             }
+            float ps0, ps1, ps2, ps3;
+            f2_unpack(ps01, ps0, ps1);
+            f2_unpack(ps23, ps2, ps3);
             // both chunks are in registers: their columns now take the codes
             tmem_st8(tv, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
             tmem_st8(tv + 8, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
@@ -420,54 +474,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   (kLog2e / sqrtf(static_cast<float>(D))),
                               1e-30f);
         float m_old = -INFINITY;
+        // probes of this block's s_full / k_full, taken one block early
+        bool pre_s = false, pre_k = false;
         for (int j = 0; j < nb; ++j) {
             // -- block j: v = fl(S s_K) (int32 -> fp32 exact, |S| <= 127^2 d
             // < 2^24), mask, row max.
-            const int b = j % SB, ab = j & 1, st = j % NS;
-            if (!warp_wait(&sm.s_full[b], (j / SB) & 1, abort_flag, 12)) break;
+            const int b = j % SB, ab = j % AB, st = j % NS;
+            if (!settle(pre_s, &sm.s_full[b], (j / SB) & 1, abort_flag, 12)) break;
             // s_K of this block: published by the producer's release-arrive
-            if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort_flag, 13)) break;
+            if (!settle(pre_k, &sm.k_full[st], (j / NS) & 1, abort_flag, 13)) break;
             tc_fence_after();
+            const bool pre_a = j < AB || mbar_test_wait(&sm.a_empty[ab][quad], ((j / AB) - 1) & 1);
+            const int jn = j + 1;
+            pre_s = jn < nb && mbar_test_wait(&sm.s_full[jn % SB], (jn / SB) & 1);
+            pre_k = jn < nb && mbar_test_wait(&sm.k_full[jn % NS], (jn / NS) & 1);
             const uint32_t ts = tS + lane_off + b * BN;
             const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
             const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
+            const int lim = causal ? min(L, qi + 1) : L;
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
             for (int ch = 0; ch < BN / 32; ++ch) {
                 uint32_t w[32];
                 tmem_ld32(ts + 32 * ch, w);
                 tmem_wait_ld();
-                float vv[32];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 k4 = sk4[8 * ch + q];
-                    const uint64_t a = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q])),
-                                                     __int2float_rn(static_cast<int32_t>(w[4 * q + 1]))),
-                                             f2_pack(k4.x, k4.y));
-                    const uint64_t e = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q + 2])),
-                                                     __int2float_rn(static_cast<int32_t>(w[4 * q + 3]))),
-                                             f2_pack(k4.z, k4.w));
-                    f2_unpack(a, vv[4 * q], vv[4 * q + 1]);
-                    f2_unpack(e, vv[4 * q + 2], vv[4 * q + 3]);
-                }
-                if (need_mask) {
-                    // keys past the end of the sequence, or after the query
-                    // (causal), get v = -inf (p = 0)
-                    const int lim = causal ? min(L, qi + 1) : L;
-                    const int key0 = j * BN + 32 * ch;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (key0 + e >= lim) vv[e] = -INFINITY;
-                }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    mx[q & 3] = fmax3(mx[q & 3], vv[4 * q], vv[4 * q + 1]);
-                    mx[(q + 2) & 3] = fmax3(mx[(q + 2) & 3], vv[4 * q + 2], vv[4 * q + 3]);
-                    w[4 * q] = __float_as_uint(vv[4 * q]);
-                    w[4 * q + 1] = __float_as_uint(vv[4 * q + 1]);
-                    w[4 * q + 2] = __float_as_uint(vv[4 * q + 2]);
-                    w[4 * q + 3] = __float_as_uint(vv[4 * q + 3]);
-                }
+                scores_to_v(w, sk4 + 8 * ch);
+                // keys past the end of the sequence, or after the query
+                // (causal), get v = -inf (p = 0)
+                if (need_mask) mask_v(w, j * BN + 32 * ch, lim);
+                max_v(w, mx);
                 tmem_st32(ts + 32 * ch, w);
             }
             mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
@@ -475,13 +510,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
             m_old = m_new;
             sm.cm_alpha[b][row] = make_float2(c * m_new, alpha);
+            // alpha of block j -> the output warp of this quadrant
+            if (!settle(pre_a, &sm.a_empty[ab][quad], ((j / AB) - 1) & 1, abort_flag, 14)) break;
+            sm.alpha_o[ab][row] = alpha;
+            mbar_arrive(&sm.a_full[ab][quad]);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.x_full[b][quad]);
-            // alpha of block j -> the output warp of this quadrant
-            if (j >= 2 && !warp_wait(&sm.a_empty[ab][quad], ((j >> 1) - 1) & 1, abort_flag, 14)) break;
-            sm.alpha_o[ab][row] = alpha;
-            mbar_arrive(&sm.a_full[ab][quad]);
         }
     } else {
         regs_to<kRegsOutput>();
@@ -495,30 +530,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < D / 2; ++i) o2[i] = 0ull;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
-            const int ab = j & 1;
+            const int ab = j % AB;
             // o = alpha o + (P V block), the int32 block turned into fp32
             // exactly (|x| <= 127^2 128 < 2^24)
             const uint32_t to = tO + 128 * (j % OB);
             if (!warp_wait(&sm.o_full[j % OB], (j / OB) & 1, abort_flag, 9)) { ok = false; break; }
-            if (!warp_wait(&sm.a_full[ab][quad], (j >> 1) & 1, abort_flag, 10)) { ok = false; break; }
+            if (!warp_wait(&sm.a_full[ab][quad], (j / AB) & 1, abort_flag, 10)) { ok = false; break; }
             tc_fence_after();
             const float alpha = sm.alpha_o[ab][row];
             mbar_arrive(&sm.a_empty[ab][quad]);
             const uint64_t a2 = f2_pack(alpha, alpha);
+            // the block in pairs of 32-column chunks; once the last pair is
+            // in registers the P V block is released for the next block
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t w[32];
-                tmem_ld32(to + lane_off + 32 * ch, w);
+            for (int pr = 0; pr < D / 64; ++pr) {
+                uint32_t w0[32], w1[32];
+                tmem_ld32(to + lane_off + 64 * pr, w0);
+                tmem_ld32(to + lane_off + 64 * pr + 32, w1);
                 tmem_wait_ld();
+                if (pr == D / 64 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(&sm.o_empty[j % OB]);
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w[2 * i])),
-                                               __int2float_rn(static_cast<int32_t>(w[2 * i + 1])));
-                    o2[16 * ch + i] = ffma2(o2[16 * ch + i], a2, x);
+                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w0[2 * i])),
+                                               __int2float_rn(static_cast<int32_t>(w0[2 * i + 1])));
+                    o2[32 * pr + i] = ffma2(o2[32 * pr + i], a2, x);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w1[2 * i])),
+                                               __int2float_rn(static_cast<int32_t>(w1[2 * i + 1])));
+                    o2[32 * pr + 16 + i] = ffma2(o2[32 * pr + 16 + i], a2, x);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&sm.o_empty[j % OB]);
         }
         if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11) && qi < L) {
             const float l = sm.lsum[0][row] + sm.lsum[1][row];
