@@ -13,22 +13,28 @@
 //   O_i   = s_V acc_i / (127 l_i)                          -> fp16
 // exp is evaluated as exp2 with log2(e) folded into the per-row constant.
 //
-// B200 design (one CTA per 128-query tile of one (b, h); 20 warps):
-//   role 16     TMA producer: Q tile once; K_hat tile, V_hat^T tile and the
-//               block's s_K values into a 5-stage shared-memory ring.
+// B200 design: a persistent kernel, one CTA per SM, each CTA walking a fixed
+// list of 128-query tiles (tile c, c + G, c + 2G, ... of the head-major
+// order).  Every role runs through the CTA's whole stream of (tile, key
+// block) pairs with ring counters that do not restart at tile boundaries, so
+// the loads and Q K^T of the next tile overlap the last blocks and the
+// epilogue of the current one.  20 warps:
+//   role 16     TMA producer: each tile's Q_hat (two Q buffers), K_hat tile,
+//               V_hat^T tile and the block's s_K values into a 5-stage
+//               shared-memory ring.
 //   role 17     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
-//               kind::i8 into one of two TMEM S buffers, running two key
-//               blocks ahead of P V; P V with the P codes read straight from
-//               TMEM (aliasing columns of the S buffer they came from) into
-//               one of two TMEM int32 blocks; owns the TMEM allocation
-//               (S0, S1: 2 x 128 columns; P V blocks: 2 x 128 columns).
+//               kind::i8 into one of three TMEM S buffers, three key blocks
+//               ahead of P V; P V with the P codes read straight from TMEM
+//               (aliasing columns of the S buffer they came from) into the
+//               TMEM int32 P V block; owns the TMEM allocation (S0..S2: 3 x
+//               128 columns; P V block: 128 columns).
 //   warps 8-11  "prep" (one thread per query row): S row -> v = S s_K in
 //               fp32 (written back over S in TMEM), causal / ragged mask,
 //               running max m and alpha.
 //   warps 12-15 output side (one thread per query row): folds each int32
 //               P V block into the row's fp32 accumulator, held in registers
 //               (o = alpha o + block), and writes the normalised fp16 row at
-//               the end.
+//               the end of each tile.
 //   warps 0-7   "exp" (two warps per TMEM lane quadrant, each one thread per
 //               query row and half of the 128 keys): reads v in 32-column
 //               chunks, p = 2^(c v - c m), the row sum, and the P codes,
@@ -38,9 +44,6 @@
 // All per-row loops walk the row in 32-column chunks (one TMEM load each) and
 // are not unrolled across chunks, which keeps the three code paths that share
 // an SM sub-partition small enough for its instruction cache.
-// The exp warps are bound by the special-function unit (one exp2 per score);
-// the prep warps' integer/FMA work for block j+1 and the output warps'
-// update for block j-1 run beside it on the same sub-partitions.
 // Every wait is bounded (clock-based); a timeout records a status word,
 // raises a CTA-wide abort flag, drains in-flight copies and MMAs, frees TMEM
 // and returns.
@@ -69,12 +72,26 @@ constexpr int AB = 4;                         // alpha ring depth (prep -> outpu
 // d-column fp32 row, takes registers from the other three.  The shares add up
 // to at most the launch total.
 constexpr int kLaunchRegs = 96;
-constexpr uint32_t kRegsExp = 72;      // each of the two exp warpgroups
-constexpr uint32_t kRegsPrep = 96;
-constexpr uint32_t kRegsOutput = 192;
-constexpr uint32_t kRegsOther = 48;
-static_assert(128 * (2 * kRegsExp + kRegsPrep + kRegsOutput + kRegsOther) <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
+template <int D>
+struct RegSplit {   // d = 128: the output row alone is 128 registers
+    static constexpr uint32_t kExp = 72;      // each of the two exp warpgroups
+    static constexpr uint32_t kPrep = 80;
+    static constexpr uint32_t kOutput = 208;
+    static constexpr uint32_t kOther = 48;
+};
+template <>
+struct RegSplit<64> {
+    static constexpr uint32_t kExp = 72;
+    static constexpr uint32_t kPrep = 96;
+    static constexpr uint32_t kOutput = 184;
+    static constexpr uint32_t kOther = 56;
+};
+template <int D>
+constexpr bool split_fits() {
+    return 128 * (2 * RegSplit<D>::kExp + RegSplit<D>::kPrep + RegSplit<D>::kOutput + RegSplit<D>::kOther) <=
+           kThreads * kLaunchRegs;
+}
+static_assert(split_fits<128>() && split_fits<64>(), "register split exceeds the launch allocation");
 // Warp roles inside the fifth warpgroup (warps 16-19).
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
@@ -144,21 +161,22 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 
 template <int D>
 struct alignas(1024) AttnSmem {
-    uint8_t q[BM * D];          // Q_hat tile, K-major, TMA-swizzled
+    uint8_t q[2][BM * D];       // Q_hat tiles (two query tiles in flight), K-major, TMA-swizzled
     uint8_t k[NS][BN * D];      // K_hat tiles
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
     float2 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha) per row and S buffer
     float alpha_o[AB][BM];      // prep -> output: alpha of block j (slot j mod AB)
-    float lsum[2][BM];          // exp -> output: final row sums of each column half
-    uint64_t q_full;
+    float lsum[2][2][BM];       // exp -> output: row sums of each key half (slot = tile mod 2)
+    uint64_t q_full[2], q_empty[2];
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
     uint64_t s_full[SB], p_full[SB];
     uint64_t x_full[SB][4];     // prep warp k -> exp warp k (same TMEM lane quadrant)
     uint64_t a_full[AB][4];     // prep warp k -> output warp k
     uint64_t a_empty[AB][4];    // output warp k -> prep warp k
     uint64_t o_full[OB], o_empty[OB];
-    uint64_t l_full, mma_drain;
+    uint64_t l_full[2], l_empty[2];
+    uint64_t mma_drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -183,6 +201,48 @@ __device__ __forceinline__ uint8_t *smem_aligned_1024() {
 template <int D>
 __device__ __forceinline__ AttnSmem<D> &get_smem() {
     return *reinterpret_cast<AttnSmem<D> *>(smem_aligned_1024());
+}
+
+// ----------------------------------------------------------- tiles ---
+
+// Query tiles in head-major order (a head's K_hat / V_hat then stay in L2
+// while the CTAs working on it are resident), the heaviest causal tile of
+// each head first.  CTA c processes tiles c, c + G, c + 2G, ... (G = grid).
+struct Tile {
+    int bh, q0, nb;   // head, first query row, key blocks
+};
+
+__device__ __forceinline__ Tile tile_at(int t, int ntiles, int L, int causal) {
+    Tile r;
+    r.bh = t / ntiles;
+    const int tt = t - r.bh * ntiles;
+    const int qt = causal ? (ntiles - 1 - tt) : tt;
+    r.q0 = qt * BM;
+    r.nb = causal ? (qt + 1) : (L + BN - 1) / BN;
+    return r;
+}
+
+// Position in this CTA's stream of (tile, key block) pairs.
+struct Cursor {
+    int t, i, j;   // tile id (>= total when done), tile count so far, key block
+    Tile T;
+};
+
+__device__ __forceinline__ Cursor cursor_begin(int ntiles, int total, int L, int causal) {
+    Cursor c;
+    c.t = blockIdx.x;
+    c.i = 0;
+    c.j = 0;
+    c.T = c.t < total ? tile_at(c.t, ntiles, L, causal) : Tile{0, 0, 0};
+    return c;
+}
+
+__device__ __forceinline__ void cursor_next(Cursor &c, int ntiles, int total, int L, int causal) {
+    if (++c.j < c.T.nb) return;
+    c.j = 0;
+    ++c.i;
+    c.t += gridDim.x;
+    if (c.t < total) c.T = tile_at(c.t, ntiles, L, causal);
 }
 
 // ------------------------------------------------------- prep pieces ---
@@ -244,18 +304,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rtid = 32 * warp + lane;
 
     const int ntiles = (L + BM - 1) / BM;
-    // Head-major order: the CTAs resident together mostly share one head's
-    // K_hat / V_hat, which then stay in L2; within a head the heaviest causal
-    // tiles go first.
-    const int bh = blockIdx.x / ntiles;
-    const int t = blockIdx.x - bh * ntiles;
-    const int qt = causal ? (ntiles - 1 - t) : t;
-    const int q0 = qt * BM;
-    const int nb = causal ? (qt + 1) : (L + BN - 1) / BN;
+    const int total = BH * ntiles;
     volatile int *abort_flag = &sm.abort_flag;
 
     if (tid == 0) {
-        mbar_init(&sm.q_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.q_full[b], 1);
+            mbar_init(&sm.q_empty[b], 1);
+            mbar_init(&sm.l_full[b], 2 * BM);
+            mbar_init(&sm.l_empty[b], BM);
+        }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sm.k_full[s], 32);
             mbar_init(&sm.v_full[s], 1);
@@ -275,7 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.o_full[b], 1);
             mbar_init(&sm.o_empty[b], BM);
         }
-        mbar_init(&sm.l_full, 2 * BM);
         mbar_init(&sm.mma_drain, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -292,43 +349,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tbase + 128 * SB;   // int32 P V block o at column tO + 128 o
 
     if (warp >= 16) {
-      regs_to<kRegsOther>();
+      regs_to<RegSplit<D>::kOther>();
       if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ---
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(&sm.q_full, BM * D);
-            tma_load_3d(&tmQ, &sm.q_full, sm.q, 0, q0, bh);
         }
-        int issued = 0;
-        for (int j = 0; j < nb; ++j) {
-            const int st = j % NS;
-            if (j >= NS && !warp_wait(&sm.kv_empty[st], ((j / NS) - 1) & 1, abort_flag, 1)) break;
-            const int key = j * BN + 4 * lane;
-            const float *src = sK + static_cast<int64_t>(bh) * L;
+        // s_K of a key block as four floats per lane (zero past the end);
+        // the loads for the next block are issued one block ahead so that
+        // their latency overlaps the wait for a free stage.
+        auto load_sk = [&](const Cursor &c) {
+            const float *src = sK + static_cast<int64_t>(c.T.bh) * L;
+            const int key = c.j * BN + 4 * lane;
             float4 v4;
             v4.x = key + 0 < L ? __ldg(src + key + 0) : 0.0f;
             v4.y = key + 1 < L ? __ldg(src + key + 1) : 0.0f;
             v4.z = key + 2 < L ? __ldg(src + key + 2) : 0.0f;
             v4.w = key + 3 < L ? __ldg(src + key + 3) : 0.0f;
-            *reinterpret_cast<float4 *>(&sm.sk[st][4 * lane]) = v4;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.k_full[st], BN * D);
-                tma_load_3d(&tmK, &sm.k_full[st], sm.k[st], 0, j * BN, bh);
-                mbar_arrive_expect_tx(&sm.v_full[st], D * BN);
-                tma_load_3d(&tmV, &sm.v_full[st], sm.v[st], j * BN, 0, bh);
-            } else {
-                mbar_arrive(&sm.k_full[st]);
+            return v4;
+        };
+        Cursor c = cursor_begin(ntiles, total, L, causal);
+        float4 sk_next = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (c.t < total) sk_next = load_sk(c);
+        int g = 0, q_issued = 0;
+        while (c.t < total) {
+            if (c.j == 0) {   // a new tile: its Q_hat into buffer i mod 2
+                const int qb = c.i & 1;
+                if (c.i >= 2 && !warp_wait(&sm.q_empty[qb], ((c.i >> 1) - 1) & 1, abort_flag, 8)) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.q_full[qb], BM * D);
+                    tma_load_3d(&tmQ, &sm.q_full[qb], sm.q[qb], 0, c.T.q0, c.T.bh);
+                }
+                q_issued = c.i + 1;
             }
+            const int st = g % NS;
+            if (g >= NS && !warp_wait(&sm.kv_empty[st], ((g / NS) - 1) & 1, abort_flag, 1)) break;
+            if (lane == 0) {
+                mbar_expect_tx(&sm.k_full[st], BN * D);
+                tma_load_3d(&tmK, &sm.k_full[st], sm.k[st], 0, c.j * BN, c.T.bh);
+                mbar_arrive_expect_tx(&sm.v_full[st], D * BN);
+                tma_load_3d(&tmV, &sm.v_full[st], sm.v[st], c.j * BN, 0, c.T.bh);
+            }
+            *reinterpret_cast<float4 *>(&sm.sk[st][4 * lane]) = sk_next;
+            mbar_arrive(&sm.k_full[st]);   // 32 arrivals + the K tile's bytes
+            cursor_next(c, ntiles, total, L, causal);
+            if (c.t < total) sk_next = load_sk(c);
             __syncwarp();
-            issued = j + 1;
+            ++g;
         }
-        // Drain: the last load issued into each stage (and Q) has landed.
-        drain_wait(&sm.q_full, 0);
-        for (int s = 0; s < NS && s < issued; ++s) {
-            const int last = s + ((issued - 1 - s) / NS) * NS;  // last block using stage s
+        // Drain: the last load issued into each stage and Q buffer has landed.
+        for (int b = 0; b < 2 && b < q_issued; ++b) {
+            const int last = b + ((q_issued - 1 - b) / 2) * 2;
+            drain_wait(&sm.q_full[b], (last >> 1) & 1);
+        }
+        for (int s = 0; s < NS && s < g; ++s) {
+            const int last = s + ((g - 1 - s) / NS) * NS;   // last block using stage s
             drain_wait(&sm.k_full[s], (last / NS) & 1);
             drain_wait(&sm.v_full[s], (last / NS) & 1);
         }
@@ -339,54 +416,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kSboQK = 8 * D;      // 8 rows of D bytes
         const uint32_t idesc_qk = make_idesc_i8(BM, BN);
         const uint32_t idesc_pv = make_idesc_i8(BM, D);
-        const uint64_t qdesc = make_sdesc(smem_u32(sm.q), kSboQK, kSwQK);
-        bool ok = warp_wait(&sm.q_full, 0, abort_flag, 2);
-        tc_fence_after();
-
-        auto mma_qk = [&](int j) {   // lane 0 only; K tile of block j has landed
-            const int st = j % NS, sb = j % SB;
-            const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
-#pragma unroll
-            for (int k = 0; k < D / 32; ++k)
-                mma_i8_ss(tS + sb * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
-            mma_commit(&sm.s_full[sb]);
-        };
-        auto mma_pv = [&](int j) {   // lane 0 only; P codes and V tile of block j ready
-            const int sb = j % SB, st = j % NS;
-            const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
-#pragma unroll
-            for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k..: see the exp warps
-                mma_i8_ts(tO + 128 * (j % OB), tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k,
-                          idesc_pv, k > 0);
-            mma_commit(&sm.o_full[j % OB]);
-            mma_commit(&sm.kv_empty[st]);
-        };
-
-        // Q K^T runs SB blocks ahead of P V: Q K^T of block j + SB reuses the
-        // S buffer of block j and is issued right after P V of block j, which
-        // the tensor pipe executes first.  P V alternates between OB blocks, so
-        // the output fold of block j overlaps P V of block j + 1.  Waits that
-        // are normally already satisfied come before the one that gates P V
-        // (the P codes), so that only the MMA issue follows it.
-        for (int j = 0; ok && j < SB && j < nb; ++j) {
-            if (!warp_wait(&sm.k_full[j % NS], (j / NS) & 1, abort_flag, 6)) { ok = false; break; }
-            tc_fence_after();
-            if (lane == 0) mma_qk(j);
-            __syncwarp();
-        }
-        for (int j = 0; ok && j < nb; ++j) {
-            const int jq = j + SB;
-            if (!warp_wait(&sm.v_full[j % NS], (j / NS) & 1, abort_flag, 4)) { ok = false; break; }
-            // P V block j % OB held block j - OB: its output fold is done
-            if (j >= OB && !warp_wait(&sm.o_empty[j % OB], ((j / OB) - 1) & 1, abort_flag, 5)) { ok = false; break; }
-            if (jq < nb && !warp_wait(&sm.k_full[jq % NS], (jq / NS) & 1, abort_flag, 6)) { ok = false; break; }
-            if (!warp_wait(&sm.p_full[j % SB], (j / SB) & 1, abort_flag, 3)) { ok = false; break; }
+        bool ok = true;
+        // qc walks the blocks whose Q K^T is issued, SB blocks ahead of pc,
+        // which walks the blocks whose P V is issued.
+        Cursor qc = cursor_begin(ntiles, total, L, causal);
+        Cursor pc = qc;
+        int gq = 0, gp = 0;
+        auto issue_qk = [&]() -> bool {   // Q K^T of block gq (cursor qc) into S buffer gq mod SB
+            const int qb = qc.i & 1, st = gq % NS, sb = gq % SB;
+            if (qc.j == 0 && !warp_wait(&sm.q_full[qb], (qc.i >> 1) & 1, abort_flag, 2)) return false;
+            if (!warp_wait(&sm.k_full[st], (gq / NS) & 1, abort_flag, 6)) return false;
             tc_fence_after();
             if (lane == 0) {
-                mma_pv(j);
-                if (jq < nb) mma_qk(jq);
+                const uint64_t qdesc = make_sdesc(smem_u32(sm.q[qb]), kSboQK, kSwQK);
+                const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
+#pragma unroll
+                for (int k = 0; k < D / 32; ++k)
+                    mma_i8_ss(tS + sb * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
+                mma_commit(&sm.s_full[sb]);
+                if (qc.j == qc.T.nb - 1) mma_commit(&sm.q_empty[qb]);   // last use of this Q tile
             }
             __syncwarp();
+            cursor_next(qc, ntiles, total, L, causal);
+            ++gq;
+            return true;
+        };
+        // Q K^T runs SB blocks ahead of P V: Q K^T of block g + SB reuses the
+        // S buffer of block g and is issued right after P V of block g, which
+        // the tensor pipe executes first.  Across a tile boundary this issues
+        // the next tile's first Q K^T while the current tile finishes.
+        while (ok && qc.t < total && gq < SB) ok = issue_qk();
+        while (ok && pc.t < total) {
+            const int st = gp % NS, sb = gp % SB;
+            if (!warp_wait(&sm.v_full[st], (gp / NS) & 1, abort_flag, 4)) break;
+            // the P V block held block g - OB: its output fold has read it
+            if (gp >= OB && !warp_wait(&sm.o_empty[gp % OB], ((gp / OB) - 1) & 1, abort_flag, 5)) break;
+            if (!warp_wait(&sm.p_full[sb], (gp / SB) & 1, abort_flag, 3)) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
+#pragma unroll
+                for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k ..: see the exp warps
+                    mma_i8_ts(tO + 128 * (gp % OB), tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1),
+                              vdesc + 2 * k, idesc_pv, k > 0);
+                mma_commit(&sm.o_full[gp % OB]);
+                mma_commit(&sm.kv_empty[st]);
+            }
+            __syncwarp();
+            cursor_next(pc, ntiles, total, L, causal);
+            ++gp;
+            if (qc.t < total) ok = issue_qk();
         }
         // Drain: every MMA this warp issued has completed before TMEM is freed.
         if (lane == 0) mma_commit(&sm.mma_drain);
@@ -396,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the other two warps of this warpgroup have no role
     } else if (warp < 8) {
-        regs_to<kRegsExp>();
+        regs_to<RegSplit<D>::kExp>();
         // ------------------------------------------------------- exp ---
         // Two warps per TMEM lane quadrant: half hf takes keys 64 hf .. 64 hf
         // + 63 of each block (chunks 2 hf, 2 hf + 1) and writes their 16 code
@@ -404,183 +483,210 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hf = warp >> 2, quad = warp & 3;
         const int row = 32 * quad + lane;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        const int qi = q0 + row;
-        // c = s_Q[i] log2(e) / sqrt(d) (see the prep warps for the clamp)
-        const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
-                                  (kLog2e / sqrtf(static_cast<float>(D))),
-                              1e-30f);
-        float l = 0.0f;
-        bool pre_x = false;   // probe of this block's x_full, taken one block early
-        for (int j = 0; j < nb; ++j) {
-            const int b = j % SB;
-            if (!settle(pre_x, &sm.x_full[b][quad], (j / SB) & 1, abort_flag, 7)) break;
-            tc_fence_after();
-            pre_x = j + 1 < nb && mbar_test_wait(&sm.x_full[(j + 1) % SB][quad], ((j + 1) / SB) & 1);
-            const float2 ca = sm.cm_alpha[b][row];
-            const float ncm = -ca.x;
-            const uint32_t tv = tS + lane_off + b * BN + 64 * hf;
-            const uint64_t c2 = f2_pack(c, c), ncm2 = f2_pack(ncm, ncm);
-            const uint64_t k127 = f2_pack(127.0f, 127.0f), magic = f2_pack(kMagic, kMagic);
-            uint64_t ps01 = 0ull, ps23 = 0ull;
-            uint32_t pk[16];
+        const uint64_t k127 = f2_pack(127.0f, 127.0f), magic = f2_pack(kMagic, kMagic);
+        bool pre_x = false;   // probe of the next block's x_full, taken one block early
+        bool ok = true;
+        int g = 0;
+        for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
+            const Tile T = tile_at(t, ntiles, L, causal);
+            const int qi = T.q0 + row;
+            // c = s_Q[i] log2(e) / sqrt(d) (see the prep warps for the clamp)
+            const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(T.bh) * L + qi) : 0.0f) *
+                                      (kLog2e / sqrtf(static_cast<float>(D))),
+                                  1e-30f);
+            const uint64_t c2 = f2_pack(c, c);
+            float l = 0.0f;
+            for (int j = 0; j < T.nb; ++j, ++g) {
+                const int b = g % SB;
+                if (!settle(pre_x, &sm.x_full[b][quad], (g / SB) & 1, abort_flag, 7)) { ok = false; break; }
+                tc_fence_after();
+                pre_x = mbar_test_wait(&sm.x_full[(g + 1) % SB][quad], ((g + 1) / SB) & 1);
+                const float2 ca = sm.cm_alpha[b][row];
+                const uint64_t ncm2 = f2_pack(-ca.x, -ca.x);
+                const uint32_t tv = tS + lane_off + b * BN + 64 * hf;
+                uint64_t ps01 = 0ull, ps23 = 0ull;
+                uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                uint32_t w[32];
-                tmem_ld32(tv + 32 * e, w);
-                tmem_wait_ld();
+                for (int e = 0; e < 2; ++e) {
+                    uint32_t w[32];
+                    tmem_ld32(tv + 32 * e, w);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
-                    float x0, x1, x2, x3;
-                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), c2, ncm2), x0, x1);
-                    f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2, ncm2), x2, x3);
-                    const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
-                    const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
-                    ps01 = fadd2(ps01, p01);
-                    ps23 = fadd2(ps23, p23);
-                    // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
-                    float t0, t1, t2, t3;
-                    f2_unpack(ffma2(p01, k127, magic), t0, t1);
-                    f2_unpack(ffma2(p23, k127, magic), t2, t3);
-                    pk[8 * e + q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
-                                         prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
+                    for (int q = 0; q < 8; ++q) {
+                        // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
+                        float x0, x1, x2, x3;
+                        f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), c2, ncm2),
+                                  x0, x1);
+                        f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2,
+                                        ncm2),
+                                  x2, x3);
+                        const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
+                        const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
+                        ps01 = fadd2(ps01, p01);
+                        ps23 = fadd2(ps23, p23);
+                        // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
+                        float t0, t1, t2, t3;
+                        f2_unpack(ffma2(p01, k127, magic), t0, t1);
+                        f2_unpack(ffma2(p23, k127, magic), t2, t3);
+                        pk[8 * e + q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
+                                             prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
+                    }
                 }
+                // both chunks are in registers: their columns now take the codes
+                tmem_st8(tv, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
+                tmem_st8(tv + 8, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
+                float ps0, ps1, ps2, ps3;
+                f2_unpack(ps01, ps0, ps1);
+                f2_unpack(ps23, ps2, ps3);
+                l = l * ca.y + ((ps0 + ps1) + (ps2 + ps3));
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.p_full[b]);
             }
-            float ps0, ps1, ps2, ps3;
-            f2_unpack(ps01, ps0, ps1);
-            f2_unpack(ps23, ps2, ps3);
-            // both chunks are in registers: their columns now take the codes
-            tmem_st8(tv, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
-            tmem_st8(tv + 8, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
-            const float ps = (ps0 + ps1) + (ps2 + ps3);
-            l = l * ca.y + ps;
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.p_full[b]);
+            if (!ok) break;
+            // this tile's half-row sum -> the output side (slot = tile mod 2)
+            const int ls = i & 1;
+            if (i >= 2 && !warp_wait(&sm.l_empty[ls], ((i >> 1) - 1) & 1, abort_flag, 17)) break;
+            sm.lsum[ls][hf][row] = l;
+            mbar_arrive(&sm.l_full[ls]);
         }
-        sm.lsum[hf][row] = l;
-        mbar_arrive(&sm.l_full);
     } else if (warp < 12) {
-        regs_to<kRegsPrep>();
+        regs_to<RegSplit<D>::kPrep>();
         // ------------------------------------------------------ prep ---
         const int row = rtid - 256;
-        const int qi = q0 + row;
         const int quad = warp - 8;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c (S_ij s_K[j]).
-        // Clamped to a tiny positive value: a zero Q row then still maps masked
-        // keys (v = -inf) to p = 0 and visible keys to p = 1.
-        const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(bh) * L + qi) : 0.0f) *
-                                  (kLog2e / sqrtf(static_cast<float>(D))),
-                              1e-30f);
-        float m_old = -INFINITY;
-        // probes of this block's s_full / k_full, taken one block early
+        // probes of the next block's s_full / k_full, taken one block early
         bool pre_s = false, pre_k = false;
-        for (int j = 0; j < nb; ++j) {
-            // -- block j: v = fl(S s_K) (int32 -> fp32 exact, |S| <= 127^2 d
-            // < 2^24), mask, row max.
-            const int b = j % SB, ab = j % AB, st = j % NS;
-            if (!settle(pre_s, &sm.s_full[b], (j / SB) & 1, abort_flag, 12)) break;
-            // s_K of this block: published by the producer's release-arrive
-            if (!settle(pre_k, &sm.k_full[st], (j / NS) & 1, abort_flag, 13)) break;
-            tc_fence_after();
-            const bool pre_a = j < AB || mbar_test_wait(&sm.a_empty[ab][quad], ((j / AB) - 1) & 1);
-            const int jn = j + 1;
-            pre_s = jn < nb && mbar_test_wait(&sm.s_full[jn % SB], (jn / SB) & 1);
-            pre_k = jn < nb && mbar_test_wait(&sm.k_full[jn % NS], (jn / NS) & 1);
-            const uint32_t ts = tS + lane_off + b * BN;
-            const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
-            const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
+        bool ok = true;
+        int g = 0;
+        for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+            const Tile T = tile_at(t, ntiles, L, causal);
+            const int qi = T.q0 + row;
+            // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c (S_ij s_K[j]).
+            // Clamped to a tiny positive value: a zero Q row then still maps masked
+            // keys (v = -inf) to p = 0 and visible keys to p = 1.
+            const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(T.bh) * L + qi) : 0.0f) *
+                                      (kLog2e / sqrtf(static_cast<float>(D))),
+                                  1e-30f);
             const int lim = causal ? min(L, qi + 1) : L;
-            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            float m_old = -INFINITY;
+            for (int j = 0; j < T.nb; ++j, ++g) {
+                // -- block j: v = fl(S s_K) (int32 -> fp32 exact, |S| <= 127^2 d
+                // < 2^24), mask, row max.
+                const int b = g % SB, ab = g % AB, st = g % NS;
+                if (!settle(pre_s, &sm.s_full[b], (g / SB) & 1, abort_flag, 12)) { ok = false; break; }
+                // s_K of this block: published by the producer's release-arrive
+                if (!settle(pre_k, &sm.k_full[st], (g / NS) & 1, abort_flag, 13)) { ok = false; break; }
+                tc_fence_after();
+                const bool pre_a = g < AB || mbar_test_wait(&sm.a_empty[ab][quad], ((g / AB) - 1) & 1);
+                pre_s = mbar_test_wait(&sm.s_full[(g + 1) % SB], ((g + 1) / SB) & 1);
+                pre_k = mbar_test_wait(&sm.k_full[(g + 1) % NS], ((g + 1) / NS) & 1);
+                const uint32_t ts = tS + lane_off + b * BN;
+                const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
+                const bool need_mask = (causal && j == T.nb - 1) || ((j + 1) * BN > L);
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                uint32_t w[32];
-                tmem_ld32(ts + 32 * ch, w);
-                tmem_wait_ld();
-                scores_to_v(w, sk4 + 8 * ch);
-                // keys past the end of the sequence, or after the query
-                // (causal), get v = -inf (p = 0)
-                if (need_mask) mask_v(w, j * BN + 32 * ch, lim);
-                max_v(w, mx);
-                tmem_st32(ts + 32 * ch, w);
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    uint32_t w[32];
+                    tmem_ld32(ts + 32 * ch, w);
+                    tmem_wait_ld();
+                    scores_to_v(w, sk4 + 8 * ch);
+                    // keys past the end of the sequence, or after the query
+                    // (causal), get v = -inf (p = 0)
+                    if (need_mask) mask_v(w, j * BN + 32 * ch, lim);
+                    max_v(w, mx);
+                    tmem_st32(ts + 32 * ch, w);
+                }
+                mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
+                const float m_new = fmaxf(m_old, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
+                const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
+                m_old = m_new;
+                sm.cm_alpha[b][row] = make_float2(c * m_new, alpha);
+                // alpha of block j -> the output warp of this quadrant
+                if (!settle(pre_a, &sm.a_empty[ab][quad], ((g / AB) - 1) & 1, abort_flag, 14)) {
+                    ok = false;
+                    break;
+                }
+                sm.alpha_o[ab][row] = alpha;
+                mbar_arrive(&sm.a_full[ab][quad]);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&sm.x_full[b][quad]);
             }
-            mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
-            const float m_new = fmaxf(m_old, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
-            const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
-            m_old = m_new;
-            sm.cm_alpha[b][row] = make_float2(c * m_new, alpha);
-            // alpha of block j -> the output warp of this quadrant
-            if (!settle(pre_a, &sm.a_empty[ab][quad], ((j / AB) - 1) & 1, abort_flag, 14)) break;
-            sm.alpha_o[ab][row] = alpha;
-            mbar_arrive(&sm.a_full[ab][quad]);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.x_full[b][quad]);
         }
     } else {
-        regs_to<kRegsOutput>();
+        regs_to<RegSplit<D>::kOutput>();
         // ------------------------------------------------ output side ---
         const int row = rtid - 384;
-        const int qi = q0 + row;
         const int quad = warp - 12;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        uint64_t o2[D / 2];   // the output row as fp32 pairs
-#pragma unroll
-        for (int i = 0; i < D / 2; ++i) o2[i] = 0ull;
         bool ok = true;
-        for (int j = 0; j < nb; ++j) {
-            const int ab = j % AB;
-            // o = alpha o + (P V block), the int32 block turned into fp32
-            // exactly (|x| <= 127^2 128 < 2^24)
-            const uint32_t to = tO + 128 * (j % OB);
-            if (!warp_wait(&sm.o_full[j % OB], (j / OB) & 1, abort_flag, 9)) { ok = false; break; }
-            if (!warp_wait(&sm.a_full[ab][quad], (j / AB) & 1, abort_flag, 10)) { ok = false; break; }
-            tc_fence_after();
-            const float alpha = sm.alpha_o[ab][row];
-            mbar_arrive(&sm.a_empty[ab][quad]);
-            const uint64_t a2 = f2_pack(alpha, alpha);
-            // the block in pairs of 32-column chunks; once the last pair is
-            // in registers the P V block is released for the next block
+        int g = 0;
+        for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
+            const Tile T = tile_at(t, ntiles, L, causal);
+            const int qi = T.q0 + row;
+            uint64_t o2[D / 2];   // the output row as fp32 pairs
 #pragma unroll
-            for (int pr = 0; pr < D / 64; ++pr) {
-                uint32_t w0[32], w1[32];
-                tmem_ld32(to + lane_off + 64 * pr, w0);
-                tmem_ld32(to + lane_off + 64 * pr + 32, w1);
-                tmem_wait_ld();
-                if (pr == D / 64 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(&sm.o_empty[j % OB]);
-                }
+            for (int e = 0; e < D / 2; ++e) o2[e] = 0ull;
+            for (int j = 0; j < T.nb; ++j, ++g) {
+                const int ab = g % AB;
+                // o = alpha o + (P V block), the int32 block turned into fp32
+                // exactly (|x| <= 127^2 128 < 2^24)
+                const uint32_t to = tO + 128 * (g % OB);
+                if (!warp_wait(&sm.o_full[g % OB], (g / OB) & 1, abort_flag, 9)) { ok = false; break; }
+                if (!warp_wait(&sm.a_full[ab][quad], (g / AB) & 1, abort_flag, 10)) { ok = false; break; }
+                tc_fence_after();
+                const float alpha = sm.alpha_o[ab][row];
+                mbar_arrive(&sm.a_empty[ab][quad]);
+                const uint64_t a2 = f2_pack(alpha, alpha);
+                // the block in pairs of 32-column chunks; once the last pair is
+                // in registers the P V block is released for the next block
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w0[2 * i])),
-                                               __int2float_rn(static_cast<int32_t>(w0[2 * i + 1])));
-                    o2[32 * pr + i] = ffma2(o2[32 * pr + i], a2, x);
-                }
+                for (int pr = 0; pr < D / 64; ++pr) {
+                    uint32_t w0[32], w1[32];
+                    tmem_ld32(to + lane_off + 64 * pr, w0);
+                    tmem_ld32(to + lane_off + 64 * pr + 32, w1);
+                    tmem_wait_ld();
+                    if (pr == D / 64 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(&sm.o_empty[g % OB]);
+                    }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w1[2 * i])),
-                                               __int2float_rn(static_cast<int32_t>(w1[2 * i + 1])));
-                    o2[32 * pr + 16 + i] = ffma2(o2[32 * pr + 16 + i], a2, x);
+                    for (int e = 0; e < 16; ++e) {
+                        const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w0[2 * e])),
+                                                   __int2float_rn(static_cast<int32_t>(w0[2 * e + 1])));
+                        o2[32 * pr + e] = ffma2(o2[32 * pr + e], a2, x);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w1[2 * e])),
+                                                   __int2float_rn(static_cast<int32_t>(w1[2 * e + 1])));
+                        o2[32 * pr + 16 + e] = ffma2(o2[32 * pr + 16 + e], a2, x);
+                    }
                 }
             }
-        }
-        if (ok && warp_wait(&sm.l_full, 0, abort_flag, 11) && qi < L) {
-            const float l = sm.lsum[0][row] + sm.lsum[1][row];
-            const float f = __ldg(sV + bh) / (127.0f * l);
-            uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(bh) * L + qi) * D);
+            if (!ok) break;
+            // the tile's row sums (both key halves) -> normalised fp16 row
+            const int ls = i & 1;
+            if (!warp_wait(&sm.l_full[ls], (i >> 1) & 1, abort_flag, 11)) break;
+            const float l = sm.lsum[ls][0][row] + sm.lsum[ls][1][row];
+            mbar_arrive(&sm.l_empty[ls]);
+            if (qi < L) {
+                const float f = __ldg(sV + T.bh) / (127.0f * l);
+                uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(T.bh) * L + qi) * D);
 #pragma unroll
-            for (int c8 = 0; c8 < D / 8; ++c8) {
-                uint4 wv;
-                __half2 *h = reinterpret_cast<__half2 *>(&wv);
+                for (int c8 = 0; c8 < D / 8; ++c8) {
+                    uint4 wv;
+                    __half2 *h = reinterpret_cast<__half2 *>(&wv);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float lo, hi;
-                    f2_unpack(o2[4 * c8 + e], lo, hi);
-                    h[e] = __floats2half2_rn(lo * f, hi * f);
+                    for (int e = 0; e < 4; ++e) {
+                        float lo, hi;
+                        f2_unpack(o2[4 * c8 + e], lo, hi);
+                        h[e] = __floats2half2_rn(lo * f, hi * f);
+                    }
+                    dst[c8] = wv;
                 }
-                dst[c8] = wv;
             }
         }
     }
@@ -711,6 +817,24 @@ int make_map(CUtensorMap *map, const void *base, uint64_t x, uint64_t y, uint64_
     return r == CUDA_SUCCESS ? INTFA_OK : INTFA_ERR_CUDA;
 }
 
+// Grid of the persistent attention kernel: one CTA per SM.  CTA c takes tiles
+// c, c + G, ...; with causal masking the per-tile work cycles with period
+// ntiles inside each head, so G is chosen coprime to ntiles, which makes every
+// CTA's tiles cover the heavy and light positions alike (one SM may idle).
+unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
+    if (nsm < 1) nsm = 1;
+    if (total <= nsm) return static_cast<unsigned>(total);
+    int g = nsm;
+    if (causal) {
+        for (int cand = nsm; cand > nsm / 2; --cand) {
+            int a = cand, b = ntiles;
+            while (b) { const int r = a % b; a = b; b = r; }
+            if (a == 1) { g = cand; break; }
+        }
+    }
+    return static_cast<unsigned>(g);
+}
+
 template <int D>
 int launch_attn(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                 const float *sK, const float *sV, int B, int H, int L, int causal, void *O,
@@ -735,7 +859,11 @@ int launch_attn(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const floa
     if (rc) return rc;
     if (fa.numRegs != kLaunchRegs) return INTFA_ERR_UNSUPPORTED;
     const int ntiles = (L + BM - 1) / BM;
-    const unsigned grid = static_cast<unsigned>(ntiles) * static_cast<unsigned>(BH);
+    int dev = 0, nsm = 0;
+    rc = cuda_status(cudaGetDevice(&dev));
+    if (!rc) rc = cuda_status(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    if (rc) return rc;
+    const unsigned grid = persistent_grid(static_cast<int64_t>(BH) * ntiles, ntiles, causal, nsm);
     attn_fwd_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, sQ, sK, sV,
                                                           static_cast<__half *>(O), BH, L, causal);
     return cuda_status(cudaGetLastError());
