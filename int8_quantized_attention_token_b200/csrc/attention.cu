@@ -165,7 +165,7 @@ struct alignas(1024) AttnSmem {
     uint8_t k[NS][BN * D];      // K_hat tiles
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
-    float2 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha) per row and S buffer
+    float4 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha, c, -) per row and S buffer
     float alpha_o[AB][BM];      // prep -> output: alpha of block j (slot j mod AB)
     float lsum[2][2][BM];       // exp -> output: row sums of each key half (slot = tile mod 2)
     uint64_t q_full[2], q_empty[2];
@@ -489,20 +489,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         int g = 0;
         for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
             const Tile T = tile_at(t, ntiles, L, causal);
-            const int qi = T.q0 + row;
-            // c = s_Q[i] log2(e) / sqrt(d) (see the prep warps for the clamp)
-            const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(T.bh) * L + qi) : 0.0f) *
-                                      (kLog2e / sqrtf(static_cast<float>(D))),
-                                  1e-30f);
-            const uint64_t c2 = f2_pack(c, c);
             float l = 0.0f;
             for (int j = 0; j < T.nb; ++j, ++g) {
                 const int b = g % SB;
                 if (!settle(pre_x, &sm.x_full[b][quad], (g / SB) & 1, abort_flag, 7)) { ok = false; break; }
                 tc_fence_after();
                 pre_x = mbar_test_wait(&sm.x_full[(g + 1) % SB][quad], ((g + 1) / SB) & 1);
-                const float2 ca = sm.cm_alpha[b][row];
-                const uint64_t ncm2 = f2_pack(-ca.x, -ca.x);
+                // (c m, alpha, c) from the prep warp: c = s_Q[i] log2(e) / sqrt(d)
+                const float4 ca = sm.cm_alpha[b][row];
+                const uint64_t ncm2 = f2_pack(-ca.x, -ca.x), c2 = f2_pack(ca.z, ca.z);
                 const uint32_t tv = tS + lane_off + b * BN + 64 * hf;
                 uint64_t ps01 = 0ull, ps23 = 0ull;
                 uint32_t pk[16];
@@ -602,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_new = fmaxf(m_old, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
                 const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
                 m_old = m_new;
-                sm.cm_alpha[b][row] = make_float2(c * m_new, alpha);
+                sm.cm_alpha[b][row] = make_float4(c * m_new, alpha, c, 0.0f);
                 // alpha of block j -> the output warp of this quadrant
                 if (!settle(pre_a, &sm.a_empty[ab][quad], ((g / AB) - 1) & 1, abort_flag, 14)) {
                     ok = false;
@@ -626,6 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
             const Tile T = tile_at(t, ntiles, L, causal);
             const int qi = T.q0 + row;
+            const float s_v = __ldg(sV + T.bh);   // needed at the tile's end; loaded early
             uint64_t o2[D / 2];   // the output row as fp32 pairs
 #pragma unroll
             for (int e = 0; e < D / 2; ++e) o2[e] = 0ull;
@@ -673,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float l = sm.lsum[ls][0][row] + sm.lsum[ls][1][row];
             mbar_arrive(&sm.l_empty[ls]);
             if (qi < L) {
-                const float f = __ldg(sV + T.bh) / (127.0f * l);
+                const float f = s_v / (127.0f * l);
                 uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(T.bh) * L + qi) * D);
 #pragma unroll
                 for (int c8 = 0; c8 < D / 8; ++c8) {
