@@ -75,8 +75,8 @@ constexpr int kLaunchRegs = 96;
 template <int D>
 struct RegSplit {   // d = 128: the output row alone is 128 registers
     static constexpr uint32_t kExp = 72;      // each of the two exp warpgroups
-    static constexpr uint32_t kPrep = 80;
-    static constexpr uint32_t kOutput = 208;
+    static constexpr uint32_t kPrep = 96;
+    static constexpr uint32_t kOutput = 192;
     static constexpr uint32_t kOther = 48;
 };
 template <>
@@ -245,6 +245,26 @@ __device__ __forceinline__ void cursor_next(Cursor &c, int ntiles, int total, in
     if (c.t < total) c.T = tile_at(c.t, ntiles, L, causal);
 }
 
+// Slot and phase parity of a ring of N mbarrier-guarded buffers, advanced one
+// block at a time (block g: idx = g mod N, ph = (g / N) mod 2) without
+// integer division.
+template <int N>
+struct Ring {
+    int idx = 0;
+    uint32_t ph = 0;
+    __device__ __forceinline__ void next() {
+        if (++idx == N) {
+            idx = 0;
+            ph ^= 1u;
+        }
+    }
+    __device__ __forceinline__ Ring after() const {
+        Ring r = *this;
+        r.next();
+        return r;
+    }
+};
+
 // ------------------------------------------------------- prep pieces ---
 
 // v = fl(S s_K) in place (int32 -> fp32 is exact: |S| <= 127^2 d < 2^24).
@@ -374,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float4 sk_next = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         if (c.t < total) sk_next = load_sk(c);
         int g = 0, q_issued = 0;
+        Ring<NS> kv;
         while (c.t < total) {
             if (c.j == 0) {   // a new tile: its Q_hat into buffer i mod 2
                 const int qb = c.i & 1;
@@ -384,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 q_issued = c.i + 1;
             }
-            const int st = g % NS;
-            if (g >= NS && !warp_wait(&sm.kv_empty[st], ((g / NS) - 1) & 1, abort_flag, 1)) break;
+            const int st = kv.idx;
+            if (g >= NS && !warp_wait(&sm.kv_empty[st], kv.ph ^ 1u, abort_flag, 1)) break;
             if (lane == 0) {
                 mbar_expect_tx(&sm.k_full[st], BN * D);
                 tma_load_3d(&tmK, &sm.k_full[st], sm.k[st], 0, c.j * BN, c.T.bh);
@@ -398,6 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c.t < total) sk_next = load_sk(c);
             __syncwarp();
             ++g;
+            kv.next();
         }
         // Drain: the last load issued into each stage and Q buffer has landed.
         for (int b = 0; b < 2 && b < q_issued; ++b) {
@@ -421,11 +443,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // which walks the blocks whose P V is issued.
         Cursor qc = cursor_begin(ntiles, total, L, causal);
         Cursor pc = qc;
-        int gq = 0, gp = 0;
+        int gq = 0;
+        Ring<NS> q_st, p_st;   // K/V stage of the Q K^T / P V block
+        Ring<SB> q_sb, p_sb;   // S buffer of the Q K^T / P V block
+        uint32_t p_oph = 0;    // o_full / o_empty parity of the P V block (one P V block)
         auto issue_qk = [&]() -> bool {   // Q K^T of block gq (cursor qc) into S buffer gq mod SB
-            const int qb = qc.i & 1, st = gq % NS, sb = gq % SB;
+            const int qb = qc.i & 1, st = q_st.idx, sb = q_sb.idx;
             if (qc.j == 0 && !warp_wait(&sm.q_full[qb], (qc.i >> 1) & 1, abort_flag, 2)) return false;
-            if (!warp_wait(&sm.k_full[st], (gq / NS) & 1, abort_flag, 6)) return false;
+            if (!warp_wait(&sm.k_full[st], q_st.ph, abort_flag, 6)) return false;
             tc_fence_after();
             if (lane == 0) {
                 const uint64_t qdesc = make_sdesc(smem_u32(sm.q[qb]), kSboQK, kSwQK);
@@ -439,6 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             cursor_next(qc, ntiles, total, L, causal);
             ++gq;
+            q_st.next();
+            q_sb.next();
             return true;
         };
         // Q K^T runs SB blocks ahead of P V: Q K^T of block g + SB reuses the
@@ -446,25 +473,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the tensor pipe executes first.  Across a tile boundary this issues
         // the next tile's first Q K^T while the current tile finishes.
         while (ok && qc.t < total && gq < SB) ok = issue_qk();
+        static_assert(OB == 1, "one P V block");
+        bool first_pv = true;
         while (ok && pc.t < total) {
-            const int st = gp % NS, sb = gp % SB;
-            if (!warp_wait(&sm.v_full[st], (gp / NS) & 1, abort_flag, 4)) break;
-            // the P V block held block g - OB: its output fold has read it
-            if (gp >= OB && !warp_wait(&sm.o_empty[gp % OB], ((gp / OB) - 1) & 1, abort_flag, 5)) break;
-            if (!warp_wait(&sm.p_full[sb], (gp / SB) & 1, abort_flag, 3)) break;
+            const int st = p_st.idx, sb = p_sb.idx;
+            if (!warp_wait(&sm.v_full[st], p_st.ph, abort_flag, 4)) break;
+            // the P V block held the previous block: its output fold has read it
+            if (!first_pv && !warp_wait(&sm.o_empty[0], p_oph ^ 1u, abort_flag, 5)) break;
+            if (!warp_wait(&sm.p_full[sb], p_sb.ph, abort_flag, 3)) break;
             tc_fence_after();
             if (lane == 0) {
                 const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
 #pragma unroll
                 for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k ..: see the exp warps
-                    mma_i8_ts(tO + 128 * (gp % OB), tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1),
-                              vdesc + 2 * k, idesc_pv, k > 0);
-                mma_commit(&sm.o_full[gp % OB]);
+                    mma_i8_ts(tO, tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k, idesc_pv,
+                              k > 0);
+                mma_commit(&sm.o_full[0]);
                 mma_commit(&sm.kv_empty[st]);
             }
             __syncwarp();
             cursor_next(pc, ntiles, total, L, causal);
-            ++gp;
+            first_pv = false;
+            p_st.next();
+            p_sb.next();
+            p_oph ^= 1u;
             if (qc.t < total) ok = issue_qk();
         }
         // Drain: every MMA this warp issued has completed before TMEM is freed.
@@ -486,15 +518,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t k127 = f2_pack(127.0f, 127.0f), magic = f2_pack(kMagic, kMagic);
         bool pre_x = false;   // probe of the next block's x_full, taken one block early
         bool ok = true;
-        int g = 0;
+        Ring<SB> sb;
         for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
             const Tile T = tile_at(t, ntiles, L, causal);
             float l = 0.0f;
-            for (int j = 0; j < T.nb; ++j, ++g) {
-                const int b = g % SB;
-                if (!settle(pre_x, &sm.x_full[b][quad], (g / SB) & 1, abort_flag, 7)) { ok = false; break; }
+            for (int j = 0; j < T.nb; ++j, sb.next()) {
+                const int b = sb.idx;
+                if (!settle(pre_x, &sm.x_full[b][quad], sb.ph, abort_flag, 7)) { ok = false; break; }
                 tc_fence_after();
-                pre_x = mbar_test_wait(&sm.x_full[(g + 1) % SB][quad], ((g + 1) / SB) & 1);
+                const Ring<SB> nx = sb.after();
+                pre_x = mbar_test_wait(&sm.x_full[nx.idx][quad], nx.ph);
                 // (c m, alpha, c) from the prep warp: c = s_Q[i] log2(e) / sqrt(d)
                 const float4 ca = sm.cm_alpha[b][row];
                 const uint64_t ncm2 = f2_pack(-ca.x, -ca.x), c2 = f2_pack(ca.z, ca.z);
@@ -555,6 +588,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool pre_s = false, pre_k = false;
         bool ok = true;
         int g = 0;
+        Ring<SB> sb;
+        Ring<NS> ks;
+        Ring<AB> as;
         for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
             const Tile T = tile_at(t, ntiles, L, causal);
             const int qi = T.q0 + row;
@@ -566,17 +602,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   1e-30f);
             const int lim = causal ? min(L, qi + 1) : L;
             float m_old = -INFINITY;
-            for (int j = 0; j < T.nb; ++j, ++g) {
+            for (int j = 0; j < T.nb; ++j, ++g, sb.next(), ks.next(), as.next()) {
                 // -- block j: v = fl(S s_K) (int32 -> fp32 exact, |S| <= 127^2 d
                 // < 2^24), mask, row max.
-                const int b = g % SB, ab = g % AB, st = g % NS;
-                if (!settle(pre_s, &sm.s_full[b], (g / SB) & 1, abort_flag, 12)) { ok = false; break; }
+                const int b = sb.idx, ab = as.idx, st = ks.idx;
+                if (!settle(pre_s, &sm.s_full[b], sb.ph, abort_flag, 12)) { ok = false; break; }
                 // s_K of this block: published by the producer's release-arrive
-                if (!settle(pre_k, &sm.k_full[st], (g / NS) & 1, abort_flag, 13)) { ok = false; break; }
+                if (!settle(pre_k, &sm.k_full[st], ks.ph, abort_flag, 13)) { ok = false; break; }
                 tc_fence_after();
-                const bool pre_a = g < AB || mbar_test_wait(&sm.a_empty[ab][quad], ((g / AB) - 1) & 1);
-                pre_s = mbar_test_wait(&sm.s_full[(g + 1) % SB], ((g + 1) / SB) & 1);
-                pre_k = mbar_test_wait(&sm.k_full[(g + 1) % NS], ((g + 1) / NS) & 1);
+                const bool pre_a = g < AB || mbar_test_wait(&sm.a_empty[ab][quad], as.ph ^ 1u);
+                const Ring<SB> nsb = sb.after();
+                const Ring<NS> nks = ks.after();
+                pre_s = mbar_test_wait(&sm.s_full[nsb.idx], nsb.ph);
+                pre_k = mbar_test_wait(&sm.k_full[nks.idx], nks.ph);
                 const uint32_t ts = tS + lane_off + b * BN;
                 const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
                 const bool need_mask = (causal && j == T.nb - 1) || ((j + 1) * BN > L);
@@ -599,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_old = m_new;
                 sm.cm_alpha[b][row] = make_float4(c * m_new, alpha, c, 0.0f);
                 // alpha of block j -> the output warp of this quadrant
-                if (!settle(pre_a, &sm.a_empty[ab][quad], ((g / AB) - 1) & 1, abort_flag, 14)) {
+                if (!settle(pre_a, &sm.a_empty[ab][quad], as.ph ^ 1u, abort_flag, 14)) {
                     ok = false;
                     break;
                 }
@@ -617,7 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp - 12;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         bool ok = true;
-        int g = 0;
+        Ring<AB> as;
+        uint32_t oph = 0;   // o_full parity (one P V block)
         for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
             const Tile T = tile_at(t, ntiles, L, causal);
             const int qi = T.q0 + row;
@@ -625,13 +664,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t o2[D / 2];   // the output row as fp32 pairs
 #pragma unroll
             for (int e = 0; e < D / 2; ++e) o2[e] = 0ull;
-            for (int j = 0; j < T.nb; ++j, ++g) {
-                const int ab = g % AB;
+            for (int j = 0; j < T.nb; ++j, as.next(), oph ^= 1u) {
+                const int ab = as.idx;
                 // o = alpha o + (P V block), the int32 block turned into fp32
                 // exactly (|x| <= 127^2 128 < 2^24)
-                const uint32_t to = tO + 128 * (g % OB);
-                if (!warp_wait(&sm.o_full[g % OB], (g / OB) & 1, abort_flag, 9)) { ok = false; break; }
-                if (!warp_wait(&sm.a_full[ab][quad], (g / AB) & 1, abort_flag, 10)) { ok = false; break; }
+                const uint32_t to = tO;
+                if (!warp_wait(&sm.o_full[0], oph, abort_flag, 9)) { ok = false; break; }
+                if (!warp_wait(&sm.a_full[ab][quad], as.ph, abort_flag, 10)) { ok = false; break; }
                 tc_fence_after();
                 const float alpha = sm.alpha_o[ab][row];
                 mbar_arrive(&sm.a_empty[ab][quad]);
@@ -646,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
                     if (pr == D / 64 - 1) {
                         tc_fence_before();
-                        mbar_arrive(&sm.o_empty[g % OB]);
+                        mbar_arrive(&sm.o_empty[0]);
                     }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
