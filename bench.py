@@ -176,18 +176,27 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
     V3 = V.reshape(BH, L, d)
 
+    fused_q = args.q_path == "fused"
+
     def step(ev=None):
-        intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
+        # a1 (K; and Q unless fused), a2 (V), then a3-a9 in the attention kernel
+        if not fused_q:
+            intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
         intfa.intfa_quantize_per_token(K, Kq, sK, stream=stream)
         intfa.intfa_quantize_per_tensor(V3, True, Vt, sV, ws, stream=stream)
         if ev is not None:
             ev[0].record(stream)
-        intfa.intfa_attention_fwd(Qq, Kq, Vt.reshape(B, H, d, ld), sQ, sK, sV.reshape(B, H), w.causal, O,
-                                  stream=stream)
+        if fused_q:   # Q quantised per token inside the attention kernel
+            intfa.intfa_attention_fwd_q16(Q, Kq, Vt.reshape(B, H, d, ld), sK, sV.reshape(B, H), w.causal, O,
+                                          s_Q=sQ, stream=stream)
+        else:
+            intfa.intfa_attention_fwd(Qq, Kq, Vt.reshape(B, H, d, ld), sQ, sK, sV.reshape(B, H), w.causal, O,
+                                      stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
-    kernels_per_step = 5  # quantise Q, quantise K, V abs-max, V convert, attention
+    # quantise K, V abs-max, V convert, attention (+ quantise Q when separate)
+    kernels_per_step = 4 if fused_q else 5
 
     for _ in range(args.warmup):
         step()
@@ -267,7 +276,9 @@ def run_gpu(args):
             "config": {**w.as_dict(), "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (fp16 Q/K/V 3x128 MiB read per step)"},
             "pct_of_int8_peak": round(100.0 * value / world / peak, 2),
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": round(achieved, 2),
+            "roofline": {"bound": "tensor",
+                         "kernel": "attn_fwd_kernel<128, Q quantised in-kernel>" if fused_q else "attn_fwd_kernel<128>",
+                         "achieved": round(achieved, 2),
                          "peak": round(peak, 1), "unit": UNIT, "frac": round(achieved / peak, 4),
                          "traffic": traffic_for(w.name),
                          "peak_note": f"{pk['source']} bf16 burst {pk['bf16_burst']} TFLOP/s x {I8_PER_BF16} "
@@ -275,7 +286,8 @@ def run_gpu(args):
                          "frac_of_sustained": round(achieved / (pk["bf16_sustained"] * I8_PER_BF16), 4),
                          "attn_ms": round(attn_mean, 5), "ops_per_launch": w.ops},
             "kernels_ms_per_step": {"attention": round(attn_mean, 5),
-                                    "quantisation": round(ms_per_step - attn_mean, 5)},
+                                    "quantisation": round(ms_per_step - attn_mean, 5),
+                                    "q_path": args.q_path},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk, "kernel_sha": kernel_sources_sha(),
         }
@@ -392,6 +404,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="libintfa", choices=["libintfa", "reference"])
+    ap.add_argument("--q-path", default="separate", choices=["fused", "separate"],
+                    help="quantise Q in its own pass (default, faster) or inside the attention kernel")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -142,6 +142,24 @@ int intfa_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q
                         int L, int d, int causal, void *O_f16, void *stream);
 
 /*
+ * The same fused attention with Q given in fp16: each 128-query tile is
+ * quantised per token inside the kernel (IntAttention section 2.1, eq. 3,
+ * token-level as INT-FlashAttention's abstract specifies; bit-identical codes
+ * and scales to intfa_quantize_per_token), so Q_hat never travels through
+ * HBM.  The pages describe quantisation and attention as separate steps; this
+ * fusion is an implementation choice of this library.
+ *
+ *   Q_f16   : fp16 [B][H][L][d], 16-byte aligned.
+ *   s_Q_out : fp32 [B][H][L] out (the per-token scales), or NULL.
+ *   Other arguments, results and error behaviour as intfa_attention_fwd; O
+ *   equals intfa_attention_fwd's output on intfa_quantize_per_token(Q) bit
+ *   for bit.
+ */
+int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *Vt_q,
+                            const float *s_K, const float *s_V, int B, int H, int L, int d,
+                            int causal, void *O_f16, float *s_Q_out, void *stream);
+
+/*
  * Debug: the integer logits S = Q_hat K_hat^T (IntAttention eq. 4) for every
  * head, int32 [B][H][L][L], computed by the same TMA + tcgen05 path the fused
  * kernel uses for its first contraction.  Same layout rules as

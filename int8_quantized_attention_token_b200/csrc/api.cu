@@ -91,7 +91,6 @@ extern "C" int intfa_forward(const void *Q_f16, const void *K_f16, const void *V
         (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return INTFA_ERR_MISALIGNED;
     uint8_t *w = static_cast<uint8_t *>(workspace);
-    int8_t *q = reinterpret_cast<int8_t *>(w + lo.q);
     int8_t *k = reinterpret_cast<int8_t *>(w + lo.k);
     int8_t *vt = reinterpret_cast<int8_t *>(w + lo.vt);
     float *sq = reinterpret_cast<float *>(w + lo.sq);
@@ -100,6 +99,10 @@ extern "C" int intfa_forward(const void *Q_f16, const void *K_f16, const void *V
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t rows = static_cast<int64_t>(B) * H * L;
     const int64_t bh = static_cast<int64_t>(B) * H;
+    // Q in its own pass: quantising it inside the attention kernel
+    // (intfa_attention_fwd_q16) saves the pass but costs more issue slots on
+    // the attention kernel's sub-partitions than the pass takes.
+    int8_t *q = reinterpret_cast<int8_t *>(w + lo.q);
     int rc = launch_quantize_per_token(Q_f16, rows, d, q, sq, s);
     if (!rc) rc = launch_quantize_per_token(K_f16, rows, d, k, sk, s);
     if (!rc) rc = launch_quantize_per_tensor(V_f16, bh, L, d, 1, vt, sv, w + lo.ws, s);

@@ -53,6 +53,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_math.cuh"
 
 namespace intfa {
 
@@ -62,7 +63,10 @@ namespace {
 
 constexpr int BM = 128;                       // query rows per CTA
 constexpr int BN = 128;                       // keys per block
-constexpr int NS = 5;                         // K/V ring depth
+// K/V ring depth
+template <bool kQ16>
+constexpr int kv_stages() { return 5; }
+constexpr int kQHalf = BM / 2;                // fp16 Q rows staged at a time (in-kernel quantiser)
 constexpr int kThreads = 640;                 // 20 warps = 5 warpgroups
 constexpr int SB = 3;                         // TMEM S buffers
 constexpr int OB = 1;                         // TMEM P V blocks
@@ -72,26 +76,28 @@ constexpr int AB = 4;                         // alpha ring depth (prep -> outpu
 // d-column fp32 row, takes registers from the other three.  The shares add up
 // to at most the launch total.
 constexpr int kLaunchRegs = 96;
-template <int D>
+template <int D, bool kQ16>
 struct RegSplit {   // d = 128: the output row alone is 128 registers
     static constexpr uint32_t kExp = 72;      // each of the two exp warpgroups
     static constexpr uint32_t kPrep = 96;
     static constexpr uint32_t kOutput = 192;
-    static constexpr uint32_t kOther = 48;
+    static constexpr uint32_t kOther = 48;   // also the in-kernel Q quantiser (roles 18, 19)
 };
-template <>
-struct RegSplit<64> {
+template <bool kQ16>
+struct RegSplit<64, kQ16> {
     static constexpr uint32_t kExp = 72;
-    static constexpr uint32_t kPrep = 96;
+    static constexpr uint32_t kPrep = kQ16 ? 88 : 96;
     static constexpr uint32_t kOutput = 184;
-    static constexpr uint32_t kOther = 56;
+    static constexpr uint32_t kOther = kQ16 ? 64 : 56;
 };
-template <int D>
+template <int D, bool kQ16>
 constexpr bool split_fits() {
-    return 128 * (2 * RegSplit<D>::kExp + RegSplit<D>::kPrep + RegSplit<D>::kOutput + RegSplit<D>::kOther) <=
-           kThreads * kLaunchRegs;
+    using R = RegSplit<D, kQ16>;
+    return 128 * (2 * R::kExp + R::kPrep + R::kOutput + R::kOther) <= kThreads * kLaunchRegs;
 }
-static_assert(split_fits<128>() && split_fits<64>(), "register split exceeds the launch allocation");
+static_assert(split_fits<128, false>() && split_fits<64, false>() && split_fits<128, true>() &&
+                  split_fits<64, true>(),
+              "register split exceeds the launch allocation");
 // Warp roles inside the fifth warpgroup (warps 16-19).
 constexpr int kProducerWarp = 16;
 constexpr int kMmaWarp = 17;
@@ -159,9 +165,11 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 
 // ------------------------------------------------------- shared memory ---
 
-template <int D>
+template <int D, bool kQ16>
 struct alignas(1024) AttnSmem {
+    static constexpr int NS = kv_stages<kQ16>();
     uint8_t q[2][BM * D];       // Q_hat tiles (two query tiles in flight), K-major, TMA-swizzled
+    uint8_t qs[kQ16 ? kQHalf * D * 2 : 1024];   // half an fp16 Q tile for the in-kernel quantiser
     uint8_t k[NS][BN * D];      // K_hat tiles
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
@@ -176,16 +184,19 @@ struct alignas(1024) AttnSmem {
     uint64_t a_empty[AB][4];    // output warp k -> prep warp k
     uint64_t o_full[OB], o_empty[OB];
     uint64_t l_full[2], l_empty[2];
+    float sq[8][BM];            // in-kernel Q quantiser -> prep: s_Q of tile i (slot i mod 8)
+    uint64_t sq_full[8];
+    uint64_t qs_full, qs_empty; // fp16 Q staging: TMA -> quantiser warps -> next TMA
     uint64_t mma_drain;
     uint32_t tmem_base;
     int abort_flag;
 };
 
-template <int D>
+template <int D, bool kQ16>
 constexpr size_t attn_smem_bytes() {
     // 1024 for manual alignment; D = 64 is padded so that only one CTA (which
     // holds all 512 TMEM columns) is resident per SM.
-    size_t s = sizeof(AttnSmem<D>) + 1024;
+    size_t s = sizeof(AttnSmem<D, kQ16>) + 1024;
     return s < 120 * 1024 ? 120 * 1024 : s;
 }
 
@@ -198,9 +209,9 @@ __device__ __forceinline__ uint8_t *smem_aligned_1024() {
     return smem_raw + off;
 }
 
-template <int D>
-__device__ __forceinline__ AttnSmem<D> &get_smem() {
-    return *reinterpret_cast<AttnSmem<D> *>(smem_aligned_1024());
+template <int D, bool kQ16>
+__device__ __forceinline__ AttnSmem<D, kQ16> &get_smem() {
+    return *reinterpret_cast<AttnSmem<D, kQ16> *>(smem_aligned_1024());
 }
 
 // ----------------------------------------------------------- tiles ---
@@ -306,13 +317,19 @@ __device__ __forceinline__ void max_v(const uint32_t (&w)[32], float (&mx)[4]) {
 
 // ---------------------------------------------------------------- kernel ---
 
-template <int D>
+// kQ16: Q arrives as fp16 (Qh) and is quantised per token inside the kernel
+// by roles 18-19 (bit-identical to quant_per_token_kernel); its scales go to
+// the prep warps through shared memory and, if sQ_out is set, to global.
+// Otherwise Q_hat arrives through tmQ and s_Q through sQ.
+template <int D, bool kQ16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
                     const float *__restrict__ sK, const float *__restrict__ sV,
-                    __half *__restrict__ O, int BH, int L, int causal) {
-    AttnSmem<D> &sm = get_smem<D>();
+                    __half *__restrict__ O, int BH, int L, int causal,
+                    const uint4 *__restrict__ Qh, float *__restrict__ sQ_out) {
+    AttnSmem<D, kQ16> &sm = get_smem<D, kQ16>();
+    constexpr int NS = AttnSmem<D, kQ16>::NS;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     // Role numbering: the producer / MMA warpgroup (roles 16-19) runs on the
@@ -329,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.q_full[b], 1);
+            mbar_init(&sm.q_full[b], kQ16 ? 64 : 1);
             mbar_init(&sm.q_empty[b], 1);
             mbar_init(&sm.l_full[b], 2 * BM);
             mbar_init(&sm.l_empty[b], BM);
@@ -353,6 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.o_full[b], 1);
             mbar_init(&sm.o_empty[b], BM);
         }
+        for (int b = 0; b < 8; ++b) mbar_init(&sm.sq_full[b], 64);
+        mbar_init(&sm.qs_full, 1);
+        mbar_init(&sm.qs_empty, 64);
         mbar_init(&sm.mma_drain, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -369,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tbase + 128 * SB;   // int32 P V block o at column tO + 128 o
 
     if (warp >= 16) {
-      regs_to<RegSplit<D>::kOther>();
+      regs_to<RegSplit<D, kQ16>::kOther>();
       if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ---
         if (lane == 0) {
@@ -396,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int g = 0, q_issued = 0;
         Ring<NS> kv;
         while (c.t < total) {
-            if (c.j == 0) {   // a new tile: its Q_hat into buffer i mod 2
+            if (!kQ16 && c.j == 0) {   // a new tile: its Q_hat into buffer i mod 2
                 const int qb = c.i & 1;
                 if (c.i >= 2 && !warp_wait(&sm.q_empty[qb], ((c.i >> 1) - 1) & 1, abort_flag, 8)) break;
                 if (lane == 0) {
@@ -422,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             kv.next();
         }
         // Drain: the last load issued into each stage and Q buffer has landed.
-        for (int b = 0; b < 2 && b < q_issued; ++b) {
+        for (int b = 0; !kQ16 && b < 2 && b < q_issued; ++b) {
             const int last = b + ((q_issued - 1 - b) / 2) * 2;
             drain_wait(&sm.q_full[b], (last >> 1) & 1);
         }
@@ -505,9 +525,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         drain_wait(&sm.mma_drain, 0);
         __syncwarp();
       }
-      // the other two warps of this warpgroup have no role
+      else if (kQ16) {
+        // ------------------------------------------ Q quantiser (18, 19) ---
+        // G lanes per row of D fp16 (8 per lane); the two warps take row
+        // slices alternately.  Codes go straight into the swizzled K-major
+        // layout the TMA would have produced (128-byte swizzle for D = 128:
+        // 16-byte chunk k of row r at k ^ (r mod 8); 64-byte for D = 64:
+        // chunk k at k ^ ((r / 2) mod 4)).
+        constexpr int G = D / 8;
+        constexpr int kRowsPerWarp = 32 / G;
+        const int wq = warp - 18, sub = lane % G;
+        bool ok = true;
+        for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
+            const Tile T = tile_at(t, ntiles, L, causal);
+            const int qb = i & 1, ss = i & 7;
+            // buffer qb held tile i - 2: its last Q K^T has been issued and run
+            if (i >= 2 && !warp_wait(&sm.q_empty[qb], ((i >> 1) - 1) & 1, abort_flag, 18)) break;
+            const uint32_t qbase = smem_u32(sm.q[qb]);
+            const uint4 *stage = reinterpret_cast<const uint4 *>(sm.qs);
+            // the tile's fp16 rows in two halves of kQHalf rows through the
+            // staging buffer: warp 18 issues the TMA once both warps have
+            // read the previous half
+            for (int h = 0; ok && h < 2; ++h) {
+                const int n = 2 * i + h;
+                if (wq == 0) {
+                    if (n >= 1 && !warp_wait(&sm.qs_empty, (n - 1) & 1, abort_flag, 21)) { ok = false; break; }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sm.qs_full, kQHalf * D * 2);
+                        tma_load_3d(&tmQ, &sm.qs_full, sm.qs, 0, T.q0 + kQHalf * h, T.bh);
+                    }
+                    __syncwarp();
+                }
+                if (!warp_wait(&sm.qs_full, n & 1, abort_flag, 20)) { ok = false; break; }
+                for (int rr = wq * kRowsPerWarp; rr < kQHalf; rr += 2 * kRowsPerWarp) {
+                    const int rs = rr + lane / G;   // row in the staging half
+                    const int r = kQHalf * h + rs;  // row in the tile
+                    const int qi = T.q0 + r;
+                    float f[8];
+                    qmath::unpack8(stage[rs * G + sub], f);   // rows past L were zero-filled by TMA
+                    float amax = qmath::absmax8(f);
+#pragma unroll
+                    for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+                    const float s = qmath::div127(amax);
+                    const uint2 w = qmath::codes8(f, s, qmath::rcp_or_zero(s));
+                    const int ch = sub >> 1;   // 16-byte chunk of bytes 8 sub .. 8 sub + 7
+                    const uint32_t sw = D == 128 ? static_cast<uint32_t>(r & 7) : static_cast<uint32_t>((r >> 1) & 3);
+                    const uint32_t addr = qbase + static_cast<uint32_t>(r * D) +
+                                          ((static_cast<uint32_t>(ch) ^ sw) << 4) + 8u * static_cast<uint32_t>(sub & 1);
+                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(w.x), "r"(w.y) : "memory");
+                    if (sub == 0) {
+                        sm.sq[ss][r] = s;
+                        if (sQ_out != nullptr && qi < L) sQ_out[static_cast<int64_t>(T.bh) * L + qi] = s;
+                    }
+                }
+                mbar_arrive(&sm.qs_empty);   // this half has been read
+            }
+            if (!ok) break;
+            fence_proxy_async_smem();   // codes visible to the tensor core
+            mbar_arrive(&sm.q_full[qb]);
+            mbar_arrive(&sm.sq_full[ss]);
+        }
+      }
+      // otherwise the other two warps of this warpgroup have no role
     } else if (warp < 8) {
-        regs_to<RegSplit<D>::kExp>();
+        regs_to<RegSplit<D, kQ16>::kExp>();
         // ------------------------------------------------------- exp ---
         // Two warps per TMEM lane quadrant: half hf takes keys 64 hf .. 64 hf
         // + 63 of each block (chunks 2 hf, 2 hf + 1) and writes their 16 code
@@ -579,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sm.l_full[ls]);
         }
     } else if (warp < 12) {
-        regs_to<RegSplit<D>::kPrep>();
+        regs_to<RegSplit<D, kQ16>::kPrep>();
         // ------------------------------------------------------ prep ---
         const int row = rtid - 256;
         const int quad = warp - 8;
@@ -591,15 +672,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         Ring<SB> sb;
         Ring<NS> ks;
         Ring<AB> as;
-        for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
             const Tile T = tile_at(t, ntiles, L, causal);
             const int qi = T.q0 + row;
+            float s_q;
+            if constexpr (kQ16) {
+                // slot i mod 8 cannot be rewritten before this read: the
+                // quantiser runs at most two tiles ahead of Q K^T, which runs
+                // at most SB = 3 blocks ahead of this warp
+                if (!warp_wait(&sm.sq_full[i & 7], (i >> 3) & 1, abort_flag, 19)) break;
+                s_q = sm.sq[i & 7][row];
+            } else {
+                s_q = qi < L ? __ldg(sQ + static_cast<int64_t>(T.bh) * L + qi) : 0.0f;
+            }
             // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c (S_ij s_K[j]).
             // Clamped to a tiny positive value: a zero Q row then still maps masked
             // keys (v = -inf) to p = 0 and visible keys to p = 1.
-            const float c = fmaxf((qi < L ? __ldg(sQ + static_cast<int64_t>(T.bh) * L + qi) : 0.0f) *
-                                      (kLog2e / sqrtf(static_cast<float>(D))),
-                                  1e-30f);
+            const float c = fmaxf(s_q * (kLog2e / sqrtf(static_cast<float>(D))), 1e-30f);
             const int lim = causal ? min(L, qi + 1) : L;
             float m_old = -INFINITY;
             for (int j = 0; j < T.nb; ++j, ++g, sb.next(), ks.next(), as.next()) {
@@ -649,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        regs_to<RegSplit<D>::kOutput>();
+        regs_to<RegSplit<D, kQ16>::kOutput>();
         // ------------------------------------------------ output side ---
         const int row = rtid - 384;
         const int quad = warp - 12;
@@ -836,17 +925,18 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 3-D uint8 tensor map: dims (x = inner, y, z), byte strides of y and z, box (bx, by, 1).
+// 3-D tensor map (uint8 unless dtype says otherwise): dims (x = inner, y, z) in
+// elements, byte strides of y and z, box (bx, by, 1) in elements.
 int make_map(CUtensorMap *map, const void *base, uint64_t x, uint64_t y, uint64_t z,
              uint64_t stride_y, uint64_t stride_z, uint32_t bx, uint32_t by,
-             CUtensorMapSwizzle swz) {
+             CUtensorMapSwizzle swz, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return INTFA_ERR_CUDA;
     const cuuint64_t dims[3] = {x, y, z};
     const cuuint64_t strides[2] = {stride_y, stride_z};
     const cuuint32_t box[3] = {bx, by, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims,
+    const CUresult r = enc(map, dtype, 3, const_cast<void *>(base), dims,
                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? INTFA_OK : INTFA_ERR_CUDA;
@@ -870,27 +960,34 @@ unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
     return static_cast<unsigned>(g);
 }
 
-template <int D>
-int launch_attn(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
-                const float *sK, const float *sV, int B, int H, int L, int causal, void *O,
-                cudaStream_t stream) {
+// Qq (int8, with sQ) when !kQ16; Qh (fp16, scales optionally to sQ_out) when kQ16.
+template <int D, bool kQ16>
+int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sQ,
+                float *sQ_out, const float *sK, const float *sV, int B, int H, int L, int causal,
+                void *O, cudaStream_t stream) {
     const int BH = B * H;
     const int64_t ld = intfa_vt_ld(L);
     const CUtensorMapSwizzle swz = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap mq, mk, mv;
-    int rc = make_map(&mq, Qq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BM, swz);
-    if (!rc) rc = make_map(&mk, Kq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BN, swz);
+    int rc = make_map(&mk, Kq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BN, swz);
+    if (!rc) {
+        if (kQ16)   // fp16 Q rows, unswizzled (the quantiser reads them with plain loads)
+            rc = make_map(&mq, Qh, D, L, BH, D * 2, static_cast<uint64_t>(L) * D * 2, D, kQHalf,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+        else
+            rc = make_map(&mq, Qq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BM, swz);
+    }
     if (!rc) rc = make_map(&mv, Vt, ld, D, BH, ld, static_cast<uint64_t>(ld) * D, BN, D,
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
-    const size_t smem = attn_smem_bytes<D>();
-    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(smem)));
+    const size_t smem = attn_smem_bytes<D, kQ16>();
+    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D, kQ16>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
     if (rc) return rc;
     // The in-kernel register split assumes exactly kLaunchRegs per thread at
     // launch; a different count could leave setmaxnreg.inc waiting forever.
     cudaFuncAttributes fa;
-    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>));
+    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kQ16>));
     if (rc) return rc;
     if (fa.numRegs != kLaunchRegs) return INTFA_ERR_UNSUPPORTED;
     const int ntiles = (L + BM - 1) / BM;
@@ -899,8 +996,9 @@ int launch_attn(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const floa
     if (!rc) rc = cuda_status(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
     if (rc) return rc;
     const unsigned grid = persistent_grid(static_cast<int64_t>(BH) * ntiles, ntiles, causal, nsm);
-    attn_fwd_kernel<D><<<grid, kThreads, smem, stream>>>(mq, mk, mv, sQ, sK, sV,
-                                                          static_cast<__half *>(O), BH, L, causal);
+    attn_fwd_kernel<D, kQ16><<<grid, kThreads, smem, stream>>>(
+        mq, mk, mv, sQ, sK, sV, static_cast<__half *>(O), BH, L, causal, static_cast<const uint4 *>(Qh),
+        sQ_out);
     return cuda_status(cudaGetLastError());
 }
 
@@ -926,8 +1024,20 @@ int launch_debug_qk(const int8_t *Qq, const int8_t *Kq, int BH, int L, int32_t *
 int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                          const float *sK, const float *sV, int B, int H, int L, int d, int causal,
                          void *O, cudaStream_t stream) {
-    if (d == 128) return launch_attn<128>(Qq, Kq, Vt, sQ, sK, sV, B, H, L, causal, O, stream);
-    if (d == 64) return launch_attn<64>(Qq, Kq, Vt, sQ, sK, sV, B, H, L, causal, O, stream);
+    if (d == 128)
+        return launch_attn<128, false>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal, O, stream);
+    if (d == 64)
+        return launch_attn<64, false>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal, O, stream);
+    return INTFA_ERR_UNSUPPORTED;
+}
+
+int launch_attention_fwd_q16(const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sK,
+                             const float *sV, int B, int H, int L, int d, int causal, void *O,
+                             float *sQ_out, cudaStream_t stream) {
+    if (d == 128)
+        return launch_attn<128, true>(nullptr, Qh, Kq, Vt, nullptr, sQ_out, sK, sV, B, H, L, causal, O, stream);
+    if (d == 64)
+        return launch_attn<64, true>(nullptr, Qh, Kq, Vt, nullptr, sQ_out, sK, sV, B, H, L, causal, O, stream);
     return INTFA_ERR_UNSUPPORTED;
 }
 
@@ -962,6 +1072,22 @@ extern "C" int intfa_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const i
         return INTFA_ERR_MISALIGNED;
     return launch_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
                                 static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *Vt_q,
+                                       const float *s_K, const float *s_V, int B, int H, int L, int d,
+                                       int causal, void *O_f16, float *s_Q_out, void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    if (!Q_f16 || !K_q || !Vt_q || !s_K || !s_V || !O_f16) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_f16) || !aligned16(K_q) || !aligned16(Vt_q) || !aligned16(O_f16) ||
+        (reinterpret_cast<uintptr_t>(s_K) & 3u) || (reinterpret_cast<uintptr_t>(s_V) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_Q_out) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    return launch_attention_fwd_q16(Q_f16, K_q, Vt_q, s_K, s_V, B, H, L, d, causal, O_f16, s_Q_out,
+                                    static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int intfa_debug_qk(const int8_t *Q_q, const int8_t *K_q, int B, int H, int L, int d,

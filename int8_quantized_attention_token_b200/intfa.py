@@ -49,6 +49,7 @@ def lib():
         "intfa_quantize_per_tensor": ([P, I64, I64, I, I, P, P, P, SZ, P], I),
         "intfa_quantize_per_tensor_noalloc": ([P, I64, I64, I, I, P, P, P], I),
         "intfa_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
+        "intfa_attention_fwd_q16": ([P, P, P, P, P, I, I, I, I, I, P, P, P], I),
         "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
         "intfa_forward_workspace_size": ([I, I, I, I], SZ),
         "intfa_forward_workspace_layout": ([I, I, I, I, ctypes.POINTER(SZ)], I),
@@ -175,6 +176,25 @@ def intfa_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, O=None, str
     _check(lib().intfa_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
                                      _ptr(s_V), B, H, L, d, int(bool(causal)), _ptr(O),
                                      _stream(stream)), "intfa_attention_fwd")
+    return O
+
+
+def intfa_attention_fwd_q16(Q, K_q, Vt_q, s_K, s_V, causal: bool, O=None, s_Q=None, stream=None):
+    """Q fp16 [B, H, L, d] (quantised per token inside the kernel); K_q, Vt_q,
+    s_K, s_V as for intfa_attention_fwd  ->  O fp16 [B, H, L, d].  If s_Q (fp32
+    [B, H, L]) is given, the kernel writes Q's per-token scales into it."""
+    _need(Q, torch.float16, "Q")
+    for t, n in ((K_q, "K_q"), (Vt_q, "Vt_q")):
+        _need(t, torch.int8, n)
+    for t, n in ((s_K, "s_K"), (s_V, "s_V")):
+        _need(t, torch.float32, n)
+    if s_Q is not None:
+        _need(s_Q, torch.float32, "s_Q")
+    B, H, L, d = Q.shape
+    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q.device) if O is None else O
+    _check(lib().intfa_attention_fwd_q16(_ptr(Q), _ptr(K_q), _ptr(Vt_q), _ptr(s_K), _ptr(s_V), B, H, L, d,
+                                         int(bool(causal)), _ptr(O), _ptr(s_Q) if s_Q is not None else None,
+                                         _stream(stream)), "intfa_attention_fwd_q16")
     return O
 
 

@@ -74,6 +74,15 @@ def test_attention_rejects(L):
     assert L.intfa_attention_fwd(*a, 1, 1, 128, 64, 0, FAKE + 8, None) == 3       # O alignment
     assert L.intfa_attention_fwd(FAKE + 1, *a[1:], 1, 1, 128, 64, 0, FAKE, None) == 3
     assert L.intfa_attention_fwd(*a, 1, 1, 300000, 64, 0, FAKE, None) == 2        # int32 bound
+    # fp16-Q variant: Q, K_q, Vt_q, s_K, s_V, B, H, L, d, causal, O, s_Q_out
+    q = [FAKE] * 5
+    assert L.intfa_attention_fwd_q16(*q, 1, 1, 128, 96, 0, FAKE, None, None) == 2    # d
+    assert L.intfa_attention_fwd_q16(*q, 1, 0, 128, 64, 0, FAKE, None, None) == 1    # H
+    assert L.intfa_attention_fwd_q16(*q, 1, 1, 128, 64, 3, FAKE, None, None) == 1    # causal flag
+    assert L.intfa_attention_fwd_q16(None, *q[1:], 1, 1, 128, 64, 0, FAKE, None, None) == 1
+    assert L.intfa_attention_fwd_q16(*q, 1, 1, 128, 64, 0, None, None, None) == 1    # O
+    assert L.intfa_attention_fwd_q16(FAKE + 2, *q[1:], 1, 1, 128, 64, 0, FAKE, None, None) == 3
+    assert L.intfa_attention_fwd_q16(*q, 1, 1, 128, 64, 0, FAKE, FAKE + 2, None) == 3  # s_Q_out
     assert L.intfa_debug_qk(FAKE, FAKE, 1, 1, 128, 32, FAKE, None) == 2
     assert L.intfa_debug_qk(FAKE, None, 1, 1, 128, 64, FAKE, None) == 1
 
