@@ -27,7 +27,10 @@
 //               ahead of P V; P V with the P codes read straight from TMEM
 //               (aliasing columns of the S buffer they came from) into the
 //               TMEM int32 P V block; owns the TMEM allocation (S0..S2: 3 x
-//               128 columns; P V block: 128 columns).
+//               128 columns; P V block: 128 columns).  Before the INT8 MMAs
+//               of a block, one fp16 MMA of constant operands sets the target
+//               accumulator to a float bias (kBiasA), so that the readers
+//               get exact fp32 values with one add instead of a conversion.
 //   warps 8-11  "prep" (one thread per query row): S row -> v = S s_K in
 //               fp32 (written back over S in TMEM), causal / ragged mask,
 //               running max m and alpha.
@@ -116,6 +119,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 // 1.5 * 2^23: for 0 <= y < 2^22, fl(y + 1.5 * 2^23) is 1.5 * 2^23 + RNE(y),
 // so RNE(y) sits in the low mantissa bits of that float.
 constexpr float kMagic = 12582912.0f;
+// Accumulator bias.  Each S buffer and the P V block are first set to the
+// fp32 value 1.5 * 2^23 (bit pattern 0x4B400000) by one fp16 MMA of constant
+// operands (16 products 1024 * 768, all exact), and the INT8 MMAs then add
+// their int32 results to that bit pattern.  For |x| < 2^22 the sum
+// 0x4B400000 + x is the bit pattern of the float 1.5 * 2^23 + x, so an
+// accumulator read as fp32 minus kMagic is exactly float(x): no int -> float
+// conversion instruction is needed (|S|, |P V| <= 127^2 * 128 < 2^22).
+constexpr uint16_t kBiasA = 0x6400;   // fp16 1024
+constexpr uint16_t kBiasB = 0x6200;   // fp16 768
+
+// (-kMagic, -kMagic) as an f32x2 operand, materialised where it is used (an
+// opaque move, so that the compiler does not keep it in registers across
+// the roles of the kernel).
+__device__ __forceinline__ uint64_t neg_bias2() {
+    uint64_t r;
+    asm volatile("mov.b64 %0, 0xCB400000CB400000;" : "=l"(r));
+    return r;
+}
 
 // -------------------------------------------------------- bounded waits ---
 
@@ -176,6 +197,7 @@ struct alignas(1024) AttnSmem {
     float4 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha, c, -) per row and S buffer
     float alpha_o[AB][BM];      // prep -> output: alpha of block j (slot j mod AB)
     float lsum[2][2][BM];       // exp -> output: row sums of each key half (slot = tile mod 2)
+    uint16_t bias_ab[2][192];   // fp16 operands of the bias MMA: 1024 (A), 768 (B)
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
     uint64_t s_full[SB], p_full[SB];
@@ -199,6 +221,9 @@ constexpr size_t attn_smem_bytes() {
     size_t s = sizeof(AttnSmem<D, kQ16>) + 1024;
     return s < 120 * 1024 ? 120 * 1024 : s;
 }
+static_assert(attn_smem_bytes<128, false>() <= 227 * 1024 && attn_smem_bytes<128, true>() <= 227 * 1024 &&
+                  attn_smem_bytes<64, false>() <= 227 * 1024 && attn_smem_bytes<64, true>() <= 227 * 1024,
+              "shared memory above the per-block limit");
 
 // Dynamic shared memory rounded up to 1024 B by pointer arithmetic on the
 // __shared__ array itself, so that the compiler keeps every access in the
@@ -278,16 +303,16 @@ struct Ring {
 
 // ------------------------------------------------------- prep pieces ---
 
-// v = fl(S s_K) in place (int32 -> fp32 is exact: |S| <= 127^2 d < 2^24).
+// v = fl(S s_K) in place, from the biased accumulator (fl(x - kMagic) = S
+// exactly).
 __device__ __forceinline__ void scores_to_v(uint32_t (&w)[32], const float4 *sk4) {
+    const uint64_t nb2 = neg_bias2();
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         const float4 k4 = sk4[q];
-        const uint64_t a = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q])),
-                                         __int2float_rn(static_cast<int32_t>(w[4 * q + 1]))),
+        const uint64_t a = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), nb2),
                                  f2_pack(k4.x, k4.y));
-        const uint64_t e = fmul2(f2_pack(__int2float_rn(static_cast<int32_t>(w[4 * q + 2])),
-                                         __int2float_rn(static_cast<int32_t>(w[4 * q + 3]))),
+        const uint64_t e = fmul2(fadd2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), nb2),
                                  f2_pack(k4.z, k4.w));
         float v0, v1, v2, v3;
         f2_unpack(a, v0, v1);
@@ -377,6 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    if (tid < 2 * 192) {
+        sm.bias_ab[tid / 192][tid % 192] = tid < 192 ? kBiasA : kBiasB;
+        fence_proxy_async_smem();   // read by the tensor core
+    }
     if (warp == kMmaWarp) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -458,6 +487,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kSboQK = 8 * D;      // 8 rows of D bytes
         const uint32_t idesc_qk = make_idesc_i8(BM, BN);
         const uint32_t idesc_pv = make_idesc_i8(BM, D);
+        // bias MMA operands: every element of A and B is the same constant, so
+        // the descriptors may let core matrices overlap (16-byte strides keep
+        // all reads inside the 384-byte arrays)
+        const uint32_t idesc_bias_s = make_idesc_f16(BM, BN);
+        const uint32_t idesc_bias_o = make_idesc_f16(BM, D);
+        const uint64_t bias_a = make_sdesc_noswz(smem_u32(sm.bias_ab[0]), 16, 16);
+        const uint64_t bias_b = make_sdesc_noswz(smem_u32(sm.bias_ab[1]), 16, 16);
         bool ok = true;
         // qc walks the blocks whose Q K^T is issued, SB blocks ahead of pc,
         // which walks the blocks whose P V is issued.
@@ -475,9 +511,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 const uint64_t qdesc = make_sdesc(smem_u32(sm.q[qb]), kSboQK, kSwQK);
                 const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
+                mma_f16_ss(tS + sb * BN, bias_a, bias_b, idesc_bias_s, 0);
 #pragma unroll
                 for (int k = 0; k < D / 32; ++k)
-                    mma_i8_ss(tS + sb * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, k > 0);
+                    mma_i8_ss(tS + sb * BN, qdesc + 2 * k, kdesc + 2 * k, idesc_qk, 1);
                 mma_commit(&sm.s_full[sb]);
                 if (qc.j == qc.T.nb - 1) mma_commit(&sm.q_empty[qb]);   // last use of this Q tile
             }
@@ -504,10 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             if (lane == 0) {
                 const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
+                mma_f16_ss(tO, bias_a, bias_b, idesc_bias_o, 0);
 #pragma unroll
                 for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k ..: see the exp warps
-                    mma_i8_ts(tO, tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k, idesc_pv,
-                              k > 0);
+                    mma_i8_ts(tO, tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k, idesc_pv, 1);
                 mma_commit(&sm.o_full[0]);
                 mma_commit(&sm.kv_empty[st]);
             }
@@ -755,8 +792,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < D / 2; ++e) o2[e] = 0ull;
             for (int j = 0; j < T.nb; ++j, as.next(), oph ^= 1u) {
                 const int ab = as.idx;
-                // o = alpha o + (P V block), the int32 block turned into fp32
-                // exactly (|x| <= 127^2 128 < 2^24)
+                // o = alpha o + (P V block), the biased block turned into fp32
+                // exactly (fl(x - kMagic), |P V| <= 127^2 128 < 2^22)
                 const uint32_t to = tO;
                 if (!warp_wait(&sm.o_full[0], oph, abort_flag, 9)) { ok = false; break; }
                 if (!warp_wait(&sm.a_full[ab][quad], as.ph, abort_flag, 10)) { ok = false; break; }
@@ -764,6 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float alpha = sm.alpha_o[ab][row];
                 mbar_arrive(&sm.a_empty[ab][quad]);
                 const uint64_t a2 = f2_pack(alpha, alpha);
+                // x - kMagic as fma(x, 1, -kMagic) (exact; compiles to fewer
+                // registers than the add form here)
+                const uint64_t nb2 = neg_bias2();
+                const uint64_t one2 = f2_pack(1.0f, 1.0f);
                 // the block in pairs of 32-column chunks; once the last pair is
                 // in registers the P V block is released for the next block
 #pragma unroll
@@ -778,14 +819,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w0[2 * e])),
-                                                   __int2float_rn(static_cast<int32_t>(w0[2 * e + 1])));
+                        const uint64_t x = ffma2(f2_pack(__uint_as_float(w0[2 * e]), __uint_as_float(w0[2 * e + 1])), one2, nb2);
                         o2[32 * pr + e] = ffma2(o2[32 * pr + e], a2, x);
                     }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const uint64_t x = f2_pack(__int2float_rn(static_cast<int32_t>(w1[2 * e])),
-                                                   __int2float_rn(static_cast<int32_t>(w1[2 * e + 1])));
+                        const uint64_t x = ffma2(f2_pack(__uint_as_float(w1[2 * e]), __uint_as_float(w1[2 * e + 1])), one2, nb2);
                         o2[32 * pr + 16 + e] = ffma2(o2[32 * pr + 16 + e], a2, x);
                     }
                 }

@@ -157,6 +157,17 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, FP16 x FP16 -> FP32.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, INT8 x INT8 -> INT32 (A read from TMEM).
 __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -302,6 +313,17 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t sbo_byte
     d |= static_cast<uint64_t>(swizzle_code & 0x7u) << 61;          // layout type
     return d;
 }
+// Shared-memory matrix descriptor, no swizzle, K-major: 8-row x 16-byte core
+// matrices, lbo_bytes apart along K and sbo_bytes apart along M / N.
+__device__ __forceinline__ uint64_t make_sdesc_noswz(uint32_t saddr, uint32_t lbo_bytes,
+                                                     uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;   // version; layout type 0 = no swizzle
+    return d;
+}
 constexpr uint32_t kSwizzle128B = 2;
 constexpr uint32_t kSwizzle64B = 4;
 
@@ -312,6 +334,14 @@ __host__ __device__ constexpr uint32_t make_idesc_i8(int M, int N) {
            | (1u << 7)                                 // A: signed 8-bit
            | (1u << 10)                                // B: signed 8-bit
            | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor, kind::f16: D = f32, A = B = f16, both K-major,
+// dense, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N) {
+    return (1u << 4)                                   // D format: f32
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8 (A, B format 0: f16)
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
