@@ -18,11 +18,11 @@
 // order).  Every role runs through the CTA's whole stream of (tile, key
 // block) pairs with ring counters that do not restart at tile boundaries, so
 // the loads and Q K^T of the next tile overlap the last blocks and the
-// epilogue of the current one.  20 warps:
-//   role 16     TMA producer: each tile's Q_hat (two Q buffers), K_hat tile,
+// epilogue of the current one.  16 warps:
+//   role 12     TMA producer: each tile's Q_hat (two Q buffers), K_hat tile,
 //               V_hat^T tile and the block's s_K values into a 5-stage
 //               shared-memory ring.
-//   role 17     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
+//   role 13     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
 //               kind::i8 into one of three TMEM S buffers, three key blocks
 //               ahead of P V; P V with the P codes read straight from TMEM
 //               (aliasing columns of the S buffer they came from) into the
@@ -31,22 +31,21 @@
 //               of a block, one fp16 MMA of constant operands sets the target
 //               accumulator to a float bias (kBiasA), so that the readers
 //               get exact fp32 values with one add instead of a conversion.
-//   warps 8-11  "prep" (one thread per query row): S row -> v = S s_K in
-//               fp32 (written back over S in TMEM), causal / ragged mask,
-//               running max m and alpha.
-//   warps 12-15 output side (one thread per query row): folds each int32
+//   roles 0-7   softmax, two warpgroups taking alternate key blocks of the
+//               stream (one thread per query row, all 128 keys of the
+//               block): pass 1 v = S s_K (written back over S), causal /
+//               ragged mask, row max; the running max m from the other
+//               warpgroup's preceding block; alpha to the output side; pass 2
+//               p = 2^(c v - c m), the row sum and the P codes, written back
+//               to TMEM as the A operand of P V.  While one warpgroup is in
+//               pass 2 (special-function bound) the other can run pass 1.
+//   roles 8-11  output side (one thread per query row): folds each int32
 //               P V block into the row's fp32 accumulator, held in registers
 //               (o = alpha o + block), and writes the normalised fp16 row at
 //               the end of each tile.
-//   warps 0-7   "exp" (two warps per TMEM lane quadrant, each one thread per
-//               query row and half of the 128 keys): reads v in 32-column
-//               chunks, p = 2^(c v - c m), the row sum, and the P codes,
-//               which it writes back to TMEM as the A operand of P V.
-//   roles 18-19 idle.
-// Roles 16-19 run on hardware warps 0-3, roles 0-15 on hardware warps 4-19.
-// All per-row loops walk the row in 32-column chunks (one TMEM load each) and
-// are not unrolled across chunks, which keeps the three code paths that share
-// an SM sub-partition small enough for its instruction cache.
+//   roles 14-15 the in-kernel Q quantiser (fp16 Q entry point), else idle.
+// Roles 12-15 run on hardware warps 0-3, roles 0-11 on hardware warps 4-15;
+// a role keeps its hardware warp's TMEM lane quadrant (role mod 4).
 // Every wait is bounded (clock-based); a timeout records a status word,
 // raises a CTA-wide abort flag, drains in-flight copies and MMAs, frees TMEM
 // and returns.
@@ -70,40 +69,39 @@ constexpr int BN = 128;                       // keys per block
 template <bool kQ16>
 constexpr int kv_stages() { return 5; }
 constexpr int kQHalf = BM / 2;                // fp16 Q rows staged at a time (in-kernel quantiser)
-constexpr int kThreads = 640;                 // 20 warps = 5 warpgroups
+constexpr int kThreads = 512;                 // 16 warps = 4 warpgroups
 constexpr int SB = 3;                         // TMEM S buffers
 constexpr int OB = 1;                         // TMEM P V blocks
-constexpr int AB = 4;                         // alpha ring depth (prep -> output side)
+constexpr int AB = 4;                         // alpha ring depth (softmax -> output side); even
 // Register split (setmaxnreg): launched with kLaunchRegs per thread (checked
 // on the host before every launch); the output warpgroup, which holds a
-// d-column fp32 row, takes registers from the other three.  The shares add up
-// to at most the launch total.
-constexpr int kLaunchRegs = 96;
+// d-column fp32 row, and the two softmax warpgroups take registers from the
+// producer / MMA warpgroup.  The shares add up to at most the launch total.
+constexpr int kLaunchRegs = 128;
 template <int D, bool kQ16>
 struct RegSplit {   // d = 128: the output row alone is 128 registers
-    static constexpr uint32_t kExp = 72;      // each of the two exp warpgroups
-    static constexpr uint32_t kPrep = 96;
+    static constexpr uint32_t kSoft = 136;    // each of the two softmax warpgroups
     static constexpr uint32_t kOutput = 192;
-    static constexpr uint32_t kOther = 48;   // also the in-kernel Q quantiser (roles 18, 19)
+    static constexpr uint32_t kOther = 48;    // also the in-kernel Q quantiser (roles 14, 15)
 };
 template <bool kQ16>
 struct RegSplit<64, kQ16> {
-    static constexpr uint32_t kExp = 72;
-    static constexpr uint32_t kPrep = kQ16 ? 88 : 96;
-    static constexpr uint32_t kOutput = 184;
-    static constexpr uint32_t kOther = kQ16 ? 64 : 56;
+    static constexpr uint32_t kSoft = 136;
+    static constexpr uint32_t kOutput = 168;
+    static constexpr uint32_t kOther = 72;
 };
 template <int D, bool kQ16>
 constexpr bool split_fits() {
     using R = RegSplit<D, kQ16>;
-    return 128 * (2 * R::kExp + R::kPrep + R::kOutput + R::kOther) <= kThreads * kLaunchRegs;
+    return 128 * (2 * R::kSoft + R::kOutput + R::kOther) <= kThreads * kLaunchRegs;
 }
 static_assert(split_fits<128, false>() && split_fits<64, false>() && split_fits<128, true>() &&
                   split_fits<64, true>(),
               "register split exceeds the launch allocation");
-// Warp roles inside the fifth warpgroup (warps 16-19).
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
+// Warp roles inside the fourth warpgroup (roles 12-15).
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kQuantWarp = 14;   // and 15
 constexpr int kTmemCols = 512;
 
 // Moves this warpgroup from kLaunchRegs to R registers per thread with the
@@ -165,14 +163,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
-// A non-blocking probe issued ahead of time (its latency then overlaps other
-// work); settle() only waits if some lane's probe found the phase incomplete.
-__device__ __forceinline__ bool settle(bool probed, uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                       uint32_t site) {
-    if (__all_sync(0xFFFFFFFFu, probed)) return true;
-    return warp_wait(bar, parity, abort_flag, site);
-}
-
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     const long long t0 = clock64();
@@ -194,16 +184,17 @@ struct alignas(1024) AttnSmem {
     uint8_t k[NS][BN * D];      // K_hat tiles
     uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
     float sk[NS][BN];           // s_K of each key block
-    float4 cm_alpha[SB][BM];    // prep -> exp: (c m_new, alpha, c, -) per row and S buffer
-    float alpha_o[AB][BM];      // prep -> output: alpha of block j (slot j mod AB)
-    float lsum[2][2][BM];       // exp -> output: row sums of each key half (slot = tile mod 2)
+    float mrow[2][BM];          // softmax warpgroup w -> the other: running max after its latest block
+    float alpha_o[AB][BM];      // softmax -> output: alpha of block g (slot g mod AB)
+    float lsum[2][2][BM];       // softmax warpgroup w -> output: its share of the row sum (slot = tile mod 2)
+    float cml[2][2][BM];        //   ... and c m at its last block of the tile (the share's reference)
     uint16_t bias_ab[2][192];   // fp16 operands of the bias MMA: 1024 (A), 768 (B)
     uint64_t q_full[2], q_empty[2];
     uint64_t k_full[NS], v_full[NS], kv_empty[NS];
     uint64_t s_full[SB], p_full[SB];
-    uint64_t x_full[SB][4];     // prep warp k -> exp warp k (same TMEM lane quadrant)
-    uint64_t a_full[AB][4];     // prep warp k -> output warp k
-    uint64_t a_empty[AB][4];    // output warp k -> prep warp k
+    uint64_t m_full[2][4];      // softmax warpgroup w, warp k: mrow[w] rows of quadrant k written
+    uint64_t a_full[AB][4];     // softmax warp k -> output warp k
+    uint64_t a_empty[AB][4];    // output warp k -> softmax warp k
     uint64_t o_full[OB], o_empty[OB];
     uint64_t l_full[2], l_empty[2];
     float sq[8][BM];            // in-kernel Q quantiser -> prep: s_Q of tile i (slot i mod 8)
@@ -340,11 +331,33 @@ __device__ __forceinline__ void max_v(const uint32_t (&w)[32], float (&mx)[4]) {
     }
 }
 
+// One 32-key chunk of v: p = 2^(c v - c m) (<= 1; 0 for masked keys), the
+// running pair sums of p, and the 32 P codes RNE(127 p) packed four per word
+// (the code is the low byte of fl(127 p + 1.5 * 2^23)).
+__device__ __forceinline__ void exp_codes(const uint32_t (&w)[32], uint64_t c2, uint64_t ncm2, uint64_t k127,
+                                          uint64_t magic, uint64_t &ps01, uint64_t &ps23, uint32_t (&pk)[8]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float x0, x1, x2, x3;
+        f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), c2, ncm2), x0, x1);
+        f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2, ncm2), x2, x3);
+        const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
+        const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
+        ps01 = fadd2(ps01, p01);
+        ps23 = fadd2(ps23, p23);
+        float t0, t1, t2, t3;
+        f2_unpack(ffma2(p01, k127, magic), t0, t1);
+        f2_unpack(ffma2(p23, k127, magic), t2, t3);
+        pk[q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
+                     prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
+    }
+}
+
 // ---------------------------------------------------------------- kernel ---
 
 // kQ16: Q arrives as fp16 (Qh) and is quantised per token inside the kernel
-// by roles 18-19 (bit-identical to quant_per_token_kernel); its scales go to
-// the prep warps through shared memory and, if sQ_out is set, to global.
+// by roles 14-15 (bit-identical to quant_per_token_kernel); its scales go to
+// the softmax warps through shared memory and, if sQ_out is set, to global.
 // Otherwise Q_hat arrives through tmQ and s_Q through sQ.
 template <int D, bool kQ16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -357,12 +370,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int NS = AttnSmem<D, kQ16>::NS;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
-    // Role numbering: the producer / MMA warpgroup (roles 16-19) runs on the
+    // Role numbering: the producer / MMA warpgroup (roles 12-15) runs on the
     // lowest hardware warps 0-3, which the warp schedulers favour, so that the
     // issue of tensor-core work is not queued behind the compute warps.  A
-    // role keeps its hardware warp's TMEM lane quadrant (role = warp - 4 mod 4).
+    // role keeps its hardware warp's TMEM lane quadrant (role mod 4).
     const int hw_warp = tid >> 5;
-    const int warp = hw_warp < 4 ? hw_warp + 16 : hw_warp - 4;
+    const int warp = hw_warp < 4 ? hw_warp + 12 : hw_warp - 4;
     const int rtid = 32 * warp + lane;
 
     const int ntiles = (L + BM - 1) / BM;
@@ -383,9 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < SB; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.p_full[b], 2 * BM);
-            for (int k = 0; k < 4; ++k) mbar_init(&sm.x_full[b][k], 32);
+            mbar_init(&sm.p_full[b], BM);
         }
+        for (int w = 0; w < 2; ++w)
+            for (int k = 0; k < 4; ++k) mbar_init(&sm.m_full[w][k], 32);
         for (int b = 0; b < AB; ++b)
             for (int k = 0; k < 4; ++k) {
                 mbar_init(&sm.a_full[b][k], 32);
@@ -417,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tbase;              // S buffer s at column 128 s
     const uint32_t tO = tbase + 128 * SB;   // int32 P V block o at column tO + 128 o
 
-    if (warp >= 16) {
+    if (warp >= 12) {
       regs_to<RegSplit<D, kQ16>::kOther>();
       if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer ---
@@ -543,8 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
                 mma_f16_ss(tO, bias_a, bias_b, idesc_bias_o, 0);
 #pragma unroll
-                for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k ..: see the exp warps
-                    mma_i8_ts(tO, tS + sb * BN + 64 * (k >> 1) + 8 * (k & 1), vdesc + 2 * k, idesc_pv, 1);
+                for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k .. 32k + 31 at column 32k
+                    mma_i8_ts(tO, tS + sb * BN + 32 * k, vdesc + 2 * k, idesc_pv, 1);
                 mma_commit(&sm.o_full[0]);
                 mma_commit(&sm.kv_empty[st]);
             }
@@ -563,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       else if (kQ16) {
-        // ------------------------------------------ Q quantiser (18, 19) ---
+        // ------------------------------------------ Q quantiser (14, 15) ---
         // G lanes per row of D fp16 (8 per lane); the two warps take row
         // slices alternately.  Codes go straight into the swizzled K-major
         // layout the TMA would have produced (128-byte swizzle for D = 128:
@@ -571,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // chunk k at k ^ ((r / 2) mod 4)).
         constexpr int G = D / 8;
         constexpr int kRowsPerWarp = 32 / G;
-        const int wq = warp - 18, sub = lane % G;
+        const int wq = warp - kQuantWarp, sub = lane % G;
         bool ok = true;
         for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
             const Tile T = tile_at(t, ntiles, L, causal);
@@ -581,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t qbase = smem_u32(sm.q[qb]);
             const uint4 *stage = reinterpret_cast<const uint4 *>(sm.qs);
             // the tile's fp16 rows in two halves of kQHalf rows through the
-            // staging buffer: warp 18 issues the TMA once both warps have
+            // staging buffer: warp 14 issues the TMA once both warps have
             // read the previous half
             for (int h = 0; ok && h < 2; ++h) {
                 const int n = 2 * i + h;
@@ -625,85 +639,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // otherwise the other two warps of this warpgroup have no role
     } else if (warp < 8) {
-        regs_to<RegSplit<D, kQ16>::kExp>();
-        // ------------------------------------------------------- exp ---
-        // Two warps per TMEM lane quadrant: half hf takes keys 64 hf .. 64 hf
-        // + 63 of each block (chunks 2 hf, 2 hf + 1) and writes their 16 code
-        // words into columns 64 hf .. 64 hf + 15, which only it reads.
-        const int hf = warp >> 2, quad = warp & 3;
+        regs_to<RegSplit<D, kQ16>::kSoft>();
+        // --------------------------------------------------- softmax ---
+        // Warpgroup ws takes the blocks g = ws, ws + 2, ... of this CTA's
+        // stream of (tile, key block) pairs; its warp quad holds TMEM lane
+        // quadrant quad (query rows 32 quad .. 32 quad + 31).
+        const int ws = warp >> 2, quad = warp & 3;
         const int row = 32 * quad + lane;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         const uint64_t k127 = f2_pack(127.0f, 127.0f), magic = f2_pack(kMagic, kMagic);
-        bool pre_x = false;   // probe of the next block's x_full, taken one block early
-        bool ok = true;
-        Ring<SB> sb;
-        for (int i = 0, t = blockIdx.x; ok && t < total; ++i, t += gridDim.x) {
-            const Tile T = tile_at(t, ntiles, L, causal);
-            float l = 0.0f;
-            for (int j = 0; j < T.nb; ++j, sb.next()) {
-                const int b = sb.idx;
-                if (!settle(pre_x, &sm.x_full[b][quad], sb.ph, abort_flag, 7)) { ok = false; break; }
-                tc_fence_after();
-                const Ring<SB> nx = sb.after();
-                pre_x = mbar_test_wait(&sm.x_full[nx.idx][quad], nx.ph);
-                // (c m, alpha, c) from the prep warp: c = s_Q[i] log2(e) / sqrt(d)
-                const float4 ca = sm.cm_alpha[b][row];
-                const uint64_t ncm2 = f2_pack(-ca.x, -ca.x), c2 = f2_pack(ca.z, ca.z);
-                const uint32_t tv = tS + lane_off + b * BN + 64 * hf;
-                uint64_t ps01 = 0ull, ps23 = 0ull;
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    uint32_t w[32];
-                    tmem_ld32(tv + 32 * e, w);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        // x = c v - c m (<= 0; -inf for masked keys), p = 2^x
-                        float x0, x1, x2, x3;
-                        f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q]), __uint_as_float(w[4 * q + 1])), c2, ncm2),
-                                  x0, x1);
-                        f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2,
-                                        ncm2),
-                                  x2, x3);
-                        const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
-                        const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
-                        ps01 = fadd2(ps01, p01);
-                        ps23 = fadd2(ps23, p23);
-                        // P code = RNE(127 p) in the low byte of fl(127 p + 1.5 * 2^23)
-                        float t0, t1, t2, t3;
-                        f2_unpack(ffma2(p01, k127, magic), t0, t1);
-                        f2_unpack(ffma2(p23, k127, magic), t2, t3);
-                        pk[8 * e + q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
-                                             prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
-                    }
-                }
-                // both chunks are in registers: their columns now take the codes
-                tmem_st8(tv, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
-                tmem_st8(tv + 8, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
-                float ps0, ps1, ps2, ps3;
-                f2_unpack(ps01, ps0, ps1);
-                f2_unpack(ps23, ps2, ps3);
-                l = l * ca.y + ((ps0 + ps1) + (ps2 + ps3));
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&sm.p_full[b]);
-            }
-            if (!ok) break;
-            // this tile's half-row sum -> the output side (slot = tile mod 2)
-            const int ls = i & 1;
-            if (i >= 2 && !warp_wait(&sm.l_empty[ls], ((i >> 1) - 1) & 1, abort_flag, 17)) break;
-            sm.lsum[ls][hf][row] = l;
-            mbar_arrive(&sm.l_full[ls]);
-        }
-    } else if (warp < 12) {
-        regs_to<RegSplit<D, kQ16>::kPrep>();
-        // ------------------------------------------------------ prep ---
-        const int row = rtid - 256;
-        const int quad = warp - 8;
-        const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        // probes of the next block's s_full / k_full, taken one block early
-        bool pre_s = false, pre_k = false;
         bool ok = true;
         int g = 0;
         Ring<SB> sb;
@@ -726,59 +670,109 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Clamped to a tiny positive value: a zero Q row then still maps masked
             // keys (v = -inf) to p = 0 and visible keys to p = 1.
             const float c = fmaxf(s_q * (kLog2e / sqrtf(static_cast<float>(D))), 1e-30f);
+            const uint64_t c2 = f2_pack(c, c);
             const int lim = causal ? min(L, qi + 1) : L;
-            float m_old = -INFINITY;
+            float l = 0.0f;              // this warpgroup's share of the row sum, relative to m_own
+            float m_own = -INFINITY;     // running max after this warpgroup's latest block of the tile
             for (int j = 0; j < T.nb; ++j, ++g, sb.next(), ks.next(), as.next()) {
-                // -- block j: v = fl(S s_K) (int32 -> fp32 exact, |S| <= 127^2 d
-                // < 2^24), mask, row max.
-                const int b = sb.idx, ab = as.idx, st = ks.idx;
-                if (!settle(pre_s, &sm.s_full[b], sb.ph, abort_flag, 12)) { ok = false; break; }
+                if ((g & 1) != ws) continue;
+                const int b = sb.idx, st = ks.idx, ab = as.idx;
+                if (!warp_wait(&sm.s_full[b], sb.ph, abort_flag, 12)) { ok = false; break; }
                 // s_K of this block: published by the producer's release-arrive
-                if (!settle(pre_k, &sm.k_full[st], ks.ph, abort_flag, 13)) { ok = false; break; }
+                if (!warp_wait(&sm.k_full[st], ks.ph, abort_flag, 13)) { ok = false; break; }
                 tc_fence_after();
-                const bool pre_a = g < AB || mbar_test_wait(&sm.a_empty[ab][quad], as.ph ^ 1u);
-                const Ring<SB> nsb = sb.after();
-                const Ring<NS> nks = ks.after();
-                pre_s = mbar_test_wait(&sm.s_full[nsb.idx], nsb.ph);
-                pre_k = mbar_test_wait(&sm.k_full[nks.idx], nks.ph);
                 const uint32_t ts = tS + lane_off + b * BN;
                 const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
                 const bool need_mask = (causal && j == T.nb - 1) || ((j + 1) * BN > L);
+                // -- pass 1: v = fl(S s_K) (written back over S), mask, row max;
+                // two 32-column chunks in flight per load
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-                for (int ch = 0; ch < BN / 32; ++ch) {
-                    uint32_t w[32];
-                    tmem_ld32(ts + 32 * ch, w);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t w0[32], w1[32];
+                    tmem_ld32(ts + 64 * h, w0);
+                    tmem_ld32(ts + 64 * h + 32, w1);
                     tmem_wait_ld();
-                    scores_to_v(w, sk4 + 8 * ch);
+                    scores_to_v(w0, sk4 + 16 * h);
+                    scores_to_v(w1, sk4 + 16 * h + 8);
                     // keys past the end of the sequence, or after the query
                     // (causal), get v = -inf (p = 0)
-                    if (need_mask) mask_v(w, j * BN + 32 * ch, lim);
-                    max_v(w, mx);
-                    tmem_st32(ts + 32 * ch, w);
+                    if (need_mask) {
+                        mask_v(w0, j * BN + 64 * h, lim);
+                        mask_v(w1, j * BN + 64 * h + 32, lim);
+                    }
+                    max_v(w0, mx);
+                    max_v(w1, mx);
+                    tmem_st32(ts + 64 * h, w0);
+                    tmem_st32(ts + 64 * h + 32, w1);
                 }
                 mbar_arrive(&sm.kv_empty[st]);   // done with this block's s_K
-                const float m_new = fmaxf(m_old, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
-                const float alpha = ex2(c * (m_old - m_new));   // 0 for the first block
-                m_old = m_new;
-                sm.cm_alpha[b][row] = make_float4(c * m_new, alpha, c, 0.0f);
-                // alpha of block j -> the output warp of this quadrant
-                if (!settle(pre_a, &sm.a_empty[ab][quad], as.ph ^ 1u, abort_flag, 14)) {
+                // running max through block g - 1 (the other warpgroup's); the
+                // wait also orders this warpgroup's mrow write after the other's
+                // read of the previous value
+                float m_prev = -INFINITY;
+                if (g > 0) {
+                    if (!warp_wait(&sm.m_full[ws ^ 1][quad], ((g - 1) >> 1) & 1, abort_flag, 15)) {
+                        ok = false;
+                        break;
+                    }
+                    if (j > 0) m_prev = sm.mrow[ws ^ 1][row];
+                }
+                const float m_new = fmaxf(m_prev, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
+                sm.mrow[ws][row] = m_new;
+                mbar_arrive(&sm.m_full[ws][quad]);
+                const float alpha = ex2(c * (m_prev - m_new));    // 0 for the tile's first block
+                const float lscale = ex2(c * (m_own - m_new));    // 0 for this warpgroup's first
+                m_own = m_new;
+                // alpha of block g -> the output warp of this quadrant (slot
+                // g mod AB was last used by block g - AB, also this warpgroup's)
+                if (g >= AB && !warp_wait(&sm.a_empty[ab][quad], as.ph ^ 1u, abort_flag, 14)) {
                     ok = false;
                     break;
                 }
                 sm.alpha_o[ab][row] = alpha;
                 mbar_arrive(&sm.a_full[ab][quad]);
+                tmem_wait_st();   // v is in TMEM before pass 2 reads it back
+                // -- pass 2: p = 2^(c v - c m), row sum, P codes; the codes of
+                // keys 32 k .. 32 k + 31 go to columns 32 k .. 32 k + 7 (already
+                // read), the A operand of the k-th P V step
+                const float cm = c * m_new;
+                const uint64_t ncm2 = f2_pack(-cm, -cm);
+                uint64_t ps01 = 0ull, ps23 = 0ull;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t w0[32], w1[32];
+                    tmem_ld32(ts + 64 * h, w0);
+                    tmem_ld32(ts + 64 * h + 32, w1);
+                    tmem_wait_ld();
+                    uint32_t pk0[8], pk1[8];
+                    exp_codes(w0, c2, ncm2, k127, magic, ps01, ps23, pk0);
+                    exp_codes(w1, c2, ncm2, k127, magic, ps01, ps23, pk1);
+                    tmem_st8(ts + 64 * h, pk0);
+                    tmem_st8(ts + 64 * h + 32, pk1);
+                }
+                float ps0, ps1, ps2, ps3;
+                f2_unpack(ps01, ps0, ps1);
+                f2_unpack(ps23, ps2, ps3);
+                l = l * lscale + ((ps0 + ps1) + (ps2 + ps3));
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&sm.x_full[b][quad]);
+                mbar_arrive(&sm.p_full[b]);
             }
+            if (!ok) break;
+            // this tile's share of the row sum -> the output side (slot = tile
+            // mod 2); c m_own is -inf if this warpgroup had no block of the tile
+            const int ls = i & 1;
+            if (i >= 2 && !warp_wait(&sm.l_empty[ls], ((i >> 1) - 1) & 1, abort_flag, 17)) break;
+            sm.lsum[ls][ws][row] = l;
+            sm.cml[ls][ws][row] = c * m_own;
+            mbar_arrive(&sm.l_full[ls]);
         }
     } else {
         regs_to<RegSplit<D, kQ16>::kOutput>();
         // ------------------------------------------------ output side ---
-        const int row = rtid - 384;
-        const int quad = warp - 12;
+        const int row = rtid - 256;
+        const int quad = warp - 8;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
         bool ok = true;
         Ring<AB> as;
@@ -830,10 +824,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) break;
-            // the tile's row sums (both key halves) -> normalised fp16 row
+            // the tile's row sum from the two softmax warpgroups' shares, each
+            // rescaled from its own reference c m_w to the final one (the
+            // larger: the running max only grows) -> normalised fp16 row
             const int ls = i & 1;
             if (!warp_wait(&sm.l_full[ls], (i >> 1) & 1, abort_flag, 11)) break;
-            const float l = sm.lsum[ls][0][row] + sm.lsum[ls][1][row];
+            const float cm0 = sm.cml[ls][0][row], cm1 = sm.cml[ls][1][row];
+            const float cmf = fmaxf(cm0, cm1);
+            const float l = sm.lsum[ls][0][row] * ex2(cm0 - cmf) + sm.lsum[ls][1][row] * ex2(cm1 - cmf);
             mbar_arrive(&sm.l_empty[ls]);
             if (qi < L) {
                 const float f = s_v / (127.0f * l);
