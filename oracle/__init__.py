@@ -21,6 +21,10 @@ and marshals numpy arrays.  Each function cites the passage it follows:
   codes against the running max of the key blocks seen so far.  This is the
   form the fused kernel computes.
 * ``attention_fp64_rows`` -- IntAttention section 2.1, eq. 1.
+* ``index_lut``, ``index_cint``, ``index_attention_rows`` -- IntAttention
+  sections 3.1-3.2 (IndexSoftmax: eqs. 7-10, the UINT8 exponential table,
+  UINT8 P times 255, integer row sums) with per-tensor Q / K scales
+  (section 3.3's default configuration).
 
 All functions are pinned by ``tests/test_oracle_*.py`` (closed forms,
 invariants, brute force on tiny inputs).
@@ -66,6 +70,13 @@ def _load():
     lib.oracle_attention_online_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
                                                  ctypes.c_int, I64, I64, I64, P, P]
     lib.oracle_attention_fp64_rows.argtypes = [P, P, P, I64, I64, ctypes.c_int, I64, I64, P]
+    lib.oracle_index_lut.argtypes = [ctypes.c_double, ctypes.c_int, P]
+    lib.oracle_index_cint.argtypes = [ctypes.c_double, I64, ctypes.c_float, ctypes.c_float]
+    lib.oracle_index_cint.restype = I64
+    lib.oracle_index_attention_rows.argtypes = [P, P, P, ctypes.c_float, ctypes.c_float,
+                                                ctypes.c_float, I64, I64, ctypes.c_int,
+                                                ctypes.c_double, ctypes.c_int, I64, I64,
+                                                P, P, P, P]
     _lib = lib
     return lib
 
@@ -205,3 +216,68 @@ def attention_fp64(Q, K, V, causal: bool):
     for h in range(BH):
         O[h] = attention_fp64_rows(Q[h], K[h], V[h], causal)
     return O
+
+
+# ---------------------------------------------------------------- IndexSoftmax
+
+INDEX_C = 6.6   # IntAttention ablation (Fig. 9): the recommended (b, c) = (5, 6.6)
+INDEX_B = 5
+
+
+def index_lut(c: float = INDEX_C, b: int = INDEX_B):
+    """The 2^b-entry UINT8 exponential table: RNE(255 exp(-c k / (2^b - 1)))."""
+    if not 1 <= b <= 8:
+        raise ValueError("b in 1..8")
+    lut = np.empty((1 << b,), np.uint8)
+    _load().oracle_index_lut(float(c), int(b), _ptr(lut))
+    return lut
+
+
+def index_cint(c: float, d: int, sQ: float, sK: float) -> int:
+    """c_int = rint(c sqrt(d) / (s_Q s_K)) in fp64, at least 1 (eq. 8)."""
+    return int(_load().oracle_index_cint(float(c), int(d), float(sQ), float(sK)))
+
+
+def index_attention_rows(Qq, Kq, Vq, sQ: float, sK: float, sV: float, causal: bool,
+                         c: float = INDEX_C, b: int = INDEX_B, r0: int = 0, r1=None,
+                         want_stats: bool = False, want_E: bool = False):
+    """One head of IndexSoftmax attention: Qq/Kq/Vq int8 [L, d] with per-tensor
+    scales.  Returns O fp64 [r1 - r0, d]; with want_stats also the integer row
+    max of Q_hat K_hat^T and the integer row sum of E (int64); with want_E the
+    UINT8 table values E [r1 - r0, L] (0 for masked keys)."""
+    if not 1 <= b <= 8:
+        raise ValueError("b in 1..8")
+    Qq = _c(Qq, np.int8)
+    Kq = _c(Kq, np.int8)
+    Vq = _c(Vq, np.int8)
+    L, d = Qq.shape
+    r1 = L if r1 is None else r1
+    n = r1 - r0
+    O = np.empty((n, d), np.float64)
+    m = np.empty((n,), np.int64) if want_stats else None
+    l = np.empty((n,), np.int64) if want_stats else None
+    E = np.empty((n, L), np.int32) if want_E else None
+    _load().oracle_index_attention_rows(_ptr(Qq), _ptr(Kq), _ptr(Vq), float(sQ), float(sK),
+                                        float(sV), L, d, int(bool(causal)), float(c), int(b),
+                                        r0, r1, _ptr(O), _ptr(m), _ptr(l), _ptr(E))
+    out = [O]
+    if want_stats:
+        out += [m, l]
+    if want_E:
+        out.append(E)
+    return out[0] if len(out) == 1 else tuple(out)
+
+
+def index_attention_fwd(Qq, Kq, Vq, sQ, sK, sV, causal: bool, c: float = INDEX_C,
+                        b: int = INDEX_B, want_stats: bool = False):
+    """All heads: int8 [BH, L, d] (V_hat row-major), per-head scales fp32
+    [BH] for Q, K and V.  Returns O fp64 [BH, L, d] (and int64 m, l [BH, L]
+    with want_stats)."""
+    BH, L, d = Qq.shape
+    O = np.empty((BH, L, d), np.float64)
+    M = np.empty((BH, L), np.int64)
+    Ls = np.empty((BH, L), np.int64)
+    for h in range(BH):
+        O[h], M[h], Ls[h] = index_attention_rows(Qq[h], Kq[h], Vq[h], float(sQ[h]), float(sK[h]),
+                                                 float(sV[h]), causal, c, b, want_stats=True)
+    return (O, M, Ls) if want_stats else O

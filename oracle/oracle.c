@@ -29,6 +29,10 @@
  *                   running max), see oracle_attention_online_rows.
  *   reference       IntAttention section 2.1, eq. 1: O = softmax(Q K^T /
  *                   sqrt(d)) V in fp64 from the unquantised inputs.
+ *   IndexSoftmax    IntAttention sections 3.1-3.2: integer clipping of the
+ *                   row-max distance, a 2^b-entry UINT8 exponential table,
+ *                   UINT8 P (times 255), integer row sums; see
+ *                   oracle_index_attention_rows.
  *
  * Causal masking keeps keys j <= i (square, top-left aligned).
  *
@@ -289,5 +293,107 @@ void oracle_attention_fp64_rows(const float *Q, const float *K, const float *V,
             for (int64_t c = 0; c < d; ++c) o[c] += a[j] * (double)V[j * d + c];
         for (int64_t c = 0; c < d; ++c) o[c] /= l;
         free(a);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* IndexSoftmax attention (IntAttention sections 3.1-3.2)               */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The exponential lookup table of IndexSoftmax (IntAttention section 3.1,
+ * "LUT-based alternative", and section 3.2, "the float table is mapped
+ * linearly onto an integer table"): 2^b UINT8 entries, entry k standing for
+ * the clipped distance k c / (2^b - 1) (the index map of eq. 10 read
+ * backwards), scaled by 255 (section 3.2: UINT8 probabilities times 255):
+ *   LUT[k] = RNE(255 exp(-c k / (2^b - 1))),   k = 0 .. 2^b - 1.
+ */
+void oracle_index_lut(double c, int b, uint8_t *lut) {
+    const int64_t n = (int64_t)1 << b;
+    for (int64_t k = 0; k < n; ++k) {
+        const double x = c * (double)k / (double)(n - 1);
+        lut[k] = (uint8_t)nearbyint(255.0 * exp(-x));
+    }
+}
+
+/*
+ * The quantisation-aligned clipping threshold (IntAttention section 3.1,
+ * eq. 8): c_int = round(c / alpha) with alpha = s_Q s_K / sqrt(d), the
+ * per-tensor scales of the default configuration (section 3.3).  Evaluated
+ * in fp64 as rint((c sqrt(d)) / (s_Q s_K)); at least 1 (a zero scale means
+ * all logits are 0 and every distance is 0, so any positive threshold gives
+ * the same result).
+ */
+int64_t oracle_index_cint(double c, int64_t d, float sQ, float sK) {
+    const double den = (double)sQ * (double)sK;
+    if (!(den > 0.0)) return 1;
+    const double v = nearbyint((c * sqrt((double)d)) / den);
+    if (v < 1.0) return 1;
+    if (v > 4.0e18) return (int64_t)4e18;
+    return (int64_t)v;
+}
+
+/*
+ * IndexSoftmax attention for rows [r0, r1) of one head (IntAttention
+ * section 3.1 eqs. 7-10, section 3.2), with the value path of eq. 5:
+ *   A_hat    = Q_hat K_hat^T                       (INT32, eq. 4)
+ *   Delta    = rowmax(A_hat) - A_hat               (eq. 7; over visible keys)
+ *   Delta'   = min(Delta, c_int)                   (eq. 9)
+ *   idx      = floor(Delta' (2^b - 1) / c_int)     (eq. 10, exact integers)
+ *   E        = LUT[idx]                            (UINT8, ~ 255 exp(-alpha Delta'))
+ *   O_i      = s_V sum_j E_ij V_hat_j / sum_j E_ij
+ * Qq, Kq, Vq: int8 [L][d]; sQ, sK, sV: the head's per-tensor scales.
+ * The normalisation by the integer row sum is applied after the P V
+ * product (the same quotient as normalising P first, without rounding the
+ * normalised probabilities to 8 bits).  Masked keys (causal, j > i) get
+ * E = 0.  Optional outputs (may be NULL): m_out / l_out [r1 - r0] (the
+ * integer row max of A_hat and the integer row sum of E), E_out
+ * [(r1 - r0) * L] (E, 0 for masked keys).
+ */
+void oracle_index_attention_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
+                                 float sQ, float sK, float sV, int64_t L, int64_t d,
+                                 int causal, double c, int b, int64_t r0, int64_t r1,
+                                 double *O, int64_t *m_out, int64_t *l_out, int32_t *E_out) {
+    uint8_t lut[256];
+    oracle_index_lut(c, b, lut);
+    const int64_t nm1 = ((int64_t)1 << b) - 1;
+    const int64_t cint = oracle_index_cint(c, d, sQ, sK);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = r0; i < r1; ++i) {
+        const int64_t n = causal ? (i + 1) : L;
+        int64_t *a = (int64_t *)malloc((size_t)n * sizeof(int64_t));
+        int64_t *acc = (int64_t *)calloc((size_t)d, sizeof(int64_t));
+        int32_t *e = (int32_t *)malloc((size_t)n * sizeof(int32_t));
+        /* eq. 4: integer logits; eq. 7: the row max over visible keys */
+        int64_t m = INT64_MIN;
+        for (int64_t j = 0; j < n; ++j) {
+            a[j] = dot_i8(Qq + i * d, Kq + j * d, d);
+            if (a[j] > m) m = a[j];
+        }
+        /* eqs. 7-10: distance, clip, index, table */
+        int64_t l = 0;
+        for (int64_t j = 0; j < n; ++j) {
+            int64_t delta = m - a[j];
+            if (delta > cint) delta = cint;
+            const int64_t idx = (delta * nm1) / cint;
+            e[j] = lut[idx];
+            l += e[j];
+        }
+        /* eq. 5: integer E V_hat, then the scale and the row-sum normalisation */
+        for (int64_t j = 0; j < n; ++j) {
+            const int8_t *v = Vq + j * d;
+            for (int64_t cc = 0; cc < d; ++cc) acc[cc] += (int64_t)e[j] * (int64_t)v[cc];
+        }
+        double *o = O + (i - r0) * d;
+        for (int64_t cc = 0; cc < d; ++cc) o[cc] = (double)sV * (double)acc[cc] / (double)l;
+        if (m_out) m_out[i - r0] = m;
+        if (l_out) l_out[i - r0] = l;
+        if (E_out) {
+            int32_t *er = E_out + (i - r0) * L;
+            for (int64_t j = 0; j < L; ++j) er[j] = (j < n) ? e[j] : 0;
+        }
+        free(a);
+        free(acc);
+        free(e);
     }
 }
