@@ -160,6 +160,40 @@ int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *
                             int causal, void *O_f16, float *s_Q_out, void *stream);
 
 /*
+ * IndexSoftmax attention (IntAttention: A Fully Integer Attention Pipeline for
+ * Efficient Edge Inference, section 3.1 eqs. 7-10, section 3.2, and eq. 5 for
+ * the value path) with per-tensor scales, section 3.3's default
+ * configuration.  Per head (scales s_Q, s_K, s_V):
+ *   A_hat  = Q_hat K_hat^T (INT8 x INT8 -> INT32); m_i = row max over visible keys
+ *   c_int  = rint((c sqrt(d)) / (s_Q s_K)) in fp64, at least 1   (eq. 8)
+ *   idx_ij = floor(min(m_i - A_hat_ij, c_int) (2^b - 1) / c_int)  (eqs. 9-10)
+ *   E_ij   = LUT[idx_ij], LUT[k] = rint(255 exp(-c k / (2^b - 1))) (UINT8 P x 255)
+ *   O_i    = s_V (sum_j E_ij V_hat_j) / (sum_j E_ij), written as fp16
+ * The row max covers the whole row before any lookup (two passes over the
+ * keys); the integer sums are exact.  The pages normalise the 8-bit
+ * probabilities before P V; here the same quotient is taken after it, which
+ * avoids rounding normalised probabilities below 1/255 to zero on long rows.
+ *
+ *   Q_q, K_q : int8 [B][H][L][d], per-tensor codes (intfa_quantize_per_tensor
+ *              with groups = B*H, transpose = 0), 16-B aligned.
+ *   Vt_q     : int8 [B][H][d][intfa_vt_ld(L)] as for intfa_attention_fwd.
+ *   s_Q, s_K, s_V : fp32 [B][H] (one scale per head each).
+ *   c, b     : clip threshold (0 < c < 1e30) and table bits (1 .. 8); the
+ *              pages recommend (b, c) = (5, 6.6).
+ *   O_f16    : fp16 [B][H][L][d] out, 16-byte aligned.
+ *   m_out, l_out : int32 [B][H][L] out or NULL: the integer row max of A_hat
+ *              and the integer row sum of E (exact, for checking).
+ *   d in {64, 128}; 1 <= L <= 65536 (int32 accumulation: 255 * 127 * L <
+ *   2^31); causal in {0, 1}.  INTFA_ERR_INVALID_ARG / UNSUPPORTED /
+ *   MISALIGNED for bad arguments, INTFA_ERR_CUDA for a failed launch; a
+ *   device-side timeout shows in intfa_device_status.
+ */
+int intfa_index_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                              const float *s_Q, const float *s_K, const float *s_V, int B,
+                              int H, int L, int d, int causal, double c, int b, void *O_f16,
+                              int32_t *m_out, int32_t *l_out, void *stream);
+
+/*
  * Debug: the integer logits S = Q_hat K_hat^T (IntAttention eq. 4) for every
  * head, int32 [B][H][L][L], computed by the same TMA + tcgen05 path the fused
  * kernel uses for its first contraction.  Same layout rules as

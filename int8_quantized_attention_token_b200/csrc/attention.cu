@@ -56,6 +56,7 @@
 #include "internal.h"
 #include "ptx.cuh"
 #include "quant_math.cuh"
+#include "tma_host.h"
 
 namespace intfa {
 
@@ -940,45 +941,6 @@ __global__ void __launch_bounds__(128, 1)
 
 // ----------------------------------------------------------- host side ---
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                             &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-        else
-            (void)cudaGetLastError();
-    }
-    return fn;
-}
-
-// 3-D tensor map (uint8 unless dtype says otherwise): dims (x = inner, y, z) in
-// elements, byte strides of y and z, box (bx, by, 1) in elements.
-int make_map(CUtensorMap *map, const void *base, uint64_t x, uint64_t y, uint64_t z,
-             uint64_t stride_y, uint64_t stride_z, uint32_t bx, uint32_t by,
-             CUtensorMapSwizzle swz, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8) {
-    EncodeTiledFn enc = get_encode_fn();
-    if (!enc) return INTFA_ERR_CUDA;
-    const cuuint64_t dims[3] = {x, y, z};
-    const cuuint64_t strides[2] = {stride_y, stride_z};
-    const cuuint32_t box[3] = {bx, by, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = enc(map, dtype, 3, const_cast<void *>(base), dims,
-                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? INTFA_OK : INTFA_ERR_CUDA;
-}
-
 // Grid of the persistent attention kernel: one CTA per SM.  CTA c takes tiles
 // c, c + G, ...; with causal masking the per-tile work cycles with period
 // ntiles inside each head, so G is chosen coprime to ntiles, which makes every
@@ -1144,7 +1106,7 @@ extern "C" int intfa_device_status(int clear, uint32_t *word) {
     using namespace intfa;
     int rc = cuda_status(cudaDeviceSynchronize());
     if (rc) return rc;
-    uint32_t w = 0;
+    uint32_t w = 0, wi = 0;
     rc = cuda_status(cudaMemcpyFromSymbol(&w, g_status, sizeof(w)));
     if (rc) return rc;
     if (clear) {
@@ -1152,6 +1114,9 @@ extern "C" int intfa_device_status(int clear, uint32_t *word) {
         rc = cuda_status(cudaMemcpyToSymbol(g_status, &z, sizeof(z)));
         if (rc) return rc;
     }
+    rc = read_index_status(clear, &wi);   // the IndexSoftmax kernel's word
+    if (rc) return rc;
+    if (!w) w = wi;
     if (word) *word = w;
     return w ? INTFA_ERR_DEVICE_TIMEOUT : INTFA_OK;
 }

@@ -31,5 +31,7 @@ int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt,
 int launch_attention_fwd_q16(const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sK,
                              const float *sV, int B, int H, int L, int d, int causal, void *O,
                              float *sQ_out, cudaStream_t stream);
+// The IndexSoftmax kernel's status word (index_attention.cu); clear resets it.
+int read_index_status(int clear, uint32_t *word);
 
 }  // namespace intfa

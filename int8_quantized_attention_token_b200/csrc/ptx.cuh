@@ -337,6 +337,15 @@ __host__ __device__ constexpr uint32_t make_idesc_i8(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::i8 with an unsigned A: D = s32, A = unsigned
+// 8-bit, B = signed 8-bit, both K-major, dense, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc_u8s8(int M, int N) {
+    return (2u << 4)                                   // D format: s32
+           | (1u << 10)                                // B: signed 8-bit (A format 0: unsigned)
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
 // Instruction descriptor, kind::f16: D = f32, A = B = f16, both K-major,
 // dense, shape M x N.
 __host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N) {

@@ -51,6 +51,7 @@ def lib():
         "intfa_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
         "intfa_attention_fwd_q16": ([P, P, P, P, P, I, I, I, I, I, P, P, P], I),
         "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
+        "intfa_index_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, ctypes.c_double, I, P, P, P, P], I),
         "intfa_forward_workspace_size": ([I, I, I, I], SZ),
         "intfa_forward_workspace_layout": ([I, I, I, I, ctypes.POINTER(SZ)], I),
         "intfa_forward": ([P, P, P, I, I, I, I, I, P, P, SZ, P], I),
@@ -195,6 +196,30 @@ def intfa_attention_fwd_q16(Q, K_q, Vt_q, s_K, s_V, causal: bool, O=None, s_Q=No
     _check(lib().intfa_attention_fwd_q16(_ptr(Q), _ptr(K_q), _ptr(Vt_q), _ptr(s_K), _ptr(s_V), B, H, L, d,
                                          int(bool(causal)), _ptr(O), _ptr(s_Q) if s_Q is not None else None,
                                          _stream(stream)), "intfa_attention_fwd_q16")
+    return O
+
+
+def intfa_index_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, c: float = 6.6, b: int = 5,
+                              O=None, m_out=None, l_out=None, stream=None):
+    """IndexSoftmax attention.  Q_q, K_q int8 [B, H, L, d] with per-head
+    scales s_Q, s_K fp32 [B, H]; Vt_q int8 [B, H, d, intfa_vt_ld(L)] with s_V
+    fp32 [B, H]; clip threshold c and table bits b  ->  O fp16 [B, H, L, d].
+    m_out / l_out (int32 [B, H, L], optional) receive the integer row max of
+    Q_hat K_hat^T and the integer row sum of the table values."""
+    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
+        _need(t, torch.int8, n)
+    for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
+        _need(t, torch.float32, n)
+    for t, n in ((m_out, "m_out"), (l_out, "l_out")):
+        if t is not None:
+            _need(t, torch.int32, n)
+    B, H, L, d = Q_q.shape
+    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
+    _check(lib().intfa_index_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
+                                           B, H, L, d, int(bool(causal)), float(c), int(b), _ptr(O),
+                                           _ptr(m_out) if m_out is not None else None,
+                                           _ptr(l_out) if l_out is not None else None,
+                                           _stream(stream)), "intfa_index_attention_fwd")
     return O
 
 

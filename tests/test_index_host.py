@@ -1,0 +1,60 @@
+"""Host-side checks of the IndexSoftmax kernel's index arithmetic.
+
+The kernel evaluates idx = floor(D' (2^b - 1) / c_int) (IntAttention section
+3.1, eq. 10) as floor(D' q) with q = (2^b - 1) / c_int rounded up to fp32,
+through one round-down fma, whenever c_int <= 2^(23 - b).  Both maps are
+non-decreasing step functions of the integer D', so they agree everywhere on
+[0, c_int] iff they agree at every step of the exact map (its first D' of
+each new value, and the D' just before it).  These tests check that, with
+exact rational arithmetic, for every b and for c_int up to and at the bound.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+
+def q_round_up(nm1: int, cint: int) -> Fraction:
+    """fp32 (2^b - 1) / c_int rounded toward +infinity, as an exact rational."""
+    exact = Fraction(nm1, cint)
+    q = np.float32(nm1 / cint)
+    if Fraction(float(q)) < exact:
+        q = np.nextafter(q, np.float32(np.inf), dtype=np.float32)
+    assert Fraction(float(q)) >= exact
+    return Fraction(float(q))
+
+
+def fast_index(dl: int, q: Fraction) -> int:
+    # fma.rm(D', q, 2^23) - 2^23 = floor(D' q) while D' q < 2^23
+    return int(dl * q // 1)
+
+
+def check(cint: int, b: int):
+    nm1 = (1 << b) - 1
+    q = q_round_up(nm1, cint)
+    points = {0, cint, cint - 1}
+    for k in range(1, nm1 + 1):
+        first = -(-k * cint // nm1)          # ceil(k c_int / nm1): first D' with idx >= k
+        points.update({first - 1, first, first + 1})
+    for dl in points:
+        if 0 <= dl <= cint:
+            assert fast_index(dl, q) == (dl * nm1) // cint, (cint, b, dl)
+
+
+@pytest.mark.parametrize("b", range(1, 9))
+def test_fast_index_exact_up_to_the_bound(b):
+    bound = 1 << (23 - b)
+    rng = np.random.default_rng(b)
+    cints = list(range(1, 200)) + [bound, bound - 1, bound - 2, bound // 2 + 1]
+    cints += [int(x) for x in rng.integers(200, bound, 300)]
+    for cint in cints:
+        check(cint, b)
+
+
+def test_fast_index_small_cint_exhaustive():
+    for b in (1, 5, 8):
+        nm1 = (1 << b) - 1
+        for cint in range(1, 300):
+            q = q_round_up(nm1, cint)
+            for dl in range(cint + 1):
+                assert fast_index(dl, q) == (dl * nm1) // cint
