@@ -7,6 +7,9 @@ and the fused INT8 attention kernel.  The metric is INT8 attention TOPS:
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...    # the CPU oracle, timed on host cores
+    python bench.py --method index ...      # the IndexSoftmax variant (IntAttention
+                                            # sections 3.1-3.2): per-tensor Q/K/V
+                                            # quantisation + the two-pass LUT kernel
 
 N > 1 runs under torchrun, one rank per GPU, each rank the full workload on
 its own GPU (independent replicas: the path has no exchange step); the time
@@ -35,11 +38,12 @@ I8_PER_BF16 = 2.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
 
-def kernel_sources_sha() -> str:
-    """Hash of the attention kernel's sources (the dominant kernel)."""
+def kernel_sources_sha(method: str = "online") -> str:
+    """Hash of the dominant kernel's sources (the attention kernel of `method`)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_quantized_attention_token_b200", "csrc")
-    for f in ("attention.cu", "ptx.cuh"):
+    files = ("attention.cu", "ptx.cuh", "quant_math.cuh") if method == "online" else ("index_attention.cu", "ptx.cuh")
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -58,15 +62,15 @@ def peaks():
                 "source": "fallback"}
 
 
-def traffic_for(workload: str):
+def traffic_for(workload: str, method: str = "online"):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
     taken on the current kernel sources; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             t = json.load(f)
-        e = t.get(workload)
-        if e and e.get("kernel_sha") == kernel_sources_sha():
+        e = t.get(workload if method == "online" else f"{workload}:{method}")
+        if e and e.get("kernel_sha") == kernel_sources_sha(method):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -177,8 +181,29 @@ def run_gpu(args):
     V3 = V.reshape(BH, L, d)
 
     fused_q = args.q_path == "fused"
+    index = args.method == "index"
+    if index:   # per-tensor Q and K codes and one scale per head
+        sQh = torch.empty(BH, dtype=torch.float32, device=dev)
+        sKh = torch.empty(BH, dtype=torch.float32, device=dev)
+        Q3, K3 = Q.reshape(BH, L, d), K.reshape(BH, L, d)
+        Qq3, Kq3 = Qq.reshape(BH, L, d), Kq.reshape(BH, L, d)
+
+    def step_index(ev=None):
+        # per-tensor quantisation of Q, K and V (transposed), then the
+        # IndexSoftmax kernel (IntAttention sections 3.1-3.2)
+        intfa.intfa_quantize_per_tensor(Q3, False, Qq3, sQh, ws, stream=stream)
+        intfa.intfa_quantize_per_tensor(K3, False, Kq3, sKh, ws, stream=stream)
+        intfa.intfa_quantize_per_tensor(V3, True, Vt, sV, ws, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        intfa.intfa_index_attention_fwd(Qq, Kq, Vt.reshape(B, H, d, ld), sQh.reshape(B, H), sKh.reshape(B, H),
+                                        sV.reshape(B, H), w.causal, args.index_c, args.index_b, O, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
 
     def step(ev=None):
+        if index:
+            return step_index(ev)
         # a1 (K; and Q unless fused), a2 (V), then a3-a9 in the attention kernel
         if not fused_q:
             intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
@@ -195,8 +220,9 @@ def run_gpu(args):
         if ev is not None:
             ev[1].record(stream)
 
-    # quantise K, V abs-max, V convert, attention (+ quantise Q when separate)
-    kernels_per_step = 4 if fused_q else 5
+    # quantise K, V abs-max, V convert, attention (+ quantise Q when separate);
+    # index: abs-max and convert for each of Q, K, V, and the attention kernel
+    kernels_per_step = 7 if index else (4 if fused_q else 5)
 
     for _ in range(args.warmup):
         step()
@@ -239,7 +265,38 @@ def run_gpu(args):
 
     # End to end through the host-buffer entry point: pinned fp16 in, fp16 out.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and index:
+        # the same step with the fp16 inputs copied from pinned host memory
+        # and O copied back, inside the timed region
+        Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
+        Op = torch.empty(B, H, L, d, dtype=torch.float16).pin_memory()
+
+        def e2e_step():
+            Q.copy_(Qp, non_blocking=True)
+            K.copy_(Kp, non_blocking=True)
+            V.copy_(Vp, non_blocking=True)
+            step_index()
+            Op.copy_(O, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e_steps = max(3, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        nbytes = B * H * L * d * 2
+        e2e = {"value": w.ops * world * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "steps": e_steps, "ms_per_step": e_ms / e_steps,
+               "api": "intfa_quantize_per_tensor x3 + intfa_index_attention_fwd with pinned host copies"}
+    elif not args.no_e2e:
         Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
         Op = torch.empty(B, H, L, d, dtype=torch.float16).pin_memory()
         wsh = torch.empty(intfa.intfa_forward_host_workspace_size(B, H, L, d), dtype=torch.uint8, device=dev)
@@ -265,7 +322,8 @@ def run_gpu(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+        cpu = cpu_baseline(w, budget_s=args.cpu_seconds, method=args.method,
+                           c=args.index_c, b=args.index_b)
 
     if rank == 0:
         line = {
@@ -274,22 +332,27 @@ def run_gpu(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
             "data": "synthetic (seeded N(0,1) fp16 Q/K/V)",
             "config": {**w.as_dict(), "parallelism": f"replicas{world}" if world > 1 else "single",
-                       "l2": "inputs larger than L2 (fp16 Q/K/V 3x128 MiB read per step)"},
+                       "l2": "inputs larger than L2 (fp16 Q/K/V 3x128 MiB read per step)",
+                       "method": args.method,
+                       **({"index_c": args.index_c, "index_b": args.index_b} if index else {})},
             "pct_of_int8_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "tensor",
-                         "kernel": "attn_fwd_kernel<128, Q quantised in-kernel>" if fused_q else "attn_fwd_kernel<128>",
+                         "kernel": ("attn_index_kernel<%d>" % d) if index else
+                                   ("attn_fwd_kernel<%d, Q quantised in-kernel>" % d if fused_q else "attn_fwd_kernel<%d>" % d),
                          "achieved": round(achieved, 2),
                          "peak": round(peak, 1), "unit": UNIT, "frac": round(achieved / peak, 4),
-                         "traffic": traffic_for(w.name),
+                         "traffic": traffic_for(w.name, args.method),
                          "peak_note": f"{pk['source']} bf16 burst {pk['bf16_burst']} TFLOP/s x {I8_PER_BF16} "
                                       "(nominal dense INT8:BF16 ratio)",
                          "frac_of_sustained": round(achieved / (pk["bf16_sustained"] * I8_PER_BF16), 4),
-                         "attn_ms": round(attn_mean, 5), "ops_per_launch": w.ops},
+                         "attn_ms": round(attn_mean, 5), "ops_per_launch": w.ops,
+                         **({"ops_note": "the method's two contractions counted once; the kernel "
+                                         "computes Q K^T twice (row-max pass and table pass)"} if index else {})},
             "kernels_ms_per_step": {"attention": round(attn_mean, 5),
                                     "quantisation": round(ms_per_step - attn_mean, 5),
                                     "q_path": args.q_path},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
-            "clocks": clk, "kernel_sha": kernel_sources_sha(),
+            "clocks": clk, "kernel_sha": kernel_sources_sha(args.method),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -299,8 +362,9 @@ def run_gpu(args):
 
 # --------------------------------------------------------------- CPU arm ---
 
-def oracle_sample(w, heads, threads=None):
-    """Run the oracle's whole path (quantise, block-wise online attention) on
+def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5):
+    """Run the oracle's whole path (quantise, block-wise online attention; or
+    for method "index" per-tensor quantisation and IndexSoftmax attention) on
     `heads` full (b, h) heads of the workload; returns (seconds, ops, cores)."""
     import numpy as np
 
@@ -311,27 +375,34 @@ def oracle_sample(w, heads, threads=None):
     oracle.set_threads(cores)
     Q, K, V = make_workload(w)
     t = 0.0
-    for (b, h) in heads:
-        q, k, v = (X[b, h].float().numpy() for X in (Q, K, V))
+    for (bi, h) in heads:
+        q, k, v = (X[bi, h].float().numpy() for X in (Q, K, V))
         t0 = time.perf_counter()
-        Qq, sQ = oracle.quantize_per_token(q)
-        Kq, sK = oracle.quantize_per_token(k)
-        Vq, sV = oracle.quantize_per_tensor(v, 1)
-        oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), w.causal, 128)
+        if method == "index":
+            Qq, sQ = oracle.quantize_per_tensor(q, 1)
+            Kq, sK = oracle.quantize_per_tensor(k, 1)
+            Vq, sV = oracle.quantize_per_tensor(v, 1)
+            oracle.index_attention_rows(Qq, Kq, Vq, float(sQ[0]), float(sK[0]), float(sV[0]), w.causal, c, b)
+        else:
+            Qq, sQ = oracle.quantize_per_token(q)
+            Kq, sK = oracle.quantize_per_token(k)
+            Vq, sV = oracle.quantize_per_tensor(v, 1)
+            oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), w.causal, 128)
         t += time.perf_counter() - t0
     ops = w.ops / (w.B * w.H) * len(heads)
     return t, ops, oracle.get_threads()
 
 
-def cpu_baseline(w, budget_s=15.0):
-    t1, ops1, cores = oracle_sample(w, [(0, 0)])
+def cpu_baseline(w, budget_s=15.0, method="online", c=6.6, b=5):
+    t1, ops1, cores = oracle_sample(w, [(0, 0)], method=method, c=c, b=b)
     n = max(1, min(w.B * w.H - 1, int(budget_s / max(t1, 1e-3)) - 1))
     heads = [((i + 1) // w.H % w.B, (i + 1) % w.H) for i in range(n)]
-    t, ops, cores = oracle_sample(w, heads)
+    t, ops, cores = oracle_sample(w, heads, method=method, c=c, b=b)
     t += t1
     ops += ops1
+    what = "per-tensor quantise + IndexSoftmax attention" if method == "index" else "quantise + online attention"
     return {"value": round(ops / t / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n + 1} of {w.B * w.H} heads at full L={w.L} (quantise + online attention), "
+            "sample": f"{n + 1} of {w.B * w.H} heads at full L={w.L} ({what}), "
                       f"{t:.1f} s on {cores} threads"}
 
 
@@ -406,6 +477,10 @@ def main():
     ap.add_argument("--impl", default="libintfa", choices=["libintfa", "reference"])
     ap.add_argument("--q-path", default="separate", choices=["fused", "separate"],
                     help="quantise Q in its own pass (default, faster) or inside the attention kernel")
+    ap.add_argument("--method", default="online", choices=["online", "index"],
+                    help="online: the INT8 FlashAttention path (default); index: the IndexSoftmax variant")
+    ap.add_argument("--index-c", type=float, default=6.6, help="IndexSoftmax clip threshold c")
+    ap.add_argument("--index-b", type=int, default=5, help="IndexSoftmax table bits b")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
