@@ -87,6 +87,23 @@ def test_attention_rejects(L):
     assert L.intfa_debug_qk(FAKE, None, 1, 1, 128, 64, FAKE, None) == 1
 
 
+def test_index_attention_rejects(L):
+    # Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, c, b, O, m_out, l_out, stream
+    a = [FAKE] * 6
+    f = L.intfa_index_attention_fwd
+    assert f(*a, 1, 1, 128, 96, 0, 6.6, 5, FAKE, None, None, None) == 2              # d
+    assert f(*a, 1, 1, 65537, 64, 0, 6.6, 5, FAKE, None, None, None) == 2            # int32 bound
+    assert f(*a, 0, 1, 128, 64, 0, 6.6, 5, FAKE, None, None, None) == 1              # B
+    assert f(*a, 1, 1, 128, 64, 2, 6.6, 5, FAKE, None, None, None) == 1              # causal flag
+    assert f(*a, 1, 1, 128, 64, 0, 0.0, 5, FAKE, None, None, None) == 1              # c
+    assert f(*a, 1, 1, 128, 64, 0, float("nan"), 5, FAKE, None, None, None) == 1
+    assert f(*a, 1, 1, 128, 64, 0, 6.6, 0, FAKE, None, None, None) == 1              # b
+    assert f(*a, 1, 1, 128, 64, 0, 6.6, 9, FAKE, None, None, None) == 1
+    assert f(*a, 1, 1, 128, 64, 0, 6.6, 5, None, None, None, None) == 1              # O
+    assert f(FAKE + 8, *a[1:], 1, 1, 128, 64, 0, 6.6, 5, FAKE, None, None, None) == 3
+    assert f(*a, 1, 1, 128, 64, 0, 6.6, 5, FAKE, FAKE + 2, None, None) == 3          # m_out
+
+
 def test_forward_rejects(L):
     assert L.intfa_forward(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, None, 0, None) == 6
     ws = intfa.intfa_forward_workspace_size(1, 1, 128, 64)
