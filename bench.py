@@ -201,9 +201,34 @@ def run_gpu(args):
         if ev is not None:
             ev[1].record(stream)
 
+    blk = args.scale_block
+    if blk > 1:   # one Q / K scale per block of blk tokens (group-wise quantisation)
+        if L % blk:
+            raise SystemExit("--scale-block must divide L")
+        sQb = torch.empty(BH * L // blk, dtype=torch.float32, device=dev)
+        sKb = torch.empty_like(sQb)
+        Qg, Kg = Q.reshape(BH * L // blk, blk, d), K.reshape(BH * L // blk, blk, d)
+        Qqg, Kqg = Qq.reshape(BH * L // blk, blk, d), Kq.reshape(BH * L // blk, blk, d)
+        wsb = torch.empty(max(1, intfa.lib().intfa_quantize_per_tensor_workspace_size(BH * L // blk)),
+                          dtype=torch.uint8, device=dev)
+
+    def step_blocks(ev=None):
+        intfa.intfa_quantize_per_tensor(Qg, False, Qqg, sQb, wsb, stream=stream)
+        intfa.intfa_quantize_per_tensor(Kg, False, Kqg, sKb, wsb, stream=stream)
+        intfa.intfa_quantize_per_tensor(V3, True, Vt, sV, ws, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        intfa.intfa_attention_fwd_blockscale(Qq, Kq, Vt.reshape(B, H, d, ld), sQb.reshape(B, H, -1),
+                                             sKb.reshape(B, H, -1), sV.reshape(B, H), w.causal, blk, O,
+                                             stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
     def step(ev=None):
         if index:
             return step_index(ev)
+        if blk > 1:
+            return step_blocks(ev)
         # a1 (K; and Q unless fused), a2 (V), then a3-a9 in the attention kernel
         if not fused_q:
             intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
@@ -222,7 +247,7 @@ def run_gpu(args):
 
     # quantise K, V abs-max, V convert, attention (+ quantise Q when separate);
     # index: abs-max and convert for each of Q, K, V, and the attention kernel
-    kernels_per_step = 7 if index else (4 if fused_q else 5)
+    kernels_per_step = 7 if (index or blk > 1) else (4 if fused_q else 5)
 
     for _ in range(args.warmup):
         step()
@@ -265,7 +290,7 @@ def run_gpu(args):
 
     # End to end through the host-buffer entry point: pinned fp16 in, fp16 out.
     e2e = None
-    if not args.no_e2e and index:
+    if not args.no_e2e and (index or blk > 1):
         # the same step with the fp16 inputs copied from pinned host memory
         # and O copied back, inside the timed region
         Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
@@ -275,7 +300,7 @@ def run_gpu(args):
             Q.copy_(Qp, non_blocking=True)
             K.copy_(Kp, non_blocking=True)
             V.copy_(Vp, non_blocking=True)
-            step_index()
+            step()
             Op.copy_(O, non_blocking=True)
 
         for _ in range(2):
@@ -295,7 +320,8 @@ def run_gpu(args):
         e2e = {"value": w.ops * world * e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
                "steps": e_steps, "ms_per_step": e_ms / e_steps,
-               "api": "intfa_quantize_per_tensor x3 + intfa_index_attention_fwd with pinned host copies"}
+               "api": ("intfa_quantize_per_tensor x3 + intfa_index_attention_fwd" if index else
+                       "intfa_quantize_per_tensor x3 + intfa_attention_fwd_blockscale") + " with pinned host copies"}
     elif not args.no_e2e:
         Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
         Op = torch.empty(B, H, L, d, dtype=torch.float16).pin_memory()
@@ -323,7 +349,7 @@ def run_gpu(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=args.cpu_seconds, method=args.method,
-                           c=args.index_c, b=args.index_b)
+                           c=args.index_c, b=args.index_b, blk=blk)
 
     if rank == 0:
         line = {
@@ -334,6 +360,7 @@ def run_gpu(args):
             "config": {**w.as_dict(), "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (fp16 Q/K/V 3x128 MiB read per step)",
                        "method": args.method,
+                       **({"scale_block": blk} if blk > 1 else {}),
                        **({"index_c": args.index_c, "index_b": args.index_b} if index else {})},
             "pct_of_int8_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "tensor",
@@ -362,7 +389,7 @@ def run_gpu(args):
 
 # --------------------------------------------------------------- CPU arm ---
 
-def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5):
+def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5, blk=1):
     """Run the oracle's whole path (quantise, block-wise online attention; or
     for method "index" per-tensor quantisation and IndexSoftmax attention) on
     `heads` full (b, h) heads of the workload; returns (seconds, ops, cores)."""
@@ -383,6 +410,13 @@ def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5):
             Kq, sK = oracle.quantize_per_tensor(k, 1)
             Vq, sV = oracle.quantize_per_tensor(v, 1)
             oracle.index_attention_rows(Qq, Kq, Vq, float(sQ[0]), float(sK[0]), float(sV[0]), w.causal, c, b)
+        elif blk > 1:   # one scale per block of blk tokens
+            n = w.L // blk
+            Qq, sQ = oracle.quantize_per_tensor(q.reshape(n, blk * w.d), n)
+            Kq, sK = oracle.quantize_per_tensor(k.reshape(n, blk * w.d), n)
+            Vq, sV = oracle.quantize_per_tensor(v, 1)
+            oracle.attention_online_rows(Qq.reshape(w.L, w.d), Kq.reshape(w.L, w.d), Vq, np.repeat(sQ, blk),
+                                         np.repeat(sK, blk), float(sV[0]), w.causal, 128)
         else:
             Qq, sQ = oracle.quantize_per_token(q)
             Kq, sK = oracle.quantize_per_token(k)
@@ -393,14 +427,15 @@ def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5):
     return t, ops, oracle.get_threads()
 
 
-def cpu_baseline(w, budget_s=15.0, method="online", c=6.6, b=5):
-    t1, ops1, cores = oracle_sample(w, [(0, 0)], method=method, c=c, b=b)
+def cpu_baseline(w, budget_s=15.0, method="online", c=6.6, b=5, blk=1):
+    t1, ops1, cores = oracle_sample(w, [(0, 0)], method=method, c=c, b=b, blk=blk)
     n = max(1, min(w.B * w.H - 1, int(budget_s / max(t1, 1e-3)) - 1))
     heads = [((i + 1) // w.H % w.B, (i + 1) % w.H) for i in range(n)]
-    t, ops, cores = oracle_sample(w, heads, method=method, c=c, b=b)
+    t, ops, cores = oracle_sample(w, heads, method=method, c=c, b=b, blk=blk)
     t += t1
     ops += ops1
-    what = "per-tensor quantise + IndexSoftmax attention" if method == "index" else "quantise + online attention"
+    what = ("per-tensor quantise + IndexSoftmax attention" if method == "index" else
+            f"per-{blk}-token-block quantise + online attention" if blk > 1 else "quantise + online attention")
     return {"value": round(ops / t / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n + 1} of {w.B * w.H} heads at full L={w.L} ({what}), "
                       f"{t:.1f} s on {cores} threads"}
@@ -481,6 +516,8 @@ def main():
                     help="online: the INT8 FlashAttention path (default); index: the IndexSoftmax variant")
     ap.add_argument("--index-c", type=float, default=6.6, help="IndexSoftmax clip threshold c")
     ap.add_argument("--index-b", type=int, default=5, help="IndexSoftmax table bits b")
+    ap.add_argument("--scale-block", type=int, default=1,
+                    help="online method: one Q / K scale per block of this many tokens (1 = per token)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -488,6 +525,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl != "reference":
         raise SystemExit("--warmup must be >= 3")
+    if args.scale_block != 1 and (args.method != "online" or args.q_path != "separate"):
+        raise SystemExit("--scale-block applies to the online method with the separate Q pass")
     if args.impl == "reference":
         run_reference(args)
     else:

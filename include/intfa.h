@@ -160,6 +160,24 @@ int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *
                             int causal, void *O_f16, float *s_Q_out, void *stream);
 
 /*
+ * The fused attention of intfa_attention_fwd with group-wise Q and K scales
+ * (IntAttention section 3.3: per-block quantisation; the scales of each
+ * group factor out of Q_hat K_hat^T exactly as per-token scales do): one scale
+ * per block of scale_block consecutive tokens of a head.
+ *
+ *   s_Q, s_K    : fp32 [B][H][ceil(L / scale_block)]; the scale of token i is
+ *                 s[i / scale_block].  Codes as from intfa_quantize_per_tensor
+ *                 with groups = B*H*L/scale_block (L a multiple of scale_block).
+ *   scale_block : a power of two, 1 .. 65536 (1 = intfa_attention_fwd).
+ *   Other arguments, layouts and error behaviour as intfa_attention_fwd;
+ *   INTFA_ERR_INVALID_ARG for any other scale_block.
+ */
+int intfa_attention_fwd_blockscale(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                   const float *s_Q, const float *s_K, const float *s_V, int B,
+                                   int H, int L, int d, int causal, int scale_block, void *O_f16,
+                                   void *stream);
+
+/*
  * IndexSoftmax attention (IntAttention: A Fully Integer Attention Pipeline for
  * Efficient Edge Inference, section 3.1 eqs. 7-10, section 3.2, and eq. 5 for
  * the value path) with per-tensor scales, section 3.3's default

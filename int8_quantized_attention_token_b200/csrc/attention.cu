@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
                     const float *__restrict__ sK, const float *__restrict__ sV,
                     __half *__restrict__ O, int BH, int L, int causal,
-                    const uint4 *__restrict__ Qh, float *__restrict__ sQ_out) {
+                    const uint4 *__restrict__ Qh, float *__restrict__ sQ_out, int sshift) {
     AttnSmem<D, kQ16> &sm = get_smem<D, kQ16>();
     constexpr int NS = AttnSmem<D, kQ16>::NS;
     const int tid = threadIdx.x;
@@ -444,14 +444,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // s_K of a key block as four floats per lane (zero past the end);
         // the loads for the next block are issued one block ahead so that
         // their latency overlaps the wait for a free stage.
+        // With scale blocks of 2^sshift tokens (sshift = 0: one scale per
+        // token) the scale of key j is s_K[j >> sshift].
+        const int64_t nsc = (static_cast<int64_t>(L) + (1 << sshift) - 1) >> sshift;
         auto load_sk = [&](const Cursor &c) {
-            const float *src = sK + static_cast<int64_t>(c.T.bh) * L;
+            const float *src = sK + static_cast<int64_t>(c.T.bh) * nsc;
             const int key = c.j * BN + 4 * lane;
             float4 v4;
-            v4.x = key + 0 < L ? __ldg(src + key + 0) : 0.0f;
-            v4.y = key + 1 < L ? __ldg(src + key + 1) : 0.0f;
-            v4.z = key + 2 < L ? __ldg(src + key + 2) : 0.0f;
-            v4.w = key + 3 < L ? __ldg(src + key + 3) : 0.0f;
+            v4.x = key + 0 < L ? __ldg(src + ((key + 0) >> sshift)) : 0.0f;
+            v4.y = key + 1 < L ? __ldg(src + ((key + 1) >> sshift)) : 0.0f;
+            v4.z = key + 2 < L ? __ldg(src + ((key + 2) >> sshift)) : 0.0f;
+            v4.w = key + 3 < L ? __ldg(src + ((key + 3) >> sshift)) : 0.0f;
             return v4;
         };
         Cursor c = cursor_begin(ntiles, total, L, causal);
@@ -665,7 +668,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!warp_wait(&sm.sq_full[i & 7], (i >> 3) & 1, abort_flag, 19)) break;
                 s_q = sm.sq[i & 7][row];
             } else {
-                s_q = qi < L ? __ldg(sQ + static_cast<int64_t>(T.bh) * L + qi) : 0.0f;
+                const int64_t nsc = (static_cast<int64_t>(L) + (1 << sshift) - 1) >> sshift;
+                s_q = qi < L ? __ldg(sQ + static_cast<int64_t>(T.bh) * nsc + (qi >> sshift)) : 0.0f;
             }
             // c = s_Q[i] log2(e) / sqrt(d), so that t_ij log2(e) = c (S_ij s_K[j]).
             // Clamped to a tiny positive value: a zero Q row then still maps masked
@@ -963,7 +967,7 @@ unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
 template <int D, bool kQ16>
 int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                 float *sQ_out, const float *sK, const float *sV, int B, int H, int L, int causal,
-                void *O, cudaStream_t stream) {
+                void *O, cudaStream_t stream, int sshift = 0) {
     const int BH = B * H;
     const int64_t ld = intfa_vt_ld(L);
     const CUtensorMapSwizzle swz = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -997,7 +1001,7 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
     const unsigned grid = persistent_grid(static_cast<int64_t>(BH) * ntiles, ntiles, causal, nsm);
     attn_fwd_kernel<D, kQ16><<<grid, kThreads, smem, stream>>>(
         mq, mk, mv, sQ, sK, sV, static_cast<__half *>(O), BH, L, causal, static_cast<const uint4 *>(Qh),
-        sQ_out);
+        sQ_out, sshift);
     return cuda_status(cudaGetLastError());
 }
 
@@ -1022,11 +1026,13 @@ int launch_debug_qk(const int8_t *Qq, const int8_t *Kq, int BH, int L, int32_t *
 
 int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                          const float *sK, const float *sV, int B, int H, int L, int d, int causal,
-                         void *O, cudaStream_t stream) {
+                         void *O, cudaStream_t stream, int sshift) {
     if (d == 128)
-        return launch_attn<128, false>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal, O, stream);
+        return launch_attn<128, false>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal, O, stream,
+                                       sshift);
     if (d == 64)
-        return launch_attn<64, false>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal, O, stream);
+        return launch_attn<64, false>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal, O, stream,
+                                      sshift);
     return INTFA_ERR_UNSUPPORTED;
 }
 
@@ -1071,6 +1077,26 @@ extern "C" int intfa_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const i
         return INTFA_ERR_MISALIGNED;
     return launch_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
                                 static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int intfa_attention_fwd_blockscale(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                              const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                                              int L, int d, int causal, int scale_block, void *O_f16,
+                                              void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    int sshift = 0;
+    while (sshift <= 16 && (1 << sshift) != scale_block) ++sshift;
+    if (sshift > 16) return INTFA_ERR_INVALID_ARG;   // a power of two in 1 .. 65536
+    if (!Q_q || !K_q || !Vt_q || !s_Q || !s_K || !s_V || !O_f16) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(Vt_q) || !aligned16(O_f16) ||
+        (reinterpret_cast<uintptr_t>(s_Q) & 3u) || (reinterpret_cast<uintptr_t>(s_K) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_V) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    return launch_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
+                                static_cast<cudaStream_t>(stream), sshift);
 }
 
 extern "C" int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *Vt_q,

@@ -25,9 +25,10 @@ int launch_quantize_per_token(const void *x, int64_t rows, int d, int8_t *xq, fl
 int launch_quantize_per_tensor(const void *x, int64_t groups, int64_t rows, int cols,
                                int transpose, int8_t *xq, float *scale, void *workspace,
                                cudaStream_t stream);
+// sshift: one scale per 2^sshift consecutive tokens of Q and K (0: per token).
 int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt,
                          const float *sQ, const float *sK, const float *sV, int B, int H, int L,
-                         int d, int causal, void *O, cudaStream_t stream);
+                         int d, int causal, void *O, cudaStream_t stream, int sshift = 0);
 int launch_attention_fwd_q16(const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sK,
                              const float *sV, int B, int H, int L, int d, int causal, void *O,
                              float *sQ_out, cudaStream_t stream);

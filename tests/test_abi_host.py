@@ -87,6 +87,18 @@ def test_attention_rejects(L):
     assert L.intfa_debug_qk(FAKE, None, 1, 1, 128, 64, FAKE, None) == 1
 
 
+def test_blockscale_attention_rejects(L):
+    a = [FAKE] * 6
+    f = L.intfa_attention_fwd_blockscale
+    assert f(*a, 1, 1, 128, 64, 0, 3, FAKE, None) == 1          # not a power of two
+    assert f(*a, 1, 1, 128, 64, 0, 0, FAKE, None) == 1
+    assert f(*a, 1, 1, 128, 64, 0, 1 << 17, FAKE, None) == 1
+    assert f(*a, 1, 1, 128, 96, 0, 128, FAKE, None) == 2        # d
+    assert f(*a, 1, 1, 128, 64, 2, 128, FAKE, None) == 1        # causal flag
+    assert f(*a, 1, 1, 128, 64, 0, 128, None, None) == 1        # O
+    assert f(FAKE + 4, *a[1:], 1, 1, 128, 64, 0, 128, FAKE, None) == 3
+
+
 def test_index_attention_rejects(L):
     # Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, c, b, O, m_out, l_out, stream
     a = [FAKE] * 6
