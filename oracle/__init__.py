@@ -21,6 +21,9 @@ and marshals numpy arrays.  Each function cites the passage it follows:
   codes against the running max of the key blocks seen so far.  This is the
   form the fused kernel computes.
 * ``attention_fp64_rows`` -- IntAttention section 2.1, eq. 1.
+* ``decode`` -- one query against a key / value cache: the online form of
+  ``attention_online_rows`` run separately on consecutive key ranges
+  (split-KV) and merged (FlashAttention's block-wise softmax at range level).
 * ``index_lut``, ``index_cint``, ``index_attention_rows`` -- IntAttention
   sections 3.1-3.2 (IndexSoftmax: eqs. 7-10, the UINT8 exponential table,
   UINT8 P times 255, integer row sums) with per-tensor Q / K scales
@@ -70,6 +73,7 @@ def _load():
     lib.oracle_attention_online_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
                                                  ctypes.c_int, I64, I64, I64, P, P]
     lib.oracle_attention_fp64_rows.argtypes = [P, P, P, I64, I64, ctypes.c_int, I64, I64, P]
+    lib.oracle_decode.argtypes = [P, ctypes.c_float, P, P, P, ctypes.c_float, I64, I64, I64, I64, P]
     lib.oracle_index_lut.argtypes = [ctypes.c_double, ctypes.c_int, P]
     lib.oracle_index_cint.argtypes = [ctypes.c_double, I64, ctypes.c_float, ctypes.c_float]
     lib.oracle_index_cint.restype = I64
@@ -281,3 +285,23 @@ def index_attention_fwd(Qq, Kq, Vq, sQ, sK, sV, causal: bool, c: float = INDEX_C
         O[h], M[h], Ls[h] = index_attention_rows(Qq[h], Kq[h], Vq[h], float(sQ[h]), float(sK[h]),
                                                  float(sV[h]), causal, c, b, want_stats=True)
     return (O, M, Ls) if want_stats else O
+
+
+# ---------------------------------------------------------------- decode
+
+def decode(q, sq: float, Kq, sK, Vq, sV: float, block: int = 128, split_len=None):
+    """One query: q int8 [d] (scale sq), Kq / Vq int8 [L, d], sK fp32 [L], sV
+    the cache's value scale.  Keys in ranges of split_len (a multiple of
+    block; default: one range).  Returns O fp64 [d]."""
+    q = _c(q, np.int8)
+    Kq = _c(Kq, np.int8)
+    Vq = _c(Vq, np.int8)
+    sK = _c(sK, np.float32)
+    L, d = Kq.shape
+    split_len = -(-L // block) * block if split_len is None else int(split_len)
+    if split_len % block:
+        raise ValueError("split_len must be a multiple of block")
+    O = np.empty((d,), np.float64)
+    _load().oracle_decode(_ptr(q), float(sq), _ptr(Kq), _ptr(sK), _ptr(Vq), float(sV), L, d, int(block),
+                          max(split_len, block), _ptr(O))
+    return O

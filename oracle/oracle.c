@@ -29,6 +29,9 @@
  *                   running max), see oracle_attention_online_rows.
  *   reference       IntAttention section 2.1, eq. 1: O = softmax(Q K^T /
  *                   sqrt(d)) V in fp64 from the unquantised inputs.
+ *   decode          one query against a key / value cache with the keys cut
+ *                   into ranges (split-KV), each range in the online order,
+ *                   merged at the end; see oracle_decode.
  *   IndexSoftmax    IntAttention sections 3.1-3.2: integer clipping of the
  *                   row-max distance, a 2^b-entry UINT8 exponential table,
  *                   UINT8 P (times 255), integer row sums; see
@@ -396,4 +399,77 @@ void oracle_index_attention_rows(const int8_t *Qq, const int8_t *Kq, const int8_
         free(acc);
         free(e);
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* decode: one query against a key / value cache, split into ranges    */
+/* ------------------------------------------------------------------ */
+
+/*
+ * One query row of the quantised attention against L keys (no mask), in the
+ * block-wise online order of oracle_attention_online_rows, with the keys cut
+ * into consecutive ranges of split_len keys (split_len a multiple of
+ * `block`).  Each range runs the online steps on its own (running max, P
+ * codes against that range's running max, integer block sums, alpha
+ * rescales), and the ranges are merged at the end (FlashAttention's
+ * block-wise softmax applied once more at range granularity):
+ *   M = max_s m_s,  O = s_V sum_s e^(m_s - M) acc_s / (127 sum_s e^(m_s - M) l_s).
+ * With split_len >= L this is exactly one row of oracle_attention_online_rows.
+ * q: int8 [d] with scale sq; Kq, Vq: int8 [L][d]; sK: fp32 [L].
+ */
+void oracle_decode(const int8_t *q, float sq, const int8_t *Kq, const float *sK, const int8_t *Vq,
+                   float sV, int64_t L, int64_t d, int64_t block, int64_t split_len, double *O) {
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    const int64_t nsplit = (L + split_len - 1) / split_len;
+    double *ms = (double *)malloc((size_t)nsplit * sizeof(double));
+    double *ls = (double *)malloc((size_t)nsplit * sizeof(double));
+    double *accs = (double *)calloc((size_t)(nsplit * d), sizeof(double));
+    double *t = (double *)malloc((size_t)block * sizeof(double));
+    int64_t *blk = (int64_t *)malloc((size_t)d * sizeof(int64_t));
+    for (int64_t s = 0; s < nsplit; ++s) {
+        const int64_t s0 = s * split_len;
+        const int64_t s1 = (s0 + split_len < L) ? s0 + split_len : L;
+        double m = -INFINITY, l = 0.0;
+        double *acc = accs + s * d;
+        for (int64_t j0 = s0; j0 < s1; j0 += block) {
+            const int64_t nb = (s1 - j0 < block) ? (s1 - j0) : block;
+            double bm = -INFINITY;
+            for (int64_t jj = 0; jj < nb; ++jj) {
+                const int64_t j = j0 + jj;
+                t[jj] = (double)dot_i8(q, Kq + j * d, d) * (double)sq * (double)sK[j] * inv_sqrt_d;
+                if (t[jj] > bm) bm = t[jj];
+            }
+            const double m_new = (bm > m) ? bm : m;
+            const double alpha = (m == -INFINITY) ? 0.0 : exp(m - m_new);
+            double psum = 0.0;
+            for (int64_t c = 0; c < d; ++c) blk[c] = 0;
+            for (int64_t jj = 0; jj < nb; ++jj) {
+                const double p = exp(t[jj] - m_new);
+                psum += p;
+                const int64_t code = (int64_t)nearbyint(127.0 * p);
+                const int8_t *v = Vq + (j0 + jj) * d;
+                for (int64_t c = 0; c < d; ++c) blk[c] += code * (int64_t)v[c];
+            }
+            for (int64_t c = 0; c < d; ++c) acc[c] = alpha * acc[c] + (double)blk[c];
+            l = alpha * l + psum;
+            m = m_new;
+        }
+        ms[s] = m;
+        ls[s] = l;
+    }
+    double M = -INFINITY;
+    for (int64_t s = 0; s < nsplit; ++s) if (ms[s] > M) M = ms[s];
+    double den = 0.0;
+    for (int64_t c = 0; c < d; ++c) O[c] = 0.0;
+    for (int64_t s = 0; s < nsplit; ++s) {
+        const double w = exp(ms[s] - M);
+        den += w * ls[s];
+        for (int64_t c = 0; c < d; ++c) O[c] += w * accs[s * d + c];
+    }
+    for (int64_t c = 0; c < d; ++c) O[c] = (double)sV * O[c] / (127.0 * den);
+    free(ms);
+    free(ls);
+    free(accs);
+    free(t);
+    free(blk);
 }
