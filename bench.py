@@ -42,7 +42,8 @@ def kernel_sources_sha(method: str = "online") -> str:
     """Hash of the dominant kernel's sources (the attention kernel of `method`)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_quantized_attention_token_b200", "csrc")
-    files = ("attention.cu", "ptx.cuh", "quant_math.cuh") if method == "online" else ("index_attention.cu", "ptx.cuh")
+    files = {"online": ("attention.cu", "ptx.cuh", "quant_math.cuh"), "index": ("index_attention.cu", "ptx.cuh"),
+             "decode": ("decode.cu", "ptx.cuh", "quant_math.cuh")}[method]
     for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
@@ -387,6 +388,139 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------- decode ---
+
+def run_decode(args):
+    """One query per head against a resident INT8 key / value cache
+    (intfa_decode_fwd: split-KV partial kernel + merge).  HBM-bound: the
+    roofline is the cache bytes read per call over the call's time."""
+    import numpy as np
+    import torch
+
+    from int8_quantized_attention_token_b200 import intfa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    B, H, L, d = (int(x) for x in args.decode_shape.split(","))
+    BH = B * H
+    splits = args.splits if args.splits > 0 else max(1, -(-4 * 148 // BH))
+    g = torch.Generator().manual_seed(0)
+    q = torch.randn(B, H, d, generator=g).half()
+    K = torch.randn(B, H, L, d, generator=g).half()
+    V = torch.randn(B, H, L, d, generator=g).half()
+    Kq, sK = intfa.intfa_quantize_per_token(K.to(dev))
+    Vq, sV = intfa.intfa_quantize_per_tensor(V.to(dev).reshape(BH, L, d), transpose=False)
+    Vq, sV = Vq.reshape(B, H, L, d), sV.reshape(B, H)
+    qd = q.to(dev)
+    O = torch.empty(B, H, d, dtype=torch.float16, device=dev)
+    ws = torch.empty(int(intfa.lib().intfa_decode_workspace_size(B, H, d, splits)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    # a buffer larger than L2, written between timed calls: the cache (2 GB at
+    # the default shape) exceeds L2 anyway, the flush keeps small shapes honest
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        intfa.intfa_decode_fwd(qd, Kq, sK, Vq, sV, splits, O, ws, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    if intfa.intfa_device_status(clear=True) != 0:
+        raise RuntimeError("a kernel timed out during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    h0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        call()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    h1 = time.perf_counter()
+    time.sleep(0.1)
+    clk = clocks.stop(h0, h1)
+    if intfa.intfa_device_status(clear=True) != 0:
+        raise RuntimeError("a kernel timed out during the timed region")
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    ms = max_over_ranks(ms, dev)
+    ops = 4.0 * d * BH * L
+    cache_bytes = BH * L * (2 * d + 4)
+    io_bytes = BH * d * 2 * 2 + BH * splits * (d + 2) * 4 * 2
+    gbs = (cache_bytes + io_bytes) / (ms * 1e-3) / 1e9
+    pk = peaks()
+
+    e2e = None
+    if not args.no_e2e:   # the query from pinned host memory, O back to the host
+        qp = q.pin_memory()
+        Op = torch.empty(B, H, d, dtype=torch.float16).pin_memory()
+        e_steps = max(3, min(args.steps, 20))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            qd.copy_(qp, non_blocking=True)
+            call()
+            Op.copy_(O, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev) / e_steps
+        e2e = {"value": ops * world / (e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": BH * d * 2,
+               "d2h_bytes_per_step": BH * d * 2, "steps": e_steps, "ms_per_step": e_ms,
+               "api": "intfa_decode_fwd with the query copied from pinned host memory and O copied back"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        cores = len(os.sched_getaffinity(0))
+        oracle.set_threads(cores)
+        nblk = -(-L // 128)
+        split_len = -(-nblk // splits) * 128
+        t, n = 0.0, 0
+        while t < args.cpu_seconds and n < BH:
+            b, h = n // H, n % H
+            t0 = time.perf_counter()
+            qq, sq = oracle.quantize_per_token(q[b, h].float().numpy()[None, :])
+            kq, sk = oracle.quantize_per_token(K[b, h].float().numpy())
+            vq, sv = oracle.quantize_per_tensor(V[b, h].float().numpy(), 1)
+            oracle.decode(qq[0], float(sq[0]), kq, sk, vq, float(sv[0]), 128, split_len)
+            t += time.perf_counter() - t0
+            n += 1
+        cpu = {"value": round(4.0 * d * L * n / t / 1e12, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{n} of {BH} heads (quantise the query and the head's cache, decode), {t:.1f} s, "
+                         "single-threaded (the decode oracle has no thread loop)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(ops * world / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic (seeded N(0,1) fp16 q/K/V)",
+            "config": {"workload": f"decode_B{B}_H{H}_L{L}_d{d}", "B": B, "H": H, "L": L, "d": d, "splits": splits,
+                       "method": "decode", "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "256 MiB buffer written between timed calls; cache of %.2f GB" % (cache_bytes / 1e9)},
+            "roofline": {"bound": "hbm", "kernel": f"decode_partial_kernel<{d}> + decode_combine_kernel<{d}>",
+                         "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": None,
+                         "peak_note": f"{pk['source']} HBM copy bandwidth",
+                         "bytes_per_call": cache_bytes + io_bytes},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clk,
+            "kernel_sha": kernel_sources_sha("decode"),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 # --------------------------------------------------------------- CPU arm ---
 
 def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5, blk=1):
@@ -512,8 +646,11 @@ def main():
     ap.add_argument("--impl", default="libintfa", choices=["libintfa", "reference"])
     ap.add_argument("--q-path", default="separate", choices=["fused", "separate"],
                     help="quantise Q in its own pass (default, faster) or inside the attention kernel")
-    ap.add_argument("--method", default="online", choices=["online", "index"],
-                    help="online: the INT8 FlashAttention path (default); index: the IndexSoftmax variant")
+    ap.add_argument("--method", default="online", choices=["online", "index", "decode"],
+                    help="online: the INT8 FlashAttention path (default); index: the IndexSoftmax variant; "
+                         "decode: one query per head against an INT8 cache")
+    ap.add_argument("--decode-shape", default="8,32,32768,128", help="decode: B,H,L,d")
+    ap.add_argument("--splits", type=int, default=0, help="decode: key ranges per head (0: auto)")
     ap.add_argument("--index-c", type=float, default=6.6, help="IndexSoftmax clip threshold c")
     ap.add_argument("--index-b", type=int, default=5, help="IndexSoftmax table bits b")
     ap.add_argument("--scale-block", type=int, default=1,
@@ -529,6 +666,8 @@ def main():
         raise SystemExit("--scale-block applies to the online method with the separate Q pass")
     if args.impl == "reference":
         run_reference(args)
+    elif args.method == "decode":
+        run_decode(args)
     else:
         run_gpu(args)
 

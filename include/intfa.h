@@ -212,6 +212,34 @@ int intfa_index_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const int8_t
                               int32_t *m_out, int32_t *l_out, void *stream);
 
 /*
+ * Decode: one query per head against an INT8 key / value cache, the online
+ * form of intfa_attention_fwd (INT-FlashAttention abstract; IntAttention eqs.
+ * 3-6, section 3.2, eq. 5) for a single query row, with the keys cut into
+ * `splits` ranges of split_len = ceil(ceil(L / 128) / splits) * 128 keys that
+ * each run the block-wise steps on their own (running max, P codes against
+ * that range's running max) and are merged at the end:
+ *   M = max_s m_s,  O = s_V sum_s e^(m_s - M) acc_s / (127 sum_s e^(m_s - M) l_s).
+ * The query is quantised per token inside the kernel (bit-identical to
+ * intfa_quantize_per_token).  No mask: every cache entry is visible.
+ *
+ *   q_f16  : fp16 [B][H][d], 16-byte aligned.
+ *   K_q    : int8 [B][H][L][d] per-token codes (intfa_quantize_per_token),
+ *            s_K fp32 [B][H][L].
+ *   V_q    : int8 [B][H][L][d] per-head codes, row-major
+ *            (intfa_quantize_per_tensor, groups = B*H, transpose = 0), s_V
+ *            fp32 [B][H].
+ *   splits : 1 .. 65535 ranges per head (ranges past the end are empty).
+ *   O_f16  : fp16 [B][H][d] out.
+ *   workspace : device scratch of intfa_decode_workspace_size(B, H, d,
+ *            splits) bytes, 16-byte aligned (the per-range partial results).
+ *   d in {64, 128}; 1 <= L <= 2^24; B*H <= 65535.
+ */
+size_t intfa_decode_workspace_size(int B, int H, int d, int splits);
+int intfa_decode_fwd(const void *q_f16, const int8_t *K_q, const float *s_K, const int8_t *V_q,
+                     const float *s_V, int B, int H, int L, int d, int splits, void *O_f16,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Debug: the integer logits S = Q_hat K_hat^T (IntAttention eq. 4) for every
  * head, int32 [B][H][L][L], computed by the same TMA + tcgen05 path the fused
  * kernel uses for its first contraction.  Same layout rules as

@@ -8,7 +8,7 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["quantize.cu", "attention.cu", "index_attention.cu", "api.cu"]
+SOURCES = ["quantize.cu", "attention.cu", "index_attention.cu", "decode.cu", "api.cu"]
 HEADERS = ["ptx.cuh", "quant_math.cuh", "internal.h", "tma_host.h"]
 LIB = os.path.join(PKG, "libintfa.so")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include", "intfa.h")

@@ -1143,6 +1143,9 @@ extern "C" int intfa_device_status(int clear, uint32_t *word) {
     rc = read_index_status(clear, &wi);   // the IndexSoftmax kernel's word
     if (rc) return rc;
     if (!w) w = wi;
+    rc = read_decode_status(clear, &wi);  // the decode kernels' word
+    if (rc) return rc;
+    if (!w) w = wi;
     if (word) *word = w;
     return w ? INTFA_ERR_DEVICE_TIMEOUT : INTFA_OK;
 }

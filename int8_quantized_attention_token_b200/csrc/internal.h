@@ -34,5 +34,7 @@ int launch_attention_fwd_q16(const void *Qh, const int8_t *Kq, const int8_t *Vt,
                              float *sQ_out, cudaStream_t stream);
 // The IndexSoftmax kernel's status word (index_attention.cu); clear resets it.
 int read_index_status(int clear, uint32_t *word);
+// The decode kernels' status word (decode.cu); clear resets it.
+int read_decode_status(int clear, uint32_t *word);
 
 }  // namespace intfa

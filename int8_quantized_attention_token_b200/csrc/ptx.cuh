@@ -110,6 +110,15 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint64_t *ba
 // ------------------------------------------------------------ tcgen05 ---
 
 // Warp-wide: allocate `ncols` TMEM columns, base address written to *dst.
+// Contiguous global -> shared copy by the copy engine (no tensor map, no
+// multicast); bytes and both addresses 16-byte aligned; completes `bytes` of
+// the mbarrier's transaction count.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(dst)),

@@ -52,6 +52,8 @@ def lib():
         "intfa_attention_fwd_q16": ([P, P, P, P, P, I, I, I, I, I, P, P, P], I),
         "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
         "intfa_attention_fwd_blockscale": ([P, P, P, P, P, P, I, I, I, I, I, I, P, P], I),
+        "intfa_decode_workspace_size": ([I, I, I, I], SZ),
+        "intfa_decode_fwd": ([P, P, P, P, P, I, I, I, I, I, P, P, SZ, P], I),
         "intfa_index_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, ctypes.c_double, I, P, P, P, P], I),
         "intfa_forward_workspace_size": ([I, I, I, I], SZ),
         "intfa_forward_workspace_layout": ([I, I, I, I, ctypes.POINTER(SZ)], I),
@@ -237,6 +239,26 @@ def intfa_index_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, c: fl
                                            _ptr(m_out) if m_out is not None else None,
                                            _ptr(l_out) if l_out is not None else None,
                                            _stream(stream)), "intfa_index_attention_fwd")
+    return O
+
+
+def intfa_decode_fwd(q, K_q, s_K, V_q, s_V, splits: int = 1, O=None, workspace=None, stream=None):
+    """One query per head against an INT8 cache: q fp16 [B, H, d]; K_q, V_q
+    int8 [B, H, L, d] (per-token K codes, per-head V codes); s_K fp32 [B, H, L];
+    s_V fp32 [B, H]  ->  O fp16 [B, H, d]."""
+    _need(q, torch.float16, "q")
+    for t, n in ((K_q, "K_q"), (V_q, "V_q")):
+        _need(t, torch.int8, n)
+    for t, n in ((s_K, "s_K"), (s_V, "s_V")):
+        _need(t, torch.float32, n)
+    B, H, L, d = K_q.shape
+    O = torch.empty((B, H, d), dtype=torch.float16, device=q.device) if O is None else O
+    wsb = int(lib().intfa_decode_workspace_size(B, H, d, int(splits)))
+    if workspace is None:
+        workspace = torch.empty((max(wsb, 16),), dtype=torch.uint8, device=q.device)
+    _check(lib().intfa_decode_fwd(_ptr(q), _ptr(K_q), _ptr(s_K), _ptr(V_q), _ptr(s_V), B, H, L, d, int(splits),
+                                  _ptr(O), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "intfa_decode_fwd")
     return O
 
 

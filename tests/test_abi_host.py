@@ -99,6 +99,22 @@ def test_blockscale_attention_rejects(L):
     assert f(FAKE + 4, *a[1:], 1, 1, 128, 64, 0, 128, FAKE, None) == 3
 
 
+def test_decode_rejects(L):
+    ws = L.intfa_decode_workspace_size(1, 2, 128, 4)
+    assert ws == 1 * 2 * 4 * 130 * 4
+    assert L.intfa_decode_workspace_size(1, 2, 96, 4) == 0
+    # q, K_q, s_K, V_q, s_V, B, H, L, d, splits, O, workspace, bytes, stream
+    f = L.intfa_decode_fwd
+    a = [FAKE] * 5
+    assert f(*a, 1, 2, 100, 96, 4, FAKE, FAKE, ws, None) == 2           # d
+    assert f(*a, 1, 2, 0, 128, 4, FAKE, FAKE, ws, None) == 1            # L
+    assert f(*a, 1, 2, 100, 128, 0, FAKE, FAKE, ws, None) == 1          # splits
+    assert f(*a, 1, 2, 100, 128, 4, FAKE, FAKE, ws - 1, None) == 1      # workspace too small
+    assert f(*a, 1, 2, 100, 128, 4, FAKE, None, ws, None) == 1
+    assert f(FAKE + 8, *a[1:], 1, 2, 100, 128, 4, FAKE, FAKE, ws, None) == 3
+    assert f(*a, 1, 2, 100, 128, 4, FAKE + 1, FAKE, ws, None) == 3      # O alignment
+
+
 def test_index_attention_rejects(L):
     # Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, c, b, O, m_out, l_out, stream
     a = [FAKE] * 6
