@@ -71,7 +71,7 @@ def _load():
     lib.oracle_attention_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
                                           ctypes.c_int, I64, I64, P, P, P, P]
     lib.oracle_attention_online_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
-                                                 ctypes.c_int, I64, I64, I64, P, P]
+                                                 ctypes.c_int, I64, I64, I64, P, P, ctypes.c_int]
     lib.oracle_attention_fp64_rows.argtypes = [P, P, P, I64, I64, ctypes.c_int, I64, I64, P]
     lib.oracle_decode.argtypes = [P, ctypes.c_float, P, P, P, ctypes.c_float, I64, I64, I64, I64, P]
     lib.oracle_index_lut.argtypes = [ctypes.c_double, ctypes.c_int, P]
@@ -162,10 +162,11 @@ def attention_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, r0: int = 0, r1=
 
 
 def attention_online_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, block: int = 128,
-                          r0: int = 0, r1=None, want_l: bool = False):
+                          r0: int = 0, r1=None, want_l: bool = False, lsum_codes: bool = False):
     """One head, block-wise online form (FlashAttention's forward workflow):
     P codes against the running max over key blocks of ``block``.  Returns O
-    fp64 [r1 - r0, d] (and the row sums l with want_l)."""
+    fp64 [r1 - r0, d] (and the row sums l with want_l).  lsum_codes: the row
+    sum from the P codes (sum P_hat / 127) instead of the unquantised p."""
     Qq = _c(Qq, np.int8)
     Kq = _c(Kq, np.int8)
     Vq = _c(Vq, np.int8)
@@ -177,7 +178,7 @@ def attention_online_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, block: in
     l = np.empty((r1 - r0,), np.float64) if want_l else None
     _load().oracle_attention_online_rows(_ptr(Qq), _ptr(Kq), _ptr(Vq), _ptr(sQ), _ptr(sK),
                                          float(sV), L, d, int(bool(causal)), int(block),
-                                         r0, r1, _ptr(O), _ptr(l))
+                                         r0, r1, _ptr(O), _ptr(l), int(bool(lsum_codes)))
     return (O, l) if want_l else O
 
 

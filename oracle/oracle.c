@@ -218,11 +218,14 @@ void oracle_attention_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
  *   l     = alpha l + sum_j p_ij
  * and finally O = s_V acc / (127 l) (IntAttention eq. 5).  With one block
  * this is exactly the two-pass function above.
+ * lsum_codes != 0 takes the other reading of the row sum: l from the P codes,
+ * l = alpha l + sum_j codes_ij / 127 (IntAttention section 3.2 quantises P
+ * before the value product; the pages do not say which p the sum uses).
  */
 void oracle_attention_online_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
                                   const float *sQ, const float *sK, float sV,
                                   int64_t L, int64_t d, int causal, int64_t block,
-                                  int64_t r0, int64_t r1, double *O, double *l_out) {
+                                  int64_t r0, int64_t r1, double *O, double *l_out, int lsum_codes) {
     const double inv_sqrt_d = 1.0 / sqrt((double)d);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t i = r0; i < r1; ++i) {
@@ -246,8 +249,8 @@ void oracle_attention_online_rows(const int8_t *Qq, const int8_t *Kq, const int8
             for (int64_t c = 0; c < d; ++c) blk[c] = 0;
             for (int64_t jj = 0; jj < nb; ++jj) {
                 double p = exp(t[jj] - m_new);
-                psum += p;
                 int64_t code = (int64_t)nearbyint(127.0 * p);
+                psum += lsum_codes ? (double)code / 127.0 : p;
                 const int8_t *v = Vq + (j0 + jj) * d;
                 for (int64_t c = 0; c < d; ++c) blk[c] += code * (int64_t)v[c];
             }

@@ -275,3 +275,37 @@ def test_online_constant_logits(causal):
     for i in range(L):
         n = i + 1 if causal else L
         np.testing.assert_allclose(O[i], 0.25 * Vq[:n].astype(np.float64).mean(0), rtol=1e-13, atol=1e-15)
+
+
+# ------------------------------------------ row sum from the P codes (f3) ---
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_codesum_constant_logits_give_mean_of_values(causal):
+    # Q_hat = 0: every code is 127, so sum codes / 127 = the number of keys and
+    # O is the mean of the visible V_hat rows, as with the p-sum
+    rng = np.random.default_rng(21)
+    L, d = 200, 64
+    Qq = np.zeros((L, d), np.int8)
+    Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d)
+    sQ = rng.uniform(0.01, 0.1, L).astype(np.float32)
+    sK = rng.uniform(0.01, 0.1, L).astype(np.float32)
+    O = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, 0.5, causal, 128, lsum_codes=True)
+    for i in range(L):
+        n = i + 1 if causal else L
+        np.testing.assert_allclose(O[i], 0.5 * Vq[:n].astype(np.float64).mean(axis=0), rtol=0, atol=1e-12)
+
+
+def test_codesum_one_block_is_the_code_weighted_mean():
+    # one key block: the online form is the two-pass form, and with the row
+    # sum taken from the codes O_i = s_V sum_j P_ij V_j / sum_j P_ij exactly,
+    # with the P codes of the (separately pinned) two-pass function
+    rng = np.random.default_rng(22)
+    L, d = 100, 128
+    Qq, Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d), rand_i8(rng, L, d)
+    sQ = rng.uniform(0.002, 0.01, L).astype(np.float32)
+    sK = rng.uniform(0.002, 0.01, L).astype(np.float32)
+    sV = float(np.float32(0.03))
+    _, P = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, sV, False, want_P=True)
+    O = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, sV, False, 128, lsum_codes=True)
+    want = sV * (P.astype(np.float64) @ Vq.astype(np.float64)) / P.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(O, want, rtol=1e-12, atol=1e-12)
