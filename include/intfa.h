@@ -160,6 +160,18 @@ int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *
                             int causal, void *O_f16, float *s_Q_out, void *stream);
 
 /*
+ * The fused attention of intfa_attention_fwd with the other reading of the
+ * row sum: l = alpha l + sum_j P_hat_ij / 127 (the sum of the INT8 P codes,
+ * IntAttention section 3.2 quantising P before the value product) instead of
+ * the sum of the unquantised p.  O = s_V acc / (127 l) is then the P-code
+ * weighted mean of V_hat.  Arguments, layouts and errors as
+ * intfa_attention_fwd.
+ */
+int intfa_attention_fwd_codesum(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                                int L, int d, int causal, void *O_f16, void *stream);
+
+/*
  * The fused attention of intfa_attention_fwd with group-wise Q and K scales
  * (IntAttention section 3.3: per-block quantisation; the scales of each
  * group factor out of Q_hat K_hat^T exactly as per-token scales do): one scale

@@ -333,10 +333,13 @@ __device__ __forceinline__ void max_v(const uint32_t (&w)[32], float (&mx)[4]) {
 }
 
 // One 32-key chunk of v: p = 2^(c v - c m) (<= 1; 0 for masked keys), the
-// running pair sums of p, and the 32 P codes RNE(127 p) packed four per word
-// (the code is the low byte of fl(127 p + 1.5 * 2^23)).
+// running pair sums of p (or, kCodes, the integer sum of the P codes), and
+// the 32 P codes RNE(127 p) packed four per word (the code is the low byte of
+// fl(127 p + 1.5 * 2^23)).
+template <bool kCodes>
 __device__ __forceinline__ void exp_codes(const uint32_t (&w)[32], uint64_t c2, uint64_t ncm2, uint64_t k127,
-                                          uint64_t magic, uint64_t &ps01, uint64_t &ps23, uint32_t (&pk)[8]) {
+                                          uint64_t magic, uint64_t &ps01, uint64_t &ps23, uint32_t (&pk)[8],
+                                          uint32_t &csum) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         float x0, x1, x2, x3;
@@ -344,13 +347,16 @@ __device__ __forceinline__ void exp_codes(const uint32_t (&w)[32], uint64_t c2, 
         f2_unpack(ffma2(f2_pack(__uint_as_float(w[4 * q + 2]), __uint_as_float(w[4 * q + 3])), c2, ncm2), x2, x3);
         const uint64_t p01 = f2_pack(ex2(x0), ex2(x1));
         const uint64_t p23 = f2_pack(ex2(x2), ex2(x3));
-        ps01 = fadd2(ps01, p01);
-        ps23 = fadd2(ps23, p23);
+        if constexpr (!kCodes) {
+            ps01 = fadd2(ps01, p01);
+            ps23 = fadd2(ps23, p23);
+        }
         float t0, t1, t2, t3;
         f2_unpack(ffma2(p01, k127, magic), t0, t1);
         f2_unpack(ffma2(p23, k127, magic), t2, t3);
         pk[q] = prmt(prmt(__float_as_uint(t0), __float_as_uint(t1), 0x0040u),
                      prmt(__float_as_uint(t2), __float_as_uint(t3), 0x0040u), 0x5410u);
+        if constexpr (kCodes) csum = __dp4a(pk[q], 0x01010101u, csum);
     }
 }
 
@@ -360,7 +366,9 @@ __device__ __forceinline__ void exp_codes(const uint32_t (&w)[32], uint64_t c2, 
 // by roles 14-15 (bit-identical to quant_per_token_kernel); its scales go to
 // the softmax warps through shared memory and, if sQ_out is set, to global.
 // Otherwise Q_hat arrives through tmQ and s_Q through sQ.
-template <int D, bool kQ16>
+// kLCodes: the row sum from the P codes, l = alpha l + sum_j P_hat_ij / 127,
+// instead of the unquantised p (the other reading of the pages).
+template <int D, bool kQ16, bool kLCodes = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
@@ -744,6 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float cm = c * m_new;
                 const uint64_t ncm2 = f2_pack(-cm, -cm);
                 uint64_t ps01 = 0ull, ps23 = 0ull;
+                uint32_t csum = 0;
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
                     uint32_t w0[32], w1[32];
@@ -751,15 +760,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(ts + 64 * h + 32, w1);
                     tmem_wait_ld();
                     uint32_t pk0[8], pk1[8];
-                    exp_codes(w0, c2, ncm2, k127, magic, ps01, ps23, pk0);
-                    exp_codes(w1, c2, ncm2, k127, magic, ps01, ps23, pk1);
+                    exp_codes<kLCodes>(w0, c2, ncm2, k127, magic, ps01, ps23, pk0, csum);
+                    exp_codes<kLCodes>(w1, c2, ncm2, k127, magic, ps01, ps23, pk1, csum);
                     tmem_st8(ts + 64 * h, pk0);
                     tmem_st8(ts + 64 * h + 32, pk1);
                 }
-                float ps0, ps1, ps2, ps3;
-                f2_unpack(ps01, ps0, ps1);
-                f2_unpack(ps23, ps2, ps3);
-                l = l * lscale + ((ps0 + ps1) + (ps2 + ps3));
+                float bsum;
+                if constexpr (kLCodes) {
+                    bsum = static_cast<float>(csum) * (1.0f / 127.0f);
+                } else {
+                    float ps0, ps1, ps2, ps3;
+                    f2_unpack(ps01, ps0, ps1);
+                    f2_unpack(ps23, ps2, ps3);
+                    bsum = (ps0 + ps1) + (ps2 + ps3);
+                }
+                l = l * lscale + bsum;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.p_full[b]);
@@ -964,7 +979,7 @@ unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
 }
 
 // Qq (int8, with sQ) when !kQ16; Qh (fp16, scales optionally to sQ_out) when kQ16.
-template <int D, bool kQ16>
+template <int D, bool kQ16, bool kLCodes = false>
 int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                 float *sQ_out, const float *sK, const float *sV, int B, int H, int L, int causal,
                 void *O, cudaStream_t stream, int sshift = 0) {
@@ -984,13 +999,13 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     const size_t smem = attn_smem_bytes<D, kQ16>();
-    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D, kQ16>,
+    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D, kQ16, kLCodes>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
     if (rc) return rc;
     // The in-kernel register split assumes exactly kLaunchRegs per thread at
     // launch; a different count could leave setmaxnreg.inc waiting forever.
     cudaFuncAttributes fa;
-    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kQ16>));
+    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kQ16, kLCodes>));
     if (rc) return rc;
     if (fa.numRegs != kLaunchRegs) return INTFA_ERR_UNSUPPORTED;
     const int ntiles = (L + BM - 1) / BM;
@@ -999,7 +1014,7 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
     if (!rc) rc = cuda_status(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
     if (rc) return rc;
     const unsigned grid = persistent_grid(static_cast<int64_t>(BH) * ntiles, ntiles, causal, nsm);
-    attn_fwd_kernel<D, kQ16><<<grid, kThreads, smem, stream>>>(
+    attn_fwd_kernel<D, kQ16, kLCodes><<<grid, kThreads, smem, stream>>>(
         mq, mk, mv, sQ, sK, sV, static_cast<__half *>(O), BH, L, causal, static_cast<const uint4 *>(Qh),
         sQ_out, sshift);
     return cuda_status(cudaGetLastError());
@@ -1097,6 +1112,25 @@ extern "C" int intfa_attention_fwd_blockscale(const int8_t *Q_q, const int8_t *K
         return INTFA_ERR_MISALIGNED;
     return launch_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
                                 static_cast<cudaStream_t>(stream), sshift);
+}
+
+extern "C" int intfa_attention_fwd_codesum(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                           const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                                           int L, int d, int causal, void *O_f16, void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    if (!Q_q || !K_q || !Vt_q || !s_Q || !s_K || !s_V || !O_f16) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(Vt_q) || !aligned16(O_f16) ||
+        (reinterpret_cast<uintptr_t>(s_Q) & 3u) || (reinterpret_cast<uintptr_t>(s_K) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_V) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        return launch_attn<128, false, true>(Q_q, nullptr, K_q, Vt_q, s_Q, nullptr, s_K, s_V, B, H, L, causal,
+                                             O_f16, s);
+    return launch_attn<64, false, true>(Q_q, nullptr, K_q, Vt_q, s_Q, nullptr, s_K, s_V, B, H, L, causal, O_f16, s);
 }
 
 extern "C" int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *Vt_q,

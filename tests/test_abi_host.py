@@ -87,6 +87,15 @@ def test_attention_rejects(L):
     assert L.intfa_debug_qk(FAKE, None, 1, 1, 128, 64, FAKE, None) == 1
 
 
+def test_codesum_attention_rejects(L):
+    a = [FAKE] * 6
+    f = L.intfa_attention_fwd_codesum
+    assert f(*a, 1, 1, 128, 96, 0, FAKE, None) == 2
+    assert f(*a, 1, 1, 128, 64, 2, FAKE, None) == 1
+    assert f(None, *a[1:], 1, 1, 128, 64, 0, FAKE, None) == 1
+    assert f(*a, 1, 1, 128, 64, 0, FAKE + 8, None) == 3
+
+
 def test_blockscale_attention_rejects(L):
     a = [FAKE] * 6
     f = L.intfa_attention_fwd_blockscale
