@@ -92,6 +92,20 @@ int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int64_t rows, i
                               size_t workspace_bytes, void *stream);
 
 /*
+ * One scale for the whole tensor (IntAttention section 2.1, eq. 3 applied to
+ * all groups together; the pages' per-tensor V taken literally, SURVEY's
+ * groups = 1 reading): s = fl32(max over all groups of max|x| / 127), the
+ * codes of every group with that s, in the same per-group layout as
+ * intfa_quantize_per_tensor (transpose 0 or 1), and s written to each of the
+ * `groups` scale slots, so that the attention entry points (one s_V per head)
+ * take it unchanged.  Arguments, workspace and errors as
+ * intfa_quantize_per_tensor.
+ */
+int intfa_quantize_global(const void *x_f16, int64_t groups, int64_t rows, int cols, int transpose,
+                          int8_t *x_q, float *scale, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/*
  * Per-tensor quantisation without any device allocation.  The pages have no
  * counterpart to this entry point; it exists for callers that cannot allocate
  * device memory themselves and therefore cannot supply the workspace that

@@ -22,9 +22,10 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Launchers implemented in quantize.cu / attention.cu (arguments already checked).
 int launch_quantize_per_token(const void *x, int64_t rows, int d, int8_t *xq, float *scale,
                               cudaStream_t stream);
+// global: one scale over all groups (written to every group's slot).
 int launch_quantize_per_tensor(const void *x, int64_t groups, int64_t rows, int cols,
                                int transpose, int8_t *xq, float *scale, void *workspace,
-                               cudaStream_t stream);
+                               cudaStream_t stream, bool global = false);
 // sshift: one scale per 2^sshift consecutive tokens of Q and K (0: per token).
 int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt,
                          const float *sQ, const float *sK, const float *sV, int B, int H, int L,

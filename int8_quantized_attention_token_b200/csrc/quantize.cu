@@ -101,6 +101,21 @@ __global__ void __launch_bounds__(256) group_amax_kernel(const uint4 *__restrict
     }
 }
 
+// Between the phases, for one scale over all groups: every group's slot gets
+// the maximum over the groups (one block).
+__global__ void __launch_bounds__(256) global_amax_kernel(unsigned *__restrict__ ws, int64_t groups) {
+    unsigned m = 0u;
+    for (int64_t g = threadIdx.x; g < groups; g += blockDim.x) m = max(m, ws[g]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ unsigned part[8];
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = part[0];
+    for (int w = 1; w < (blockDim.x >> 5); ++w) m = max(m, part[w]);
+    for (int64_t g = threadIdx.x; g < groups; g += blockDim.x) ws[g] = m;
+}
+
 // Phase 2, same layout as the input.
 __global__ void __launch_bounds__(256) group_convert_kernel(const uint4 *__restrict__ x,
                                                             int64_t n8,
@@ -215,7 +230,7 @@ int launch_quantize_per_token(const void *x, int64_t rows, int d, int8_t *xq, fl
 
 int launch_quantize_per_tensor(const void *x, int64_t groups, int64_t rows, int cols,
                                int transpose, int8_t *xq, float *scale, void *workspace,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, bool global) {
     if (groups == 0) return INTFA_OK;
     unsigned *ws = static_cast<unsigned *>(workspace);
     int rc = cuda_status(cudaMemsetAsync(ws, 0, static_cast<size_t>(groups) * sizeof(unsigned), stream));
@@ -229,6 +244,11 @@ int launch_quantize_per_tensor(const void *x, int64_t groups, int64_t rows, int 
     group_amax_kernel<<<dim3(chunks, static_cast<unsigned>(groups)), 256, 0, stream>>>(xv, n8, ws);
     rc = cuda_status(cudaGetLastError());
     if (rc) return rc;
+    if (global) {
+        global_amax_kernel<<<1, 256, 0, stream>>>(ws, groups);
+        rc = cuda_status(cudaGetLastError());
+        if (rc) return rc;
+    }
     if (!transpose) {
         int cb = static_cast<int>((n8 + 255) / 256);
         const int cap = static_cast<int>((148 * 16 + groups - 1) / groups);
@@ -289,6 +309,27 @@ extern "C" int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int6
         return INTFA_ERR_MISALIGNED;
     return launch_quantize_per_tensor(x_f16, groups, rows, cols, transpose, x_q, scale, workspace,
                                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int intfa_quantize_global(const void *x_f16, int64_t groups, int64_t rows, int cols, int transpose,
+                                     int8_t *x_q, float *scale, void *workspace, size_t workspace_bytes,
+                                     void *stream) {
+    using namespace intfa;
+    if (groups < 0 || rows < 0 || cols <= 0) return INTFA_ERR_INVALID_ARG;
+    if (transpose != 0 && transpose != 1) return INTFA_ERR_INVALID_ARG;
+    if (cols % 8 != 0) return INTFA_ERR_UNSUPPORTED;
+    if (transpose && cols > 256) return INTFA_ERR_UNSUPPORTED;
+    if (groups == 0 || rows == 0) return INTFA_OK;
+    if (groups > 65535) return INTFA_ERR_UNSUPPORTED;
+    if (rows > (INT64_MAX / 4) / cols / groups) return INTFA_ERR_INVALID_ARG;
+    if (!x_f16 || !x_q || !scale) return INTFA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < intfa_quantize_per_tensor_workspace_size(groups))
+        return INTFA_ERR_WORKSPACE;
+    if (!aligned16(x_f16) || !aligned16(x_q) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return INTFA_ERR_MISALIGNED;
+    return launch_quantize_per_tensor(x_f16, groups, rows, cols, transpose, x_q, scale, workspace,
+                                      static_cast<cudaStream_t>(stream), true);
 }
 
 // ------------------------------------------- per tensor, no allocation ---

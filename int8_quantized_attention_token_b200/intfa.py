@@ -47,6 +47,7 @@ def lib():
         "intfa_quantize_per_tensor_workspace_size": ([I64], SZ),
         "intfa_vt_ld": ([I64], I64),
         "intfa_quantize_per_tensor": ([P, I64, I64, I, I, P, P, P, SZ, P], I),
+        "intfa_quantize_global": ([P, I64, I64, I, I, P, P, P, SZ, P], I),
         "intfa_quantize_per_tensor_noalloc": ([P, I64, I64, I, I, P, P, P], I),
         "intfa_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
         "intfa_attention_fwd_q16": ([P, P, P, P, P, I, I, I, I, I, P, P, P], I),
@@ -144,6 +145,27 @@ def intfa_quantize_per_tensor(x: torch.Tensor, transpose: bool = False, x_q=None
     _check(lib().intfa_quantize_per_tensor(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
                                            _ptr(scale), _ptr(workspace), workspace.numel(),
                                            _stream(stream)), "intfa_quantize_per_tensor")
+    return x_q, scale
+
+
+def intfa_quantize_global(x: torch.Tensor, transpose: bool = False, x_q=None, scale=None, workspace=None,
+                          stream=None):
+    """fp16 [groups, rows, cols] -> codes with one scale over all groups (in
+    the per-group layout of intfa_quantize_per_tensor) and fp32 [groups]
+    scales, all equal."""
+    _need(x, torch.float16, "x")
+    if x.dim() != 3:
+        raise ValueError("x must be [groups, rows, cols]")
+    g, rows, cols = x.shape
+    if x_q is None:
+        shape = (g, cols, intfa_vt_ld(rows)) if transpose else (g, rows, cols)
+        x_q = torch.empty(shape, dtype=torch.int8, device=x.device)
+    scale = torch.empty((g,), dtype=torch.float32, device=x.device) if scale is None else scale
+    wsb = int(lib().intfa_quantize_per_tensor_workspace_size(g))
+    if workspace is None:
+        workspace = torch.empty((max(wsb, 1),), dtype=torch.uint8, device=x.device)
+    _check(lib().intfa_quantize_global(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q), _ptr(scale),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)), "intfa_quantize_global")
     return x_q, scale
 
 

@@ -64,6 +64,16 @@ def test_quantize_per_tensor_rejects(L):
     assert L.intfa_quantize_per_tensor(FAKE, 0, 10, 64, 0, None, None, None, 0, None) == 0
 
 
+def test_quantize_global_rejects(L):
+    ws = L.intfa_quantize_per_tensor_workspace_size(4)
+    f = L.intfa_quantize_global
+    assert f(FAKE, 4, 10, 12, 0, FAKE, FAKE, FAKE, ws, None) == 2      # cols % 8
+    assert f(FAKE, 4, 10, 64, 2, FAKE, FAKE, FAKE, ws, None) == 1      # transpose flag
+    assert f(FAKE, 4, 10, 64, 0, FAKE, FAKE, FAKE, ws - 1, None) == 6  # workspace
+    assert f(FAKE + 4, 4, 10, 64, 0, FAKE, FAKE, FAKE, ws, None) == 3
+    assert f(FAKE, 0, 10, 64, 0, None, None, None, 0, None) == 0       # nothing to do
+
+
 def test_attention_rejects(L):
     a = [FAKE] * 6
     assert L.intfa_attention_fwd(*a, 1, 1, 128, 96, 0, FAKE, None) == 2           # d
