@@ -67,6 +67,7 @@ def _load():
     lib.oracle_get_threads.restype = ctypes.c_int
     lib.oracle_quantize_per_token.argtypes = [P, I64, I64, P, P]
     lib.oracle_quantize_per_tensor.argtypes = [P, I64, I64, P, P]
+    lib.oracle_quantize_per_token_bits.argtypes = [P, I64, I64, ctypes.c_int, P, P]
     lib.oracle_qk_int32.argtypes = [P, P, I64, I64, I64, P]
     lib.oracle_attention_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
                                           ctypes.c_int, I64, I64, P, P, P, P]
@@ -109,6 +110,20 @@ def quantize_per_token(x):
     q = np.empty(x.shape, np.int8)
     s = np.empty(x.shape[:-1], np.float32)
     _load().oracle_quantize_per_token(_ptr(x), rows, d, _ptr(q), _ptr(s))
+    return q, s
+
+
+def quantize_per_token_bits(x, bits: int):
+    """x: float32 [..., d]; b-bit symmetric codes (qmax = 2^(b-1) - 1) in int8
+    and fp32 scales max|x| / qmax per row."""
+    if not 2 <= bits <= 8:
+        raise ValueError("bits in 2..8")
+    x = _c(x, np.float32)
+    d = x.shape[-1]
+    rows = x.size // d if d else 0
+    q = np.empty(x.shape, np.int8)
+    s = np.empty(x.shape[:-1], np.float32)
+    _load().oracle_quantize_per_token_bits(_ptr(x), rows, d, int(bits), _ptr(q), _ptr(s))
     return q, s
 
 

@@ -110,6 +110,35 @@ void oracle_quantize_per_token(const float *x, int64_t rows, int64_t d,
     }
 }
 
+/* Per-token with b-bit symmetric codes (the pages' INT4 remark, INT-FA
+ * abstract; eq. 3 with 127 replaced by qmax = 2^(b-1) - 1): s = max|x| / qmax
+ * (one IEEE fp32 division), codes RNE(x / s) clamped to [-qmax, qmax], stored
+ * one per int8.  b = 8 is oracle_quantize_per_token. */
+void oracle_quantize_per_token_bits(const float *x, int64_t rows, int64_t d, int bits,
+                                    int8_t *xq, float *scale) {
+    const float qmax = (float)((1 << (bits - 1)) - 1);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const float *xr = x + r * d;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < d; ++k) {
+            float a = fabsf(xr[k]);
+            if (a > amax) amax = a;
+        }
+        const float s = amax / qmax;
+        scale[r] = s;
+        for (int64_t k = 0; k < d; ++k) {
+            float c = 0.0f;
+            if (s != 0.0f) {
+                c = nearbyintf(xr[k] / s);
+                if (c > qmax) c = qmax;
+                if (c < -qmax) c = -qmax;
+            }
+            xq[r * d + k] = (int8_t)c;
+        }
+    }
+}
+
 /* Per-tensor: `groups` contiguous groups of `group_len` values, one scale
  * per group (for V: groups = B*H, group_len = L*d). */
 void oracle_quantize_per_tensor(const float *x, int64_t groups,

@@ -152,3 +152,42 @@ def test_per_tensor_one_scale_per_group(groups):
         assert s[g] == np.float32(sg)
         assert q[g].ravel().tolist() == codes
     assert s[-1] == np.float32(fl32(Fraction(9) / 127))
+
+
+# ------------------------------------------------ b-bit codes (INT4 remark) ---
+
+def test_bits8_is_the_int8_quantiser():
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((50, 128)) * 3).astype(np.float16).astype(np.float32)
+    q8, s8 = oracle.quantize_per_token(x)
+    qb, sb = oracle.quantize_per_token_bits(x, 8)
+    np.testing.assert_array_equal(q8, qb)
+    np.testing.assert_array_equal(s8.view(np.uint32), sb.view(np.uint32))
+
+
+def test_bits4_hand_table():
+    # x = [1, -0.5, 0.25, 0.07]: s = fl32(1/7) = 0.142857149... (above 1/7), so
+    # -0.5/s = -3.4999998 in fp32 (no tie) -> -3; 0.25/s = 1.7499999 -> 2;
+    # 0.07/s = 0.49 -> 0; 1/s rounds to 7
+    x = np.array([[1.0, -0.5, 0.25, 0.07, 0, 0, 0, 0]], np.float32)
+    q, s = oracle.quantize_per_token_bits(x, 4)
+    assert s[0] == np.float32(1.0) / np.float32(7.0)
+    assert list(q[0, :4]) == [7, -3, 2, 0]
+    # a genuine tie: 0.5 with s = 1/4 exactly (amax 1.75 = 7/4): 0.5/0.25 = 2.0,
+    # 0.625/0.25 = 2.5 -> 2 (even), 0.875/0.25 = 3.5 -> 4 (even)
+    y = np.array([[1.75, 0.5, 0.625, 0.875, 0, 0, 0, 0]], np.float32)
+    q, s = oracle.quantize_per_token_bits(y, 4)
+    assert s[0] == np.float32(0.25)
+    assert list(q[0, :4]) == [7, 2, 2, 4]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 6])
+def test_bits_round_trip_and_range(bits):
+    rng = np.random.default_rng(bits)
+    x = (rng.standard_normal((40, 64)) * 2).astype(np.float16).astype(np.float32)
+    q, s = oracle.quantize_per_token_bits(x, bits)
+    qmax = (1 << (bits - 1)) - 1
+    assert np.abs(q).max() <= qmax
+    assert np.all(np.abs(q).max(axis=1) == qmax)            # the arg-max row entry hits +-qmax
+    err = np.abs(x - s[:, None].astype(np.float64) * q)
+    assert np.all(err <= s[:, None] / 2 * (1 + 1e-6) + 1e-12)
