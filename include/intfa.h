@@ -85,6 +85,18 @@ int intfa_quantize_per_token(const void *x_f16, int64_t rows, int d, int8_t *x_q
  *            aligned; its contents on entry do not matter.
  * cols must be a multiple of 8 and, with transpose, at most 256.
  */
+/*
+ * Per-token quantisation with b-bit symmetric codes (the pages' remark that
+ * the token-level scheme extends to INT4; IntAttention eq. 3 with 127
+ * replaced by qmax = 2^(b-1) - 1): s = fl32(max|x| / qmax), codes
+ * clamp(RNE(x / s), -qmax, qmax) stored one per int8, so the INT8 attention
+ * entry points take them unchanged (tcgen05 has no narrower integer MMA).
+ * bits in 2..8 (8 gives intfa_quantize_per_token's codes and scales);
+ * other arguments and errors as intfa_quantize_per_token.
+ */
+int intfa_quantize_per_token_bits(const void *x_f16, int64_t rows, int d, int bits, int8_t *x_q,
+                                  float *scale, void *stream);
+
 size_t intfa_quantize_per_tensor_workspace_size(int64_t groups);
 int64_t intfa_vt_ld(int64_t rows);
 int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int64_t rows, int cols,

@@ -209,6 +209,56 @@ int grid_for(int64_t work_items, int per_block) {
 
 }  // namespace
 
+// b-bit symmetric codes, one scale per row: s = fl(max|x| / qmax) and
+// code = clamp(RNE(x / s), -qmax, qmax), both IEEE divisions (a variant for
+// narrow codes, not on the INT8 hot path).  G lanes per row of 8 G values.
+template <int G>
+__global__ void __launch_bounds__(256) quant_per_token_bits_kernel(const uint4 *__restrict__ x, int64_t rows,
+                                                                 float qmax, uint2 *__restrict__ xq,
+                                                                 float *__restrict__ scale) {
+    const int sub = threadIdx.x % G;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / G) + threadIdx.x / G;
+    const bool live = row < rows;
+    float f[8];
+    float amax = 0.0f;
+    if (live) {
+        unpack8(__ldg(x + row * G + sub), f);
+        amax = absmax8(f);
+    }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (!live) return;
+    const float s = __fdiv_rn(amax, qmax);
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        int c = 0;
+        if (s != 0.0f) c = max(-static_cast<int>(qmax), min(static_cast<int>(qmax), __float2int_rn(__fdiv_rn(f[e], s))));
+        w[e >> 2] |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * (e & 3));
+    }
+    xq[row * G + sub] = make_uint2(w[0], w[1]);
+    if (sub == 0) scale[row] = s;
+}
+
+int launch_quantize_per_token_bits(const void *x, int64_t rows, int d, int bits, int8_t *xq, float *scale,
+                                   cudaStream_t stream) {
+    if (rows == 0) return INTFA_OK;
+    const uint4 *xv = static_cast<const uint4 *>(x);
+    uint2 *qv = reinterpret_cast<uint2 *>(xq);
+    const float qmax = static_cast<float>((1 << (bits - 1)) - 1);
+    const int grid = grid_for(rows, 256 / (d / 8));
+    switch (d) {
+        case 8: quant_per_token_bits_kernel<1><<<grid, 256, 0, stream>>>(xv, rows, qmax, qv, scale); break;
+        case 16: quant_per_token_bits_kernel<2><<<grid, 256, 0, stream>>>(xv, rows, qmax, qv, scale); break;
+        case 32: quant_per_token_bits_kernel<4><<<grid, 256, 0, stream>>>(xv, rows, qmax, qv, scale); break;
+        case 64: quant_per_token_bits_kernel<8><<<grid, 256, 0, stream>>>(xv, rows, qmax, qv, scale); break;
+        case 128: quant_per_token_bits_kernel<16><<<grid, 256, 0, stream>>>(xv, rows, qmax, qv, scale); break;
+        case 256: quant_per_token_bits_kernel<32><<<grid, 256, 0, stream>>>(xv, rows, qmax, qv, scale); break;
+        default: return INTFA_ERR_UNSUPPORTED;
+    }
+    return cuda_status(cudaGetLastError());
+}
+
 int launch_quantize_per_token(const void *x, int64_t rows, int d, int8_t *xq, float *scale,
                               cudaStream_t stream) {
     if (rows == 0) return INTFA_OK;
@@ -281,6 +331,19 @@ extern "C" int intfa_quantize_per_token(const void *x_f16, int64_t rows, int d, 
         return INTFA_ERR_MISALIGNED;
     if (d >= 16 && !aligned16(x_q)) return INTFA_ERR_MISALIGNED;
     return launch_quantize_per_token(x_f16, rows, d, x_q, scale, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int intfa_quantize_per_token_bits(const void *x_f16, int64_t rows, int d, int bits, int8_t *x_q,
+                                             float *scale, void *stream) {
+    using namespace intfa;
+    if (rows < 0 || bits < 2 || bits > 8) return INTFA_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_f16 || !x_q || !scale)) return INTFA_ERR_INVALID_ARG;
+    if (!(d == 8 || d == 16 || d == 32 || d == 64 || d == 128 || d == 256)) return INTFA_ERR_UNSUPPORTED;
+    if (rows > (INT64_MAX / 2) / d) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(x_f16) || (reinterpret_cast<uintptr_t>(x_q) & 7u) != 0 ||
+        (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return INTFA_ERR_MISALIGNED;
+    return launch_quantize_per_token_bits(x_f16, rows, d, bits, x_q, scale, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" size_t intfa_quantize_per_tensor_workspace_size(int64_t groups) {

@@ -44,6 +44,7 @@ def lib():
     sig = {
         "intfa_status_string": ([I], ctypes.c_char_p),
         "intfa_quantize_per_token": ([P, I64, I, P, P, P], I),
+        "intfa_quantize_per_token_bits": ([P, I64, I, I, P, P, P], I),
         "intfa_quantize_per_tensor_workspace_size": ([I64], SZ),
         "intfa_vt_ld": ([I64], I64),
         "intfa_quantize_per_tensor": ([P, I64, I64, I, I, P, P, P, SZ, P], I),
@@ -122,6 +123,18 @@ def intfa_quantize_per_token(x: torch.Tensor, x_q=None, scale=None, stream=None)
     scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if scale is None else scale
     _check(lib().intfa_quantize_per_token(_ptr(x), rows, d, _ptr(x_q), _ptr(scale), _stream(stream)),
            "intfa_quantize_per_token")
+    return x_q, scale
+
+
+def intfa_quantize_per_token_bits(x: torch.Tensor, bits: int, x_q=None, scale=None, stream=None):
+    """fp16 [..., d] -> b-bit codes (in int8, |code| <= 2^(bits-1) - 1) and fp32 [...] scales."""
+    _need(x, torch.float16, "x")
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    x_q = torch.empty(x.shape, dtype=torch.int8, device=x.device) if x_q is None else x_q
+    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if scale is None else scale
+    _check(lib().intfa_quantize_per_token_bits(_ptr(x), rows, d, int(bits), _ptr(x_q), _ptr(scale), _stream(stream)),
+           "intfa_quantize_per_token_bits")
     return x_q, scale
 
 

@@ -64,6 +64,15 @@ def test_quantize_per_tensor_rejects(L):
     assert L.intfa_quantize_per_tensor(FAKE, 0, 10, 64, 0, None, None, None, 0, None) == 0
 
 
+def test_quantize_bits_rejects(L):
+    f = L.intfa_quantize_per_token_bits
+    assert f(FAKE, 10, 64, 1, FAKE, FAKE, None) == 1      # bits
+    assert f(FAKE, 10, 64, 9, FAKE, FAKE, None) == 1
+    assert f(FAKE, 10, 96, 4, FAKE, FAKE, None) == 2      # d
+    assert f(FAKE + 4, 10, 64, 4, FAKE, FAKE, None) == 3
+    assert f(FAKE, 0, 64, 4, None, None, None) == 0
+
+
 def test_quantize_global_rejects(L):
     ws = L.intfa_quantize_per_tensor_workspace_size(4)
     f = L.intfa_quantize_global
