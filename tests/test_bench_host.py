@@ -61,3 +61,31 @@ def test_reference_arm_json_line():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                         "--warmup", "3"], capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_variant_argument_checks():
+    for extra in (["--method", "index", "--scale-block", "128"], ["--method", "decode", "--lsum", "codes"],
+                  ["--q-path", "fused", "--scale-block", "64"], ["--scale-block", "64", "--lsum", "codes"],
+                  ["--warmup", "2"]):
+        r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *extra], capture_output=True,
+                           text=True, timeout=120, cwd=ROOT)
+        assert r.returncode != 0, extra
+
+
+def test_kernel_hashes_per_method():
+    sys.path.insert(0, ROOT)
+    import bench
+    hashes = {m: bench.kernel_sources_sha(m) for m in ("online", "index", "decode")}
+    assert len(set(hashes.values())) == 3
+    assert all(len(h) == 16 and int(h, 16) >= 0 for h in hashes.values())
+
+
+def test_cpu_baseline_variants_run_the_oracle():
+    sys.path.insert(0, ROOT)
+    import bench
+    from int8_quantized_attention_token_b200.workloads import by_name
+    w = by_name("attn_B1_H1_L128_d64")
+    for kw, word in (({}, "online"), ({"method": "index"}, "IndexSoftmax"), ({"blk": 64}, "block"),
+                     ({"lcodes": True}, "online")):
+        r = bench.cpu_baseline(w, budget_s=0.2, **kw)
+        assert r["kind"] == "oracle" and r["value"] > 0 and word in r["sample"]
