@@ -19,7 +19,8 @@ and marshals numpy arrays.  Each function cites the passage it follows:
 * ``attention_online_rows`` -- the same steps in FlashAttention's block-wise
   online order (INT-FlashAttention abstract; FlashAttention-3 abstract): P
   codes against the running max of the key blocks seen so far.  This is the
-  form the fused kernel computes.
+  form the fused kernel computes.  ``p_levels=255`` stores P as UINT8
+  (RNE(255 p)), the unsigned scheme of IntAttention's Table 5 ablation.
 * ``attention_fp64_rows`` -- IntAttention section 2.1, eq. 1.
 * ``decode`` -- one query against a key / value cache: the online form of
   ``attention_online_rows`` run separately on consecutive key ranges
@@ -72,7 +73,7 @@ def _load():
     lib.oracle_attention_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
                                           ctypes.c_int, I64, I64, P, P, P, P]
     lib.oracle_attention_online_rows.argtypes = [P, P, P, P, P, ctypes.c_float, I64, I64,
-                                                 ctypes.c_int, I64, I64, I64, P, P, ctypes.c_int]
+                                                 ctypes.c_int, I64, I64, I64, P, P, ctypes.c_int, ctypes.c_int]
     lib.oracle_attention_fp64_rows.argtypes = [P, P, P, I64, I64, ctypes.c_int, I64, I64, P]
     lib.oracle_decode.argtypes = [P, ctypes.c_float, P, P, P, ctypes.c_float, I64, I64, I64, I64, P]
     lib.oracle_index_lut.argtypes = [ctypes.c_double, ctypes.c_int, P]
@@ -177,11 +178,16 @@ def attention_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, r0: int = 0, r1=
 
 
 def attention_online_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, block: int = 128,
-                          r0: int = 0, r1=None, want_l: bool = False, lsum_codes: bool = False):
+                          r0: int = 0, r1=None, want_l: bool = False, lsum_codes: bool = False,
+                          p_levels: int = 127):
     """One head, block-wise online form (FlashAttention's forward workflow):
     P codes against the running max over key blocks of ``block``.  Returns O
     fp64 [r1 - r0, d] (and the row sums l with want_l).  lsum_codes: the row
-    sum from the P codes (sum P_hat / 127) instead of the unquantised p."""
+    sum from the P codes (sum P_hat / p_levels) instead of the unquantised p.
+    p_levels: 127 (P codes RNE(127 p), INT8) or 255 (RNE(255 p), UINT8 --
+    IntAttention Table 5's unsigned scheme)."""
+    if p_levels not in (127, 255):
+        raise ValueError("p_levels must be 127 or 255")
     Qq = _c(Qq, np.int8)
     Kq = _c(Kq, np.int8)
     Vq = _c(Vq, np.int8)
@@ -193,7 +199,7 @@ def attention_online_rows(Qq, Kq, Vq, sQ, sK, sV: float, causal: bool, block: in
     l = np.empty((r1 - r0,), np.float64) if want_l else None
     _load().oracle_attention_online_rows(_ptr(Qq), _ptr(Kq), _ptr(Vq), _ptr(sQ), _ptr(sK),
                                          float(sV), L, d, int(bool(causal)), int(block),
-                                         r0, r1, _ptr(O), _ptr(l), int(bool(lsum_codes)))
+                                         r0, r1, _ptr(O), _ptr(l), int(bool(lsum_codes)), int(p_levels))
     return (O, l) if want_l else O
 
 

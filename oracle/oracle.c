@@ -250,11 +250,16 @@ void oracle_attention_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
  * lsum_codes != 0 takes the other reading of the row sum: l from the P codes,
  * l = alpha l + sum_j codes_ij / 127 (IntAttention section 3.2 quantises P
  * before the value product; the pages do not say which p the sum uses).
+ * p_levels is the largest P code: 127 (P stored as INT8, the INT-FlashAttention
+ * pipeline) or 255 (P stored as UINT8, codes RNE(255 p), the scheme that
+ * IntAttention's Table 5 ablation favours); 127 above stands for p_levels.
  */
 void oracle_attention_online_rows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq,
                                   const float *sQ, const float *sK, float sV,
                                   int64_t L, int64_t d, int causal, int64_t block,
-                                  int64_t r0, int64_t r1, double *O, double *l_out, int lsum_codes) {
+                                  int64_t r0, int64_t r1, double *O, double *l_out, int lsum_codes,
+                                  int p_levels) {
+    const double levels = (double)p_levels;
     const double inv_sqrt_d = 1.0 / sqrt((double)d);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t i = r0; i < r1; ++i) {
@@ -278,8 +283,8 @@ void oracle_attention_online_rows(const int8_t *Qq, const int8_t *Kq, const int8
             for (int64_t c = 0; c < d; ++c) blk[c] = 0;
             for (int64_t jj = 0; jj < nb; ++jj) {
                 double p = exp(t[jj] - m_new);
-                int64_t code = (int64_t)nearbyint(127.0 * p);
-                psum += lsum_codes ? (double)code / 127.0 : p;
+                int64_t code = (int64_t)nearbyint(levels * p);
+                psum += lsum_codes ? (double)code / levels : p;
                 const int8_t *v = Vq + (j0 + jj) * d;
                 for (int64_t c = 0; c < d; ++c) blk[c] += code * (int64_t)v[c];
             }
@@ -288,7 +293,7 @@ void oracle_attention_online_rows(const int8_t *Qq, const int8_t *Kq, const int8
             m = m_new;
         }
         double *o = O + (i - r0) * d;
-        for (int64_t c = 0; c < d; ++c) o[c] = (double)sV * acc[c] / (127.0 * l);
+        for (int64_t c = 0; c < d; ++c) o[c] = (double)sV * acc[c] / (levels * l);
         if (l_out) l_out[i - r0] = l;
         free(t);
         free(acc);

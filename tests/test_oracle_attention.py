@@ -309,3 +309,107 @@ def test_codesum_one_block_is_the_code_weighted_mean():
     O = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, sV, False, 128, lsum_codes=True)
     want = sV * (P.astype(np.float64) @ Vq.astype(np.float64)) / P.sum(axis=1, keepdims=True)
     np.testing.assert_allclose(O, want, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------- UINT8 P codes, RNE(255 p) (Table 5 scheme) ---
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("lsum_codes", [False, True])
+def test_uint8_p_constant_logits_give_mean_of_values(causal, lsum_codes):
+    # Q_hat = 0: every p is 1, every code 255; O is the mean of the visible V_hat
+    rng = np.random.default_rng(31)
+    L, d = 260, 64
+    Qq = np.zeros((L, d), np.int8)
+    Kq, Vq = rand_i8(rng, L, d), rand_i8(rng, L, d)
+    s = rng.uniform(0.01, 0.1, L).astype(np.float32)
+    O = oracle.attention_online_rows(Qq, Kq, Vq, s, s, 0.25, causal, 128, lsum_codes=lsum_codes,
+                                     p_levels=255)
+    for i in range(L):
+        n = i + 1 if causal else L
+        np.testing.assert_allclose(O[i], 0.25 * Vq[:n].astype(np.float64).mean(0), rtol=1e-13, atol=1e-15)
+
+
+def test_uint8_p_hand_built_two_blocks():
+    # the two-block example with 255 levels: codes RNE(255 e^(t - m)) against
+    # the running max (1, then 3), acc and l rescaled by e^(1 - 3)
+    d = 64
+    a, b = 64, [0, 1, 3, 2]                 # t_j = a b_j sQ sK / 8 = b_j
+    L = len(b)
+    Qq = np.zeros((L, d), np.int8)
+    Qq[0, 0] = a
+    Kq = np.zeros((L, d), np.int8)
+    Kq[:, 0] = b
+    sQ = np.full(L, 0.125, np.float32)
+    sK = np.full(L, 1.0, np.float32)
+    rng = np.random.default_rng(32)
+    Vq = rand_i8(rng, L, d)
+    c1 = [round(255 * math.exp(t - 1)) for t in (0, 1)]     # [94, 255]
+    c2 = [round(255 * math.exp(t - 3)) for t in (3, 2)]     # [255, 94]
+    assert c1 == [94, 255] and c2 == [255, 94]
+    alpha = math.exp(1 - 3)
+    acc = [alpha * (c1[0] * int(Vq[0, c]) + c1[1] * int(Vq[1, c])) + (c2[0] * int(Vq[2, c]) + c2[1] * int(Vq[3, c]))
+           for c in range(d)]
+    for lsum_codes in (False, True):
+        O, l = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, 0.5, False, block=2, r0=0, r1=1,
+                                            want_l=True, lsum_codes=lsum_codes, p_levels=255)
+        if lsum_codes:
+            lw = alpha * (94 + 255) / 255 + (255 + 94) / 255
+        else:
+            lw = alpha * (math.exp(-1) + 1) + (1 + math.exp(-1))
+        assert l[0] == pytest.approx(lw, rel=1e-15)
+        np.testing.assert_allclose(O[0], [0.5 * x / (255 * lw) for x in acc], rtol=1e-13)
+
+
+def test_uint8_p_codes_use_the_full_byte():
+    # one key block, logits spread over [-6, 0]: RNE(255 p) reaches 255 at the
+    # row max and the code-weighted mean with the codes recomputed from the
+    # logits by hand (t_j = a b_j sQ sK / sqrt(d) with S_0j = a b_j)
+    d = 128
+    a = 127
+    b = list(range(-127, 1, 8))             # 16 keys
+    L = len(b)
+    Qq = np.zeros((L, d), np.int8)
+    Qq[0, 0] = a
+    Kq = np.zeros((L, d), np.int8)
+    Kq[:, 0] = b
+    sQ = np.full(L, 0.0625, np.float32)
+    sK = np.full(L, 0.0625, np.float32)
+    rng = np.random.default_rng(33)
+    Vq = rand_i8(rng, L, d)
+    t = [a * bj * 0.0625 * 0.0625 / math.sqrt(d) for bj in b]
+    mx = max(t)
+    codes = [round(255 * math.exp(tj - mx)) for tj in t]
+    assert max(codes) == 255 and min(codes) < 127
+    O = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, 0.5, False, 128, r0=0, r1=1, lsum_codes=True,
+                                     p_levels=255)
+    want = [0.5 * sum(codes[j] * int(Vq[j, c]) for j in range(L)) / sum(codes) for c in range(d)]
+    np.testing.assert_allclose(O[0], want, rtol=1e-13)
+
+
+def test_uint8_p_rejects_other_levels():
+    Qq = np.zeros((4, 64), np.int8)
+    s = np.ones(4, np.float32)
+    with pytest.raises(ValueError):
+        oracle.attention_online_rows(Qq, Qq, Qq, s, s, 1.0, False, p_levels=128)
+
+
+def test_uint8_p_error_below_int8_p():
+    # IntAttention Table 5: UINT8 P (range [0, 1] over all 256 codes) keeps
+    # attention closer to full precision than signed INT8 P (half the codes).
+    # Same quantised Q / K / V, online form, against fp64 attention of the
+    # unquantised inputs: cosine similarity higher and RMSE lower.
+    rng = np.random.default_rng(34)
+    L, d = 512, 64
+    q, k, v = (rng.standard_normal((L, d)).astype(np.float32) for _ in range(3))
+    Qq, sQ = oracle.quantize_per_token(q)
+    Kq, sK = oracle.quantize_per_token(k)
+    Vq, sV = oracle.quantize_per_tensor(v, 1)
+    ref = oracle.attention_fp64_rows(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64), True)
+    stats = {}
+    for lv in (127, 255):
+        O = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), True, 128, p_levels=lv)
+        cos = (O * ref).sum() / math.sqrt((O * O).sum() * (ref * ref).sum())
+        rmse = math.sqrt(((O - ref) ** 2).mean())
+        stats[lv] = (cos, rmse)
+    assert stats[255][0] > stats[127][0]
+    assert stats[255][1] < stats[127][1]
