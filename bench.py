@@ -240,6 +240,10 @@ def run_gpu(args):
         if fused_q:   # Q quantised per token inside the attention kernel
             intfa.intfa_attention_fwd_q16(Q, Kq, Vt.reshape(B, H, d, ld), sK, sV.reshape(B, H), w.causal, O,
                                           s_Q=sQ, stream=stream)
+        elif args.p_levels != 127:   # UINT8 P codes RNE(255 p)
+            intfa.intfa_attention_fwd_pcodes(Qq, Kq, Vt.reshape(B, H, d, ld), sQ, sK, sV.reshape(B, H), w.causal,
+                                             p_levels=args.p_levels, lsum_codes=args.lsum == "codes", O=O,
+                                             stream=stream)
         elif args.lsum == "codes":   # row sum from the P codes
             intfa.intfa_attention_fwd_codesum(Qq, Kq, Vt.reshape(B, H, d, ld), sQ, sK, sV.reshape(B, H), w.causal,
                                               O, stream=stream)
@@ -353,7 +357,8 @@ def run_gpu(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, budget_s=args.cpu_seconds, method=args.method,
-                           c=args.index_c, b=args.index_b, blk=blk, lcodes=args.lsum == "codes")
+                           c=args.index_c, b=args.index_b, blk=blk, lcodes=args.lsum == "codes",
+                           p_levels=args.p_levels)
 
     if rank == 0:
         line = {
@@ -366,6 +371,7 @@ def run_gpu(args):
                        "method": args.method,
                        **({"scale_block": blk} if blk > 1 else {}),
                        **({"lsum": "codes"} if args.lsum == "codes" else {}),
+                       **({"p_levels": args.p_levels} if args.p_levels != 127 else {}),
                        **({"index_c": args.index_c, "index_b": args.index_b} if index else {})},
             "pct_of_int8_peak": round(100.0 * value / world / peak, 2),
             "roofline": {"bound": "tensor",
@@ -529,7 +535,7 @@ def run_decode(args):
 
 # --------------------------------------------------------------- CPU arm ---
 
-def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5, blk=1, lcodes=False):
+def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5, blk=1, lcodes=False, p_levels=127):
     """Run the oracle's whole path (quantise, block-wise online attention; or
     for method "index" per-tensor quantisation and IndexSoftmax attention) on
     `heads` full (b, h) heads of the workload; returns (seconds, ops, cores)."""
@@ -561,17 +567,19 @@ def oracle_sample(w, heads, threads=None, method="online", c=6.6, b=5, blk=1, lc
             Qq, sQ = oracle.quantize_per_token(q)
             Kq, sK = oracle.quantize_per_token(k)
             Vq, sV = oracle.quantize_per_tensor(v, 1)
-            oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), w.causal, 128, lsum_codes=lcodes)
+            oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]), w.causal, 128, lsum_codes=lcodes,
+                                         p_levels=p_levels)
         t += time.perf_counter() - t0
     ops = w.ops / (w.B * w.H) * len(heads)
     return t, ops, oracle.get_threads()
 
 
-def cpu_baseline(w, budget_s=15.0, method="online", c=6.6, b=5, blk=1, lcodes=False):
-    t1, ops1, cores = oracle_sample(w, [(0, 0)], method=method, c=c, b=b, blk=blk, lcodes=lcodes)
+def cpu_baseline(w, budget_s=15.0, method="online", c=6.6, b=5, blk=1, lcodes=False, p_levels=127):
+    t1, ops1, cores = oracle_sample(w, [(0, 0)], method=method, c=c, b=b, blk=blk, lcodes=lcodes,
+                                    p_levels=p_levels)
     n = max(1, min(w.B * w.H - 1, int(budget_s / max(t1, 1e-3)) - 1))
     heads = [((i + 1) // w.H % w.B, (i + 1) % w.H) for i in range(n)]
-    t, ops, cores = oracle_sample(w, heads, method=method, c=c, b=b, blk=blk, lcodes=lcodes)
+    t, ops, cores = oracle_sample(w, heads, method=method, c=c, b=b, blk=blk, lcodes=lcodes, p_levels=p_levels)
     t += t1
     ops += ops1
     what = ("per-tensor quantise + IndexSoftmax attention" if method == "index" else
@@ -661,6 +669,8 @@ def main():
     ap.add_argument("--index-b", type=int, default=5, help="IndexSoftmax table bits b")
     ap.add_argument("--lsum", default="p", choices=["p", "codes"],
                     help="online method: row sum from the unquantised p (default) or from the P codes")
+    ap.add_argument("--p-levels", type=int, default=127, choices=[127, 255],
+                    help="online method: P codes RNE(127 p) as INT8 (default) or RNE(255 p) as UINT8")
     ap.add_argument("--scale-block", type=int, default=1,
                     help="online method: one Q / K scale per block of this many tokens (1 = per token)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -670,10 +680,11 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl != "reference":
         raise SystemExit("--warmup must be >= 3")
-    if (args.scale_block != 1 or args.lsum != "p") and (args.method != "online" or args.q_path != "separate"):
-        raise SystemExit("--scale-block / --lsum apply to the online method with the separate Q pass")
-    if args.scale_block != 1 and args.lsum != "p":
-        raise SystemExit("--scale-block and --lsum codes are separate variants")
+    if (args.scale_block != 1 or args.lsum != "p" or args.p_levels != 127) and \
+            (args.method != "online" or args.q_path != "separate"):
+        raise SystemExit("--scale-block / --lsum / --p-levels apply to the online method with the separate Q pass")
+    if args.scale_block != 1 and (args.lsum != "p" or args.p_levels != 127):
+        raise SystemExit("--scale-block and --lsum codes / --p-levels 255 are separate variants")
     if args.impl == "reference":
         run_reference(args)
     elif args.method == "decode":

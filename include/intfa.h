@@ -198,6 +198,30 @@ int intfa_attention_fwd_codesum(const int8_t *Q_q, const int8_t *K_q, const int8
                                 int L, int d, int causal, void *O_f16, void *stream);
 
 /*
+ * The fused attention of intfa_attention_fwd with the P-code range and the
+ * row-sum reading chosen by the caller.
+ *
+ *   p_levels   : 127 -- P_hat = RNE(127 p) stored as INT8 (IntAttention
+ *                section 3.2, the INT-FlashAttention pipeline; the codes of
+ *                intfa_attention_fwd);
+ *                255 -- P_hat = RNE(255 p) stored as UINT8 and multiplied as
+ *                unsigned tensor-core operands (the unsigned scheme of
+ *                IntAttention's Table 5 ablation, which spends all 256 codes
+ *                on p in [0, 1]).  O = s_V (P_hat V_hat) / (p_levels l).
+ *   lsum_codes : 0 -- l from the unquantised p (as intfa_attention_fwd);
+ *                1 -- l from the codes, sum P_hat / p_levels (as
+ *                intfa_attention_fwd_codesum when p_levels = 127).
+ *   Other arguments, layouts and error behaviour as intfa_attention_fwd;
+ *   INTFA_ERR_INVALID_ARG for any other p_levels or lsum_codes.
+ *   (127, 0) and (127, 1) give output bit-identical to intfa_attention_fwd
+ *   and intfa_attention_fwd_codesum.
+ */
+int intfa_attention_fwd_pcodes(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                               const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                               int L, int d, int causal, int p_levels, int lsum_codes, void *O_f16,
+                               void *stream);
+
+/*
  * The fused attention of intfa_attention_fwd with group-wise Q and K scales
  * (IntAttention section 3.3: per-block quantisation; the scales of each
  * group factor out of Q_hat K_hat^T exactly as per-token scales do): one scale

@@ -368,7 +368,11 @@ __device__ __forceinline__ void exp_codes(const uint32_t (&w)[32], uint64_t c2, 
 // Otherwise Q_hat arrives through tmQ and s_Q through sQ.
 // kLCodes: the row sum from the P codes, l = alpha l + sum_j P_hat_ij / 127,
 // instead of the unquantised p (the other reading of the pages).
-template <int D, bool kQ16, bool kLCodes = false>
+// kU8P: P codes RNE(255 p) stored as UINT8 and multiplied as unsigned A
+// operands (IntAttention Table 5's unsigned scheme; |P V| per block <=
+// 255 * 127 * 128 < 2^22 keeps the biased accumulator exact); 127 becomes 255
+// in the code rounding, the code sum and the epilogue.
+template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
@@ -377,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint4 *__restrict__ Qh, float *__restrict__ sQ_out, int sshift) {
     AttnSmem<D, kQ16> &sm = get_smem<D, kQ16>();
     constexpr int NS = AttnSmem<D, kQ16>::NS;
+    constexpr float kLevels = kU8P ? 255.0f : 127.0f;   // largest P code
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     // Role numbering: the producer / MMA warpgroup (roles 12-15) runs on the
@@ -512,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kSwQK = (D == 128) ? kSwizzle128B : kSwizzle64B;
         constexpr uint32_t kSboQK = 8 * D;      // 8 rows of D bytes
         const uint32_t idesc_qk = make_idesc_i8(BM, BN);
-        const uint32_t idesc_pv = make_idesc_i8(BM, D);
+        const uint32_t idesc_pv = kU8P ? make_idesc_u8s8(BM, D) : make_idesc_i8(BM, D);
         // bias MMA operands: every element of A and B is the same constant, so
         // the descriptors may let core matrices overlap (16-byte strides keep
         // all reads inside the 384-byte arrays)
@@ -659,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ws = warp >> 2, quad = warp & 3;
         const int row = 32 * quad + lane;
         const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
-        const uint64_t k127 = f2_pack(127.0f, 127.0f), magic = f2_pack(kMagic, kMagic);
+        const uint64_t k127 = f2_pack(kLevels, kLevels), magic = f2_pack(kMagic, kMagic);
         bool ok = true;
         int g = 0;
         Ring<SB> sb;
@@ -767,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 float bsum;
                 if constexpr (kLCodes) {
-                    bsum = static_cast<float>(csum) * (1.0f / 127.0f);
+                    bsum = static_cast<float>(csum) * (1.0f / kLevels);
                 } else {
                     float ps0, ps1, ps2, ps3;
                     f2_unpack(ps01, ps0, ps1);
@@ -854,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float l = sm.lsum[ls][0][row] * ex2(cm0 - cmf) + sm.lsum[ls][1][row] * ex2(cm1 - cmf);
             mbar_arrive(&sm.l_empty[ls]);
             if (qi < L) {
-                const float f = s_v / (127.0f * l);
+                const float f = s_v / (kLevels * l);
                 uint4 *dst = reinterpret_cast<uint4 *>(O + (static_cast<int64_t>(T.bh) * L + qi) * D);
 #pragma unroll
                 for (int c8 = 0; c8 < D / 8; ++c8) {
@@ -979,7 +984,7 @@ unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
 }
 
 // Qq (int8, with sQ) when !kQ16; Qh (fp16, scales optionally to sQ_out) when kQ16.
-template <int D, bool kQ16, bool kLCodes = false>
+template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false>
 int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                 float *sQ_out, const float *sK, const float *sV, int B, int H, int L, int causal,
                 void *O, cudaStream_t stream, int sshift = 0) {
@@ -999,13 +1004,13 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     const size_t smem = attn_smem_bytes<D, kQ16>();
-    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D, kQ16, kLCodes>,
+    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D, kQ16, kLCodes, kU8P>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
     if (rc) return rc;
     // The in-kernel register split assumes exactly kLaunchRegs per thread at
     // launch; a different count could leave setmaxnreg.inc waiting forever.
     cudaFuncAttributes fa;
-    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kQ16, kLCodes>));
+    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kQ16, kLCodes, kU8P>));
     if (rc) return rc;
     if (fa.numRegs != kLaunchRegs) return INTFA_ERR_UNSUPPORTED;
     const int ntiles = (L + BM - 1) / BM;
@@ -1014,7 +1019,7 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
     if (!rc) rc = cuda_status(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
     if (rc) return rc;
     const unsigned grid = persistent_grid(static_cast<int64_t>(BH) * ntiles, ntiles, causal, nsm);
-    attn_fwd_kernel<D, kQ16, kLCodes><<<grid, kThreads, smem, stream>>>(
+    attn_fwd_kernel<D, kQ16, kLCodes, kU8P><<<grid, kThreads, smem, stream>>>(
         mq, mk, mv, sQ, sK, sV, static_cast<__half *>(O), BH, L, causal, static_cast<const uint4 *>(Qh),
         sQ_out, sshift);
     return cuda_status(cudaGetLastError());
@@ -1131,6 +1136,42 @@ extern "C" int intfa_attention_fwd_codesum(const int8_t *Q_q, const int8_t *K_q,
         return launch_attn<128, false, true>(Q_q, nullptr, K_q, Vt_q, s_Q, nullptr, s_K, s_V, B, H, L, causal,
                                              O_f16, s);
     return launch_attn<64, false, true>(Q_q, nullptr, K_q, Vt_q, s_Q, nullptr, s_K, s_V, B, H, L, causal, O_f16, s);
+}
+
+extern "C" int intfa_attention_fwd_pcodes(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                          const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                                          int L, int d, int causal, int p_levels, int lsum_codes, void *O_f16,
+                                          void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    if ((p_levels != 127 && p_levels != 255) || (lsum_codes != 0 && lsum_codes != 1)) return INTFA_ERR_INVALID_ARG;
+    if (!Q_q || !K_q || !Vt_q || !s_Q || !s_K || !s_V || !O_f16) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(Vt_q) || !aligned16(O_f16) ||
+        (reinterpret_cast<uintptr_t>(s_Q) & 3u) || (reinterpret_cast<uintptr_t>(s_K) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_V) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+#define INTFA_PCODES_LAUNCH(DD, LC, U8)                                                                      \
+    return launch_attn<DD, false, LC, U8>(Q_q, nullptr, K_q, Vt_q, s_Q, nullptr, s_K, s_V, B, H, L, causal, \
+                                          O_f16, s)
+    const bool u8 = p_levels == 255;
+    if (d == 128) {
+        if (u8) {
+            if (lsum_codes) INTFA_PCODES_LAUNCH(128, true, true);
+            INTFA_PCODES_LAUNCH(128, false, true);
+        }
+        if (lsum_codes) INTFA_PCODES_LAUNCH(128, true, false);
+        INTFA_PCODES_LAUNCH(128, false, false);
+    }
+    if (u8) {
+        if (lsum_codes) INTFA_PCODES_LAUNCH(64, true, true);
+        INTFA_PCODES_LAUNCH(64, false, true);
+    }
+    if (lsum_codes) INTFA_PCODES_LAUNCH(64, true, false);
+    INTFA_PCODES_LAUNCH(64, false, false);
+#undef INTFA_PCODES_LAUNCH
 }
 
 extern "C" int intfa_attention_fwd_q16(const void *Q_f16, const int8_t *K_q, const int8_t *Vt_q,

@@ -54,6 +54,7 @@ def lib():
         "intfa_attention_fwd_q16": ([P, P, P, P, P, I, I, I, I, I, P, P, P], I),
         "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
         "intfa_attention_fwd_codesum": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
+        "intfa_attention_fwd_pcodes": ([P, P, P, P, P, P, I, I, I, I, I, I, I, P, P], I),
         "intfa_attention_fwd_blockscale": ([P, P, P, P, P, P, I, I, I, I, I, I, P, P], I),
         "intfa_decode_workspace_size": ([I, I, I, I], SZ),
         "intfa_decode_fwd": ([P, P, P, P, P, I, I, I, I, I, P, P, SZ, P], I),
@@ -230,6 +231,23 @@ def intfa_attention_fwd_codesum(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, O=N
     _check(lib().intfa_attention_fwd_codesum(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
                                              B, H, L, d, int(bool(causal)), _ptr(O), _stream(stream)),
            "intfa_attention_fwd_codesum")
+    return O
+
+
+def intfa_attention_fwd_pcodes(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, p_levels: int = 255,
+                               lsum_codes: bool = False, O=None, stream=None):
+    """intfa_attention_fwd with P codes RNE(p_levels p): 127 (INT8 P) or 255
+    (UINT8 P); lsum_codes takes the row sum from the codes (sum P_hat / p_levels)."""
+    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
+        _need(t, torch.int8, n)
+    for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
+        _need(t, torch.float32, n)
+    B, H, L, d = Q_q.shape
+    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
+    _check(lib().intfa_attention_fwd_pcodes(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
+                                            B, H, L, d, int(bool(causal)), int(p_levels), int(bool(lsum_codes)),
+                                            _ptr(O), _stream(stream)),
+           "intfa_attention_fwd_pcodes")
     return O
 
 

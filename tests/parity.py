@@ -6,10 +6,12 @@ import torch
 import oracle
 
 
-def oracle_heads(Q, K, V, causal, heads, rows=None, two_pass=False, fp64=False, block=128):
+def oracle_heads(Q, K, V, causal, heads, rows=None, two_pass=False, fp64=False, block=128,
+                 p_levels=127, lsum_codes=False):
     """Q, K, V: fp16 CPU [B, H, L, d].  For each (b, h) in heads, quantise that
-    head with the oracle and run the online form (and optionally the two-pass
-    form and unquantised fp64 attention) on `rows` (all rows if None).
+    head with the oracle and run the online form (P codes RNE(p_levels p),
+    row sum from the codes with lsum_codes; optionally also the two-pass form
+    and unquantised fp64 attention) on `rows` (all rows if None).
     Returns {(b, h): dict(rows=..., O=..., O2=..., Ox=...)}."""
     out = {}
     L = Q.shape[2]
@@ -34,7 +36,8 @@ def oracle_heads(Q, K, V, causal, heads, rows=None, two_pass=False, fp64=False, 
                 stop += 1
             r0, r1 = int(rr[start]), int(rr[stop - 1]) + 1
             res["O"][start:stop] = oracle.attention_online_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]),
-                                                                causal, block, r0, r1)
+                                                                causal, block, r0, r1,
+                                                                lsum_codes=lsum_codes, p_levels=p_levels)
             if two_pass:
                 res["O2"][start:stop] = oracle.attention_rows(Qq, Kq, Vq, sQ, sK, float(sV[0]),
                                                               causal, r0, r1)

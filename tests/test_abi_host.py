@@ -115,6 +115,19 @@ def test_codesum_attention_rejects(L):
     assert f(*a, 1, 1, 128, 64, 0, FAKE + 8, None) == 3
 
 
+def test_pcodes_attention_rejects(L):
+    a = [FAKE] * 6
+    f = L.intfa_attention_fwd_pcodes
+    assert f(*a, 1, 1, 128, 64, 0, 128, 0, FAKE, None) == 1     # p_levels not 127 / 255
+    assert f(*a, 1, 1, 128, 64, 0, 0, 0, FAKE, None) == 1
+    assert f(*a, 1, 1, 128, 64, 0, 255, 2, FAKE, None) == 1     # lsum_codes flag
+    assert f(*a, 1, 1, 128, 96, 0, 255, 0, FAKE, None) == 2     # d
+    assert f(*a, 1, 1, 128, 64, 2, 255, 0, FAKE, None) == 1     # causal flag
+    assert f(*a, 1, 1, 128, 64, 0, 255, 0, None, None) == 1     # O
+    assert f(None, *a[1:], 1, 1, 128, 64, 0, 255, 0, FAKE, None) == 1
+    assert f(FAKE + 4, *a[1:], 1, 1, 128, 64, 0, 255, 0, FAKE, None) == 3
+
+
 def test_blockscale_attention_rejects(L):
     a = [FAKE] * 6
     f = L.intfa_attention_fwd_blockscale

@@ -66,7 +66,8 @@ def test_reference_arm_json_line():
 def test_variant_argument_checks():
     for extra in (["--method", "index", "--scale-block", "128"], ["--method", "decode", "--lsum", "codes"],
                   ["--q-path", "fused", "--scale-block", "64"], ["--scale-block", "64", "--lsum", "codes"],
-                  ["--warmup", "2"]):
+                  ["--method", "index", "--p-levels", "255"], ["--scale-block", "64", "--p-levels", "255"],
+                  ["--p-levels", "128"], ["--warmup", "2"]):
         r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *extra], capture_output=True,
                            text=True, timeout=120, cwd=ROOT)
         assert r.returncode != 0, extra
@@ -86,6 +87,6 @@ def test_cpu_baseline_variants_run_the_oracle():
     from int8_quantized_attention_token_b200.workloads import by_name
     w = by_name("attn_B1_H1_L128_d64")
     for kw, word in (({}, "online"), ({"method": "index"}, "IndexSoftmax"), ({"blk": 64}, "block"),
-                     ({"lcodes": True}, "online")):
+                     ({"lcodes": True}, "online"), ({"p_levels": 255, "lcodes": True}, "online")):
         r = bench.cpu_baseline(w, budget_s=0.2, **kw)
         assert r["kind"] == "oracle" and r["value"] > 0 and word in r["sample"]
