@@ -113,3 +113,18 @@ def test_forward_entry_points_match_kernels():
     intfa.intfa_forward_host(Q.pin_memory(), K.pin_memory(), V.pin_memory(), True, Oh, ws)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(O1, Oh.float().numpy())
+
+
+@pytest.mark.parametrize("L,d,causal", [(131072, 64, False), (131072 - 37, 128, True)])
+def test_longest_supported_sequence(L, d, causal):
+    """The largest L the entry point accepts (and a ragged one just below it):
+    1024 query tiles of one head, every key block of a row; sampled rows."""
+    Q, K, V = make_qkv(1, 1, L, d, seed=77 + d)
+    O = run_gpu(Q, K, V, causal)
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([np.arange(0, 3), np.arange(L - 3, L), rng.choice(L, 10, replace=False)]))
+    ref = oracle_heads(Q, K, V, causal, [(0, 0)], rows=rows)
+    got = O[0, 0][rows]
+    assert np.isfinite(got).all()
+    mx, mre = gap(got, ref[(0, 0)]["O"])
+    assert mx <= TOL_MAXABS and mre <= TOL_MRE, (mx, mre)
