@@ -327,10 +327,17 @@ int intfa_forward(const void *Q_f16, const void *K_f16, const void *V_f16, int B
 
 /*
  * The same from HOST memory: copies Q, K, V (fp16, host, pinned for
- * asynchronous copies) to the device, runs intfa_forward and copies O back to
- * O_f16_host.  workspace: intfa_forward_host_workspace_size(B, H, L, d) bytes
- * of device memory, 256-byte aligned.  Asynchronous on `stream`: O_f16_host
- * is valid after the stream is synchronised.
+ * asynchronous copies) to the device, runs the path of intfa_forward and
+ * copies O back to O_f16_host.  workspace:
+ * intfa_forward_host_workspace_size(B, H, L, d) bytes of device memory,
+ * 256-byte aligned.  Asynchronous on `stream`: O_f16_host is valid after the
+ * stream is synchronised.  The heads are processed in chunks (at most 16, at
+ * least 4 MiB of fp16 per tensor each): chunk c's input copies, its
+ * quantisation + attention and its output copy overlap with the other chunks'
+ * copies in the opposite direction.  The copies run on two streams of the
+ * library's own (one pair per device, created on the first call and kept for
+ * the life of the process); calls are serialised by a host mutex while they
+ * queue their work.  Output bit-identical to intfa_forward.
  */
 size_t intfa_forward_host_workspace_size(int B, int H, int L, int d);
 int intfa_forward_host(const void *Q_f16_host, const void *K_f16_host, const void *V_f16_host,

@@ -1,6 +1,8 @@
 // api.cu -- the whole-path entry points of libintfa (quantise Q/K per token,
 // V per head, then the fused attention; and the same from host buffers) and
 // the status strings.  See include/intfa.h for the contract of each call.
+#include <mutex>
+
 #include "internal.h"
 
 namespace {
@@ -110,6 +112,57 @@ extern "C" int intfa_forward(const void *Q_f16, const void *K_f16, const void *V
     return rc;
 }
 
+namespace {
+
+// Copy streams and events of one device for the pipelined host path: made on
+// the first call on that device and kept for the life of the process (no
+// allocation of device memory; nothing is created on later calls).
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, in = nullptr, out = nullptr, done = nullptr;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_pipe_mu;             // guards g_pipes and keeps each call's enqueue sequence whole
+HostPipe g_pipes[kMaxDevices];
+
+int get_pipe(HostPipe **out) {
+    int dev = 0;
+    int rc = intfa::cuda_status(cudaGetDevice(&dev));
+    if (rc) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return INTFA_ERR_UNSUPPORTED;
+    HostPipe &p = g_pipes[dev];
+    if (!p.done) {
+        HostPipe n;
+        rc = intfa::cuda_status(cudaStreamCreateWithFlags(&n.h2d, cudaStreamNonBlocking));
+        if (!rc) rc = intfa::cuda_status(cudaStreamCreateWithFlags(&n.d2h, cudaStreamNonBlocking));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.start, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.in, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.out, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.done, cudaEventDisableTiming));
+        if (rc) {
+            if (n.h2d) cudaStreamDestroy(n.h2d);
+            if (n.d2h) cudaStreamDestroy(n.d2h);
+            for (cudaEvent_t e : {n.start, n.in, n.out, n.done})
+                if (e) cudaEventDestroy(e);
+            return rc;
+        }
+        p = n;
+    }
+    *out = &p;
+    return INTFA_OK;
+}
+
+// Heads per chunk of the host pipeline: at most 16 chunks, and at least 4 MiB
+// of fp16 per tensor per copy so that each copy runs at full link speed.
+int64_t heads_per_chunk(int64_t bh, int64_t head_bytes) {
+    const int64_t by_count = (bh + 15) / 16;
+    const int64_t by_size = ((int64_t{4} << 20) + head_bytes - 1) / head_bytes;
+    int64_t hc = by_count > by_size ? by_count : by_size;
+    return hc < bh ? hc : bh;
+}
+
+}  // namespace
+
 extern "C" int intfa_forward_host(const void *Q_f16_host, const void *K_f16_host,
                                   const void *V_f16_host, int B, int H, int L, int d, int causal,
                                   void *O_f16_host, void *workspace, size_t workspace_bytes,
@@ -120,17 +173,62 @@ extern "C" int intfa_forward_host(const void *Q_f16_host, const void *K_f16_host
         if (B <= 0 || H <= 0 || L <= 0) return INTFA_ERR_INVALID_ARG;
         return INTFA_ERR_UNSUPPORTED;
     }
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
     if (!Q_f16_host || !K_f16_host || !V_f16_host || !O_f16_host) return INTFA_ERR_INVALID_ARG;
     if (!workspace || workspace_bytes < lo.host_end) return INTFA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return INTFA_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_pipe_mu);
+    HostPipe *pp = nullptr;
+    int rc = get_pipe(&pp);
+    if (rc) return rc;
+    const HostPipe &pipe = *pp;
     uint8_t *w = static_cast<uint8_t *>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t bytes = static_cast<size_t>(B) * H * L * d * 2;
-    int rc = cuda_status(cudaMemcpyAsync(w + lo.hq, Q_f16_host, bytes, cudaMemcpyHostToDevice, s));
-    if (!rc) rc = cuda_status(cudaMemcpyAsync(w + lo.hk, K_f16_host, bytes, cudaMemcpyHostToDevice, s));
-    if (!rc) rc = cuda_status(cudaMemcpyAsync(w + lo.hv, V_f16_host, bytes, cudaMemcpyHostToDevice, s));
-    if (!rc) rc = intfa_forward(w + lo.hq, w + lo.hk, w + lo.hv, B, H, L, d, causal, w + lo.ho,
-                                workspace, lo.end, stream);
-    if (!rc) rc = cuda_status(cudaMemcpyAsync(O_f16_host, w + lo.ho, bytes, cudaMemcpyDeviceToHost, s));
-    return rc;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    const int64_t ld = intfa_vt_ld(L);
+    const size_t head_bytes = static_cast<size_t>(L) * d * 2;   // fp16 of one head
+    const int64_t hc = heads_per_chunk(bh, static_cast<int64_t>(head_bytes));
+    // Heads are independent: chunk c's host-to-device copies (stream h2d),
+    // its quantisation and attention (the caller's stream) and its output copy
+    // (stream d2h) overlap with the neighbouring chunks' copies in the other
+    // direction.  Every chunk owns its own slice of the staging buffers, so
+    // nothing is overwritten while still in use.
+    rc = cuda_status(cudaEventRecord(pipe.start, s));   // work already queued on the caller's stream
+    if (!rc) rc = cuda_status(cudaStreamWaitEvent(pipe.h2d, pipe.start, 0));
+    if (!rc) rc = cuda_status(cudaStreamWaitEvent(pipe.d2h, pipe.start, 0));
+    for (int64_t h0 = 0; !rc && h0 < bh; h0 += hc) {
+        const int64_t nh = bh - h0 < hc ? bh - h0 : hc;
+        const size_t off = static_cast<size_t>(h0) * head_bytes, bytes = static_cast<size_t>(nh) * head_bytes;
+        rc = cuda_status(cudaMemcpyAsync(w + lo.hq + off, static_cast<const uint8_t *>(Q_f16_host) + off, bytes,
+                                         cudaMemcpyHostToDevice, pipe.h2d));
+        if (!rc) rc = cuda_status(cudaMemcpyAsync(w + lo.hk + off, static_cast<const uint8_t *>(K_f16_host) + off,
+                                                  bytes, cudaMemcpyHostToDevice, pipe.h2d));
+        if (!rc) rc = cuda_status(cudaMemcpyAsync(w + lo.hv + off, static_cast<const uint8_t *>(V_f16_host) + off,
+                                                  bytes, cudaMemcpyHostToDevice, pipe.h2d));
+        if (!rc) rc = cuda_status(cudaEventRecord(pipe.in, pipe.h2d));
+        if (!rc) rc = cuda_status(cudaStreamWaitEvent(s, pipe.in, 0));
+        const int64_t rows = nh * L, r0 = h0 * L;
+        int8_t *q = reinterpret_cast<int8_t *>(w + lo.q) + r0 * d;
+        int8_t *k = reinterpret_cast<int8_t *>(w + lo.k) + r0 * d;
+        int8_t *vt = reinterpret_cast<int8_t *>(w + lo.vt) + h0 * d * ld;
+        float *sq = reinterpret_cast<float *>(w + lo.sq) + r0;
+        float *sk = reinterpret_cast<float *>(w + lo.sk) + r0;
+        float *sv = reinterpret_cast<float *>(w + lo.sv) + h0;
+        if (!rc) rc = launch_quantize_per_token(w + lo.hq + off, rows, d, q, sq, s);
+        if (!rc) rc = launch_quantize_per_token(w + lo.hk + off, rows, d, k, sk, s);
+        if (!rc) rc = launch_quantize_per_tensor(w + lo.hv + off, nh, L, d, 1, vt, sv, w + lo.ws, s);
+        if (!rc) rc = launch_attention_fwd(q, k, vt, sq, sk, sv, 1, static_cast<int>(nh), L, d, causal,
+                                           w + lo.ho + off, s);
+        if (!rc) rc = cuda_status(cudaEventRecord(pipe.out, s));
+        if (!rc) rc = cuda_status(cudaStreamWaitEvent(pipe.d2h, pipe.out, 0));
+        if (!rc) rc = cuda_status(cudaMemcpyAsync(static_cast<uint8_t *>(O_f16_host) + off, w + lo.ho + off, bytes,
+                                                  cudaMemcpyDeviceToHost, pipe.d2h));
+    }
+    // Whatever happened above, the caller's stream ends behind both copy
+    // streams, so synchronising it covers every copy this call queued.
+    int rc2 = cuda_status(cudaEventRecord(pipe.in, pipe.h2d));
+    if (!rc2) rc2 = cuda_status(cudaStreamWaitEvent(pipe.d2h, pipe.in, 0));
+    if (!rc2) rc2 = cuda_status(cudaEventRecord(pipe.done, pipe.d2h));
+    if (!rc2) rc2 = cuda_status(cudaStreamWaitEvent(s, pipe.done, 0));
+    return rc ? rc : rc2;
 }

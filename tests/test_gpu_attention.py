@@ -128,3 +128,30 @@ def test_longest_supported_sequence(L, d, causal):
     assert np.isfinite(got).all()
     mx, mre = gap(got, ref[(0, 0)]["O"])
     assert mx <= TOL_MAXABS and mre <= TOL_MRE, (mx, mre)
+
+
+@pytest.mark.parametrize("B,H,L,d,causal", [(2, 5, 4096, 128, True), (1, 6, 8192, 64, False)])
+def test_forward_host_chunks_match_device_path(B, H, L, d, causal):
+    """intfa_forward_host pipelines its copies over chunks of 4 heads here
+    (1 MiB of fp16 per head and tensor; the last chunk ragged).  Each chunk is
+    its own attention launch, so tiles meet other CTAs and other softmax
+    warpgroups than in one launch over all heads; the two warpgroups' shares
+    of the row sum then add in another order, which may move O by an fp16 ulp.
+    Against intfa_forward: within 1e-3 of max|O| (fp16 rounding level) and in
+    the parity bar; two host calls on the same buffers: the same bytes."""
+    Q, K, V = make_qkv(B, H, L, d, seed=31 + H)
+    Od = intfa.intfa_forward(Q.cuda(), K.cuda(), V.cuda(), causal).float().cpu().numpy()
+    ws = torch.empty(intfa.intfa_forward_host_workspace_size(B, H, L, d), dtype=torch.uint8, device="cuda")
+    Qp, Kp, Vp = Q.pin_memory(), K.pin_memory(), V.pin_memory()
+    outs = []
+    for _ in range(2):
+        Oh = torch.full((B, H, L, d), float("nan"), dtype=torch.float16).pin_memory()
+        intfa.intfa_forward_host(Qp, Kp, Vp, causal, Oh, ws)
+        torch.cuda.synchronize()
+        assert intfa.intfa_device_status(clear=True) == 0
+        outs.append(Oh.clone())
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    Oh = outs[0].float().numpy()
+    assert np.isfinite(Oh).all()
+    mx, mre = gap(Oh, Od)
+    assert mx <= 1e-3 and mre <= 1e-4, (mx, mre)
