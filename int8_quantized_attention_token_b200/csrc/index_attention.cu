@@ -15,14 +15,18 @@
 // pages' two-pass form), so the integer accumulators need no rescaling: the
 // P V products of all key blocks accumulate in TMEM.
 //
-// B200 design: one CTA per (128-query tile, head), 6 warps:
-//   warps 0-3  one thread per query row (TMEM lane quadrant = warp): pass A
-//              row max, pass B distances, table lookups, P codes and the
-//              integer row sum, then the epilogue.
-//   warp 4     TMA producer: the Q_hat tile, then for each of the 2 nb steps
+// B200 design: one CTA per (128-query tile, head), 10 warps:
+//   warps 0-7  two threads per query row: warp w reads TMEM lane quadrant
+//              w mod 4 and key half w / 4 (64 of each block's 128 keys).
+//              Pass A: the half's row max; the two halves meet once, through
+//              shared memory, after the last block.  Pass B: distances,
+//              table lookups, P codes of the half's keys and its integer row
+//              sum; the halves add their sums once at the end and each
+//              writes half of the output row.
+//   warp 8     TMA producer: the Q_hat tile, then for each of the 2 nb steps
 //              (nb key blocks, twice) the K_hat tile and, in pass B, the
 //              V_hat^T tile, through a 4-stage ring.
-//   warp 5     MMA issuer (one lane), TMEM owner: Q K^T of every step into
+//   warp 9     MMA issuer (one lane), TMEM owner: Q K^T of every step into
 //              one of two S buffers (first set to a float bias by an fp16 MMA
 //              so that S reads back as fp32 exactly), and in pass B the P V
 //              products, accumulated in an int32 TMEM block.
@@ -47,9 +51,14 @@ constexpr int BM = 128;                 // query rows per CTA
 constexpr int BN = 128;                 // keys per block
 constexpr int NS = 4;                   // K / V ring depth
 constexpr int SB = 2;                   // TMEM S buffers
-constexpr int kThreads = 192;           // 6 warps
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kParts = 2;          // row warps per TMEM lane quadrant (key parts of a block)
+static_assert(kParts == 1 || kParts == 2 || kParts == 4, "a block's 4 chunks split evenly");
+constexpr int kRowWarps = 4 * kParts;
+constexpr int kChunks = 4 / kParts;     // 32-key chunks of a block per row warp
+constexpr int kThreads = 32 * (kRowWarps + 2);
+constexpr int kProducerWarp = kRowWarps;
+constexpr int kMmaWarp = kRowWarps + 1;
+constexpr int kRowBarrier = 1;          // named barrier of the row warps
 constexpr int kTmemCols = 512;          // S0, S1 (2 x 128) + P V accumulator (128)
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
 constexpr uint32_t kSleepNs = 1000000;
@@ -76,6 +85,8 @@ struct alignas(1024) IdxSmem {
     uint64_t pv_done[SB];       // pass B: P V of the step in buffer b done
     uint64_t acc_full;          // all P V products of the tile done
     uint64_t mma_drain;
+    float half_max[kParts][BM];      // each key part's row max (biased float)
+    uint32_t half_sum[kParts][BM];   // each key part's integer row sum
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -120,6 +131,12 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
             return;
         }
     }
+}
+
+// The row warps (warps 0-7) meet: every row warp reaches each call exactly
+// once, whatever happened to its waits before.
+__device__ __forceinline__ void row_barrier() {
+    asm volatile("bar.sync %0, %1;" ::"n"(kRowBarrier), "n"(32 * kRowWarps) : "memory");
 }
 
 // c_int of eq. 8 in fp64: rint((c sqrt(d)) / (s_Q s_K)), at least 1 (and at
@@ -180,13 +197,13 @@ __device__ __forceinline__ void lookup_chunk(const uint32_t (&w)[32], float mbf,
     }
 }
 
-template <bool kFast>
-__device__ __forceinline__ void lookup_block(uint32_t (&w)[4][32], float mbf, float cf, float q,
+template <bool kFast, int NCH>
+__device__ __forceinline__ void lookup_block(uint32_t (&w)[NCH][32], float mbf, float cf, float q,
                                              unsigned long long cint, uint32_t nm1, const uint8_t *lut,
                                              bool need_mask, int key0, int lim, uint32_t &l,
                                              uint32_t ts) {
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 0; ch < NCH; ++ch) {
         uint32_t pk[8];
         if (need_mask)
             lookup_chunk<kFast, true>(w[ch], mbf, cf, q, cint, nm1, lut, key0 + 32 * ch, lim, l, pk);
@@ -222,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < SB; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.s_read[b], BM);
-            mbar_init(&sm.p_full[b], BM);
+            mbar_init(&sm.s_read[b], kParts * BM);   // every row warp reads its part
+            mbar_init(&sm.p_full[b], kParts * BM);
             mbar_init(&sm.pv_done[b], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -337,33 +354,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------ rows (warps 0-3) ---
-        const int row = 32 * warp + lane;
+        // ------------------------------------------ rows (warps 0-7) ---
+        const int quad = warp & 3, half = warp >> 2;
+        const int row = 32 * quad + lane;
         const int qi = q0 + row;
         const int lim = causal ? min(L, qi + 1) : L;
-        const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
+        const int kofs = 32 * kChunks * half;   // this warp's keys in each block
         bool ok = true;
-        uint32_t w[4][32];
-        // -- pass A: the integer row max over visible keys (as a biased float)
+        uint32_t w[kChunks][32];
+        // -- pass A: the integer row max over this half's visible keys (as a biased float)
         float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int j = 0; j < nb; ++j) {
             const int s = j, b = s & 1;
             if (!warp_wait(&sm.s_full[b], (s >> 1) & 1, abort_flag, 8)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t ts = tS + lane_off + b * BN;
+            const uint32_t ts = tS + lane_off + b * BN + kofs;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) tmem_ld32(ts + 32 * ch, w[ch]);
+            for (int ch = 0; ch < kChunks; ++ch) tmem_ld32(ts + 32 * ch, w[ch]);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.s_read[b]);
             if ((causal && j == nb - 1) || ((j + 1) * BN > L)) {
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) mask_zero(w[ch], j * BN + 32 * ch, lim);
+                for (int ch = 0; ch < kChunks; ++ch) mask_zero(w[ch], j * BN + kofs + 32 * ch, lim);
             }
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) max_chunk(w[ch], mx);
+            for (int ch = 0; ch < kChunks; ++ch) max_chunk(w[ch], mx);
         }
-        const float mbf = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        sm.half_max[half][row] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        row_barrier();
+        float mbf = sm.half_max[0][row];
+#pragma unroll
+        for (int h = 1; h < kParts; ++h) mbf = fmaxf(mbf, sm.half_max[h][row]);
         // -- the head's clip threshold and index scale
         const long long cint = clip_threshold(c, D, __ldg(sQ + bh), __ldg(sK + bh));
         const bool fast = cint <= (1ll << (23 - bits));
@@ -371,34 +394,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         // q = (2^b - 1) / c_int rounded up: then floor(D' q) = floor(D' (2^b - 1) / c_int)
         // for every integer 0 <= D' <= c_int while c_int <= 2^(23 - b)
         const float q = __fdiv_ru(static_cast<float>(nm1), cf);
-        // -- pass B: distances, table, P codes, integer row sum
+        // -- pass B: distances, table, P codes, integer row sum of this half
         uint32_t l = 0;
         for (int j = 0; ok && j < nb; ++j) {
             const int s = nb + j, b = s & 1;
             if (!warp_wait(&sm.s_full[b], (s >> 1) & 1, abort_flag, 9)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t ts = tS + lane_off + b * BN;
+            const uint32_t ts = tS + lane_off + b * BN + kofs;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) tmem_ld32(ts + 32 * ch, w[ch]);
+            for (int ch = 0; ch < kChunks; ++ch) tmem_ld32(ts + 32 * ch, w[ch]);
             tmem_wait_ld();
             const bool need_mask = (causal && j == nb - 1) || ((j + 1) * BN > L);
             if (fast)
-                lookup_block<true>(w, mbf, cf, q, static_cast<unsigned long long>(cint), nm1, sm.lut,
-                                   need_mask, j * BN, lim, l, ts);
+                lookup_block<true, kChunks>(w, mbf, cf, q, static_cast<unsigned long long>(cint), nm1, sm.lut,
+                                      need_mask, j * BN + kofs, lim, l, ts);
             else
-                lookup_block<false>(w, mbf, cf, q, static_cast<unsigned long long>(cint), nm1, sm.lut,
-                                    need_mask, j * BN, lim, l, ts);
+                lookup_block<false, kChunks>(w, mbf, cf, q, static_cast<unsigned long long>(cint), nm1, sm.lut,
+                                       need_mask, j * BN + kofs, lim, l, ts);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_full[b]);
         }
-        // -- epilogue: O = s_V acc / l
+        sm.half_sum[half][row] = l;
+        row_barrier();
+        uint32_t lrow = 0;
+#pragma unroll
+        for (int h = 0; h < kParts; ++h) lrow += sm.half_sum[h][row];
+        // -- epilogue: O = s_V acc / l, each half writing D / 2 channels
         if (ok && warp_wait(&sm.acc_full, 0, abort_flag, 10)) {
             tc_fence_after();
-            const float f = __ldg(sV + bh) / static_cast<float>(l);   // l >= 255 (the max key)
+            const float f = __ldg(sV + bh) / static_cast<float>(lrow);   // l >= 255 (the max key)
             const int64_t obase = (static_cast<int64_t>(bh) * L + qi) * D;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
+            for (int ch = half; ch < D / 32; ch += kParts) {
                 uint32_t a[32];
                 tmem_ld32(tO + lane_off + 32 * ch, a);
                 tmem_wait_ld();
@@ -416,10 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (qi < L) {
+            if (qi < L && half == 0) {
                 const int64_t r = static_cast<int64_t>(bh) * L + qi;
                 if (m_out) m_out[r] = __float2int_rn(mbf - kBias);
-                if (l_out) l_out[r] = static_cast<int32_t>(l);
+                if (l_out) l_out[r] = static_cast<int32_t>(lrow);
             }
         }
     }
