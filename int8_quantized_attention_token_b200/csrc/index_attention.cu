@@ -25,11 +25,14 @@
 //              writes half of the output row.
 //   warp 8     TMA producer: the Q_hat tile, then for each of the 2 nb steps
 //              (nb key blocks, twice) the K_hat tile and, in pass B, the
-//              V_hat^T tile, through a 4-stage ring.
+//              V_hat^T tile, through a 2-stage ring.
 //   warp 9     MMA issuer (one lane), TMEM owner: Q K^T of every step into
-//              one of two S buffers (first set to a float bias by an fp16 MMA
+//              the S buffer (first set to a float bias by an fp16 MMA
 //              so that S reads back as fp32 exactly), and in pass B the P V
 //              products, accumulated in an int32 TMEM block.
+// Two CTAs share an SM (256 TMEM columns, 96 registers per thread and ~84 KB
+// of shared memory each): one CTA's row warps work while the other's MMAs
+// run, in place of a second S buffer within the CTA.
 // Every wait is bounded (clock-based); a timeout records a status word,
 // raises a CTA-wide abort flag, drains in-flight copies and MMAs, frees TMEM
 // and returns.
@@ -49,8 +52,9 @@ namespace {
 
 constexpr int BM = 128;                 // query rows per CTA
 constexpr int BN = 128;                 // keys per block
-constexpr int NS = 4;                   // K / V ring depth
-constexpr int SB = 2;                   // TMEM S buffers
+constexpr int NS = 2;                   // K / V ring depth
+constexpr int SB = 1;                   // TMEM S buffers (two CTAs per SM overlap each other's steps)
+constexpr int kMinBlocks = 2;           // CTAs per SM: TMEM, registers and shared memory sized for two
 constexpr int kParts = 2;          // row warps per TMEM lane quadrant (key parts of a block)
 static_assert(kParts == 1 || kParts == 2 || kParts == 4, "a block's 4 chunks split evenly");
 constexpr int kRowWarps = 4 * kParts;
@@ -59,7 +63,8 @@ constexpr int kThreads = 32 * (kRowWarps + 2);
 constexpr int kProducerWarp = kRowWarps;
 constexpr int kMmaWarp = kRowWarps + 1;
 constexpr int kRowBarrier = 1;          // named barrier of the row warps
-constexpr int kTmemCols = 512;          // S0, S1 (2 x 128) + P V accumulator (128)
+constexpr int kTmemCols = 256;          // the S buffer (128 columns) + the P V accumulator (<= 128)
+static_assert(SB * BN + 128 <= kTmemCols, "TMEM columns");
 constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
 constexpr uint32_t kSleepNs = 1000000;
 // Accumulator bias: 1.5 * 2^23 as fp32 has the bit pattern 0x4B400000; an
@@ -214,7 +219,7 @@ __device__ __forceinline__ void lookup_block(uint32_t (&w)[NCH][32], float mbf, 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
     attn_index_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
                       const float *__restrict__ sK, const float *__restrict__ sV,
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tS = sm.tmem_base;           // S buffer b at column 128 b
-    const uint32_t tO = sm.tmem_base + 2 * BN;  // int32 P V accumulator
+    const uint32_t tO = sm.tmem_base + SB * BN;  // int32 P V accumulator
 
     if (warp == kProducerWarp) {
         // ----------------------------------------------- TMA producer ---
@@ -304,12 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bias_a = make_sdesc_noswz(smem_u32(sm.bias_ab[0]), 16, 16);
             const uint64_t bias_b = make_sdesc_noswz(smem_u32(sm.bias_ab[1]), 16, 16);
             const uint64_t qdesc = make_sdesc(smem_u32(sm.q), kSbo, kSw);
-            uint32_t n_read[SB] = {0, 0}, n_pv[SB] = {0, 0}, n_p[SB] = {0, 0};
+            uint32_t n_read[SB] = {}, n_pv[SB] = {}, n_p[SB] = {};
             bool ok = wait_bar(&sm.q_full, 0, abort_flag, 2);
             // Q K^T of step s into S buffer s mod 2, once the step two back has
             // released it (pass A: the row warps read it; pass B: its P V ran)
             auto issue_qk = [&](int s) -> bool {
-                const int st = s % NS, b = s & 1;
+                const int st = s % NS, b = s % SB;
                 if (!wait_bar(&sm.full[st], (s / NS) & 1, abort_flag, 3)) return false;
                 if (s >= SB) {
                     if (s - SB < nb) {
@@ -330,11 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (s < nb) mma_commit(&sm.empty[st]);   // pass A: only the K tile was used
                 return true;
             };
-            if (ok) ok = issue_qk(0);
-            if (ok && T > 1) ok = issue_qk(1);
+            for (int s0 = 0; ok && s0 < SB && s0 < T; ++s0) ok = issue_qk(s0);
             for (int s = 0; ok && s < T; ++s) {
                 if (s >= nb) {
-                    const int j = s - nb, b = s & 1, st = s % NS;
+                    const int j = s - nb, b = s % SB, st = s % NS;
                     if (!wait_bar(&sm.p_full[b], n_p[b] & 1, abort_flag, 6)) break;
                     ++n_p[b];
                     tc_fence_after();
@@ -366,8 +370,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // -- pass A: the integer row max over this half's visible keys (as a biased float)
         float mx[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for (int j = 0; j < nb; ++j) {
-            const int s = j, b = s & 1;
-            if (!warp_wait(&sm.s_full[b], (s >> 1) & 1, abort_flag, 8)) { ok = false; break; }
+            const int s = j, b = s % SB;
+            if (!warp_wait(&sm.s_full[b], (s / SB) & 1, abort_flag, 8)) { ok = false; break; }
             tc_fence_after();
             const uint32_t ts = tS + lane_off + b * BN + kofs;
 #pragma unroll
@@ -397,8 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // -- pass B: distances, table, P codes, integer row sum of this half
         uint32_t l = 0;
         for (int j = 0; ok && j < nb; ++j) {
-            const int s = nb + j, b = s & 1;
-            if (!warp_wait(&sm.s_full[b], (s >> 1) & 1, abort_flag, 9)) { ok = false; break; }
+            const int s = nb + j, b = s % SB;
+            if (!warp_wait(&sm.s_full[b], (s / SB) & 1, abort_flag, 9)) { ok = false; break; }
             tc_fence_after();
             const uint32_t ts = tS + lane_off + b * BN + kofs;
 #pragma unroll
