@@ -138,6 +138,13 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// One byte of shared memory at a 32-bit shared-window address.
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
 // The row warps (warps 0-7) meet: every row warp reaches each call exactly
 // once, whatever happened to its waits before.
 __device__ __forceinline__ void row_barrier() {
@@ -178,24 +185,30 @@ __device__ __forceinline__ void max_chunk(const uint32_t (&w)[32], float (&mx)[4
 template <bool kFast, bool kMask>
 __device__ __forceinline__ void lookup_chunk(const uint32_t (&w)[32], float mbf, float cf, float q,
                                              unsigned long long cint, uint32_t nm1,
-                                             const uint8_t *lut, int key0, int lim, uint32_t &l,
-                                             uint32_t (&pk)[8]) {
+                                             const uint8_t *lut, uint32_t lut_biased, int key0, int lim,
+                                             uint32_t &l, uint32_t (&pk)[8]) {
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
         uint32_t e[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-            // distance to the row max: both are integers + 1.5 * 2^23, so the
-            // difference is exact
-            const float dl = fminf(mbf - __uint_as_float(w[4 * g + t]), cf);
-            uint32_t idx;
-            if constexpr (kFast)
-                idx = __float_as_uint(__fmaf_rd(dl, q, 8388608.0f)) - 0x4B000000u;
-            else
-                idx = static_cast<uint32_t>((static_cast<unsigned long long>(dl) * nm1) / cint);
-            idx = min(idx, nm1);
-            e[t] = lut[idx];
-            if (kMask && key0 + 4 * g + t >= lim) e[t] = 0u;
+            const bool masked = kMask && key0 + 4 * g + t >= lim;
+            if constexpr (kFast) {
+                // a masked key looks up D' = 0 (its value is zeroed below);
+                // a visible one has 0 <= D' <= c_int, so D' q + 2^23 rounded
+                // down is 0x4B000000 + idx with idx <= 2^b - 1, and adding its
+                // bits to the table's shared address minus 0x4B000000 gives
+                // the entry's address in one integer add
+                const float sv = masked ? mbf : __uint_as_float(w[4 * g + t]);
+                const float dl = fminf(mbf - sv, cf);   // exact: both are integers + 1.5 * 2^23
+                e[t] = lds_u8(lut_biased + __float_as_uint(__fmaf_rd(dl, q, 8388608.0f)));
+            } else {
+                const float dl = fminf(mbf - __uint_as_float(w[4 * g + t]), cf);
+                uint32_t idx = static_cast<uint32_t>((static_cast<unsigned long long>(dl) * nm1) / cint);
+                idx = min(idx, nm1);
+                e[t] = lut[idx];
+            }
+            if (masked) e[t] = 0u;
         }
         pk[g] = prmt(prmt(e[0], e[1], 0x0040u), prmt(e[2], e[3], 0x0040u), 0x5410u);
         l = __dp4a(pk[g], 0x01010101u, l);
@@ -207,13 +220,14 @@ __device__ __forceinline__ void lookup_block(uint32_t (&w)[NCH][32], float mbf, 
                                              unsigned long long cint, uint32_t nm1, const uint8_t *lut,
                                              bool need_mask, int key0, int lim, uint32_t &l,
                                              uint32_t ts) {
+    const uint32_t lut_biased = smem_u32(lut) - 0x4B000000u;   // wraps; the add in lookup_chunk wraps back
 #pragma unroll
     for (int ch = 0; ch < NCH; ++ch) {
         uint32_t pk[8];
         if (need_mask)
-            lookup_chunk<kFast, true>(w[ch], mbf, cf, q, cint, nm1, lut, key0 + 32 * ch, lim, l, pk);
+            lookup_chunk<kFast, true>(w[ch], mbf, cf, q, cint, nm1, lut, lut_biased, key0 + 32 * ch, lim, l, pk);
         else
-            lookup_chunk<kFast, false>(w[ch], mbf, cf, q, cint, nm1, lut, key0 + 32 * ch, lim, l, pk);
+            lookup_chunk<kFast, false>(w[ch], mbf, cf, q, cint, nm1, lut, lut_biased, key0 + 32 * ch, lim, l, pk);
         tmem_st8(ts + 32 * ch, pk);   // codes of keys 32 ch .. 32 ch + 31: the A operand of P V step ch
     }
 }
