@@ -179,3 +179,11 @@ def test_forward_rejects(L):
     assert L.intfa_forward(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, FAKE + 16, ws, None) == 3
     assert L.intfa_forward(FAKE, FAKE, FAKE, 1, 1, 128, 80, 0, FAKE, FAKE, ws, None) == 2
     assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, FAKE, ws, None) == 6
+    wsh = intfa.intfa_forward_host_workspace_size(1, 1, 128, 64)
+    # every check of the host path runs before it touches a stream or the device
+    assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 64, 2, FAKE, FAKE, wsh, None) == 1   # causal flag
+    assert L.intfa_forward_host(None, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, FAKE, wsh, None) == 1
+    assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, None, FAKE, wsh, None) == 1   # O
+    assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, FAKE + 16, wsh, None) == 3
+    assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 96, 0, FAKE, FAKE, wsh, None) == 2   # d
+    assert L.intfa_forward_host(FAKE, FAKE, FAKE, 0, 1, 128, 64, 0, FAKE, FAKE, wsh, None) == 1   # B
