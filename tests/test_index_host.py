@@ -58,3 +58,30 @@ def test_fast_index_small_cint_exhaustive():
             q = q_round_up(nm1, cint)
             for dl in range(cint + 1):
                 assert fast_index(dl, q) == (dl * nm1) // cint
+
+
+def fma_rd_bits(dl: int, q: Fraction) -> int:
+    """Bits of fl_down(D' q + 2^23) as fp32 (D' q < 2^23: the value stays in
+    [2^23, 2^24), where fp32 has unit spacing)."""
+    v = (dl * q + (1 << 23)) // 1
+    assert (1 << 23) <= v < (1 << 24)
+    return 0x4B000000 + (v - (1 << 23))
+
+
+@pytest.mark.parametrize("b", [1, 5, 8])
+def test_table_address_one_add_stays_in_table(b):
+    # The kernel reads entry idx at (base - 0x4B000000) + bits, both mod 2^32,
+    # with no clamp: for every visible key (0 <= D' <= c_int) and for a masked
+    # key (looked up at D' = 0) the address must land in [base, base + 2^b - 1].
+    nm1 = (1 << b) - 1
+    rng = np.random.default_rng(40 + b)
+    bound = 1 << (23 - b)
+    for base in (0, 1024, 0xFFFFF000, int(rng.integers(0, 1 << 32))):
+        for cint in [1, 2, 3, nm1, nm1 + 1, bound] + [int(x) for x in rng.integers(1, bound, 20)]:
+            q = q_round_up(nm1, cint)
+            for dl in {0, 1, cint // 2, cint - 1, cint}:
+                if not 0 <= dl <= cint:
+                    continue
+                addr = ((base - 0x4B000000) + fma_rd_bits(dl, q)) % (1 << 32)
+                off = (addr - base) % (1 << 32)
+                assert off == (dl * nm1) // cint <= nm1, (base, cint, dl)
