@@ -16,6 +16,7 @@ bool make_layout(int B, int H, int L, int d, Layout *lo) {
     if (B <= 0 || H <= 0 || L <= 0 || (d != 64 && d != 128)) return false;
     const size_t bh = static_cast<size_t>(B) * H;
     if (bh > (1u << 24) || L > 131072) return false;
+    if (bh * ((static_cast<size_t>(L) + 127) / 128) > 0x7FFFFFFFu) return false;   // tile count fits an int
     const size_t n = bh * static_cast<size_t>(L);              // token rows
     const size_t ld = static_cast<size_t>(intfa_vt_ld(L));
     size_t off = 0;

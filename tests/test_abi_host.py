@@ -187,3 +187,6 @@ def test_forward_rejects(L):
     assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, FAKE, FAKE + 16, wsh, None) == 3
     assert L.intfa_forward_host(FAKE, FAKE, FAKE, 1, 1, 128, 96, 0, FAKE, FAKE, wsh, None) == 2   # d
     assert L.intfa_forward_host(FAKE, FAKE, FAKE, 0, 1, 128, 64, 0, FAKE, FAKE, wsh, None) == 1   # B
+    # B H ceil(L / 128) query tiles must fit an int (here 2^24 heads of 1024 tiles)
+    assert intfa.intfa_forward_workspace_size(1 << 12, 1 << 12, 131072, 64) == 0
+    assert L.intfa_forward(FAKE, FAKE, FAKE, 1 << 12, 1 << 12, 131072, 64, 0, FAKE, FAKE, ws, None) == 2
