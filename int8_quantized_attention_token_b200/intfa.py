@@ -53,6 +53,8 @@ def lib():
         "intfa_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
         "intfa_attention_fwd_q16": ([P, P, P, P, P, I, I, I, I, I, P, P, P], I),
         "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
+        "intfa_debug_attention_scores": ([P, P, P, P, P, P, I, I, I, I, I, P, P, P], I),
+        "intfa_debug_wait_timeout": ([P, P, P, P, P, P, I, I, I, I, I, P, I64, P], I),
         "intfa_attention_fwd_codesum": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
         "intfa_attention_fwd_pcodes": ([P, P, P, P, P, P, I, I, I, I, I, I, I, P, P], I),
         "intfa_attention_fwd_blockscale": ([P, P, P, P, P, P, I, I, I, I, I, I, P, P], I),
@@ -100,13 +102,33 @@ def _ptr(t) -> int:
     return t.data_ptr()
 
 
-def _need(t: torch.Tensor, dtype, name: str):
-    if not t.is_cuda:
+def _need(t: torch.Tensor, dtype, name: str, shape=None, device=None):
+    """t must be a contiguous CUDA tensor of `dtype` (and of `shape` / on
+    `device` when given): the library writes through raw pointers, so a wrong
+    size or a tensor on another GPU must be caught before any launch."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _out(t, shape, dtype, device, name: str):
+    """A caller-provided output (checked like an input), or a new tensor."""
+    if t is None:
+        return torch.empty(tuple(shape), dtype=dtype, device=device)
+    _need(t, dtype, name, shape=shape, device=device)
+    return t
+
+
+def _on(device):
+    """The library launches on the current CUDA device: make it x's."""
+    return torch.cuda.device(device)
 
 
 # ------------------------------------------------------------- entry points ---
@@ -120,10 +142,11 @@ def intfa_quantize_per_token(x: torch.Tensor, x_q=None, scale=None, stream=None)
     _need(x, torch.float16, "x")
     d = x.shape[-1]
     rows = x.numel() // d if d else 0
-    x_q = torch.empty(x.shape, dtype=torch.int8, device=x.device) if x_q is None else x_q
-    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if scale is None else scale
-    _check(lib().intfa_quantize_per_token(_ptr(x), rows, d, _ptr(x_q), _ptr(scale), _stream(stream)),
-           "intfa_quantize_per_token")
+    x_q = _out(x_q, x.shape, torch.int8, x.device, "x_q")
+    scale = _out(scale, x.shape[:-1], torch.float32, x.device, "scale")
+    with _on(x.device):
+        _check(lib().intfa_quantize_per_token(_ptr(x), rows, d, _ptr(x_q), _ptr(scale), _stream(stream)),
+               "intfa_quantize_per_token")
     return x_q, scale
 
 
@@ -132,11 +155,30 @@ def intfa_quantize_per_token_bits(x: torch.Tensor, bits: int, x_q=None, scale=No
     _need(x, torch.float16, "x")
     d = x.shape[-1]
     rows = x.numel() // d if d else 0
-    x_q = torch.empty(x.shape, dtype=torch.int8, device=x.device) if x_q is None else x_q
-    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if scale is None else scale
-    _check(lib().intfa_quantize_per_token_bits(_ptr(x), rows, d, int(bits), _ptr(x_q), _ptr(scale), _stream(stream)),
-           "intfa_quantize_per_token_bits")
+    x_q = _out(x_q, x.shape, torch.int8, x.device, "x_q")
+    scale = _out(scale, x.shape[:-1], torch.float32, x.device, "scale")
+    with _on(x.device):
+        _check(lib().intfa_quantize_per_token_bits(_ptr(x), rows, d, int(bits), _ptr(x_q), _ptr(scale),
+                                                   _stream(stream)), "intfa_quantize_per_token_bits")
     return x_q, scale
+
+
+def _tensor_outputs(x, transpose, x_q, scale):
+    """Codes ([g, rows, cols], or [g, cols, intfa_vt_ld(rows)] transposed)
+    and the g scales of a per-tensor quantisation of x [g, rows, cols]."""
+    g, rows, cols = x.shape
+    shape = (g, cols, intfa_vt_ld(rows)) if transpose else (g, rows, cols)
+    return (_out(x_q, shape, torch.int8, x.device, "x_q"),
+            _out(scale, (g,), torch.float32, x.device, "scale"))
+
+
+def _workspace(ws, nbytes, device):
+    if ws is None:
+        return torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=device)
+    _need(ws, torch.uint8, "workspace", device=device)
+    if ws.numel() < nbytes:
+        raise ValueError(f"workspace must hold {nbytes} bytes, got {ws.numel()}")
+    return ws
 
 
 def intfa_quantize_per_tensor(x: torch.Tensor, transpose: bool = False, x_q=None, scale=None,
@@ -149,16 +191,12 @@ def intfa_quantize_per_tensor(x: torch.Tensor, transpose: bool = False, x_q=None
     if x.dim() != 3:
         raise ValueError("x must be [groups, rows, cols]")
     g, rows, cols = x.shape
-    if x_q is None:
-        shape = (g, cols, intfa_vt_ld(rows)) if transpose else (g, rows, cols)
-        x_q = torch.empty(shape, dtype=torch.int8, device=x.device)
-    scale = torch.empty((g,), dtype=torch.float32, device=x.device) if scale is None else scale
-    wsb = int(lib().intfa_quantize_per_tensor_workspace_size(g))
-    if workspace is None:
-        workspace = torch.empty((max(wsb, 1),), dtype=torch.uint8, device=x.device)
-    _check(lib().intfa_quantize_per_tensor(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
-                                           _ptr(scale), _ptr(workspace), workspace.numel(),
-                                           _stream(stream)), "intfa_quantize_per_tensor")
+    x_q, scale = _tensor_outputs(x, transpose, x_q, scale)
+    workspace = _workspace(workspace, int(lib().intfa_quantize_per_tensor_workspace_size(g)), x.device)
+    with _on(x.device):
+        _check(lib().intfa_quantize_per_tensor(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
+                                               _ptr(scale), _ptr(workspace), workspace.numel(),
+                                               _stream(stream)), "intfa_quantize_per_tensor")
     return x_q, scale
 
 
@@ -171,15 +209,12 @@ def intfa_quantize_global(x: torch.Tensor, transpose: bool = False, x_q=None, sc
     if x.dim() != 3:
         raise ValueError("x must be [groups, rows, cols]")
     g, rows, cols = x.shape
-    if x_q is None:
-        shape = (g, cols, intfa_vt_ld(rows)) if transpose else (g, rows, cols)
-        x_q = torch.empty(shape, dtype=torch.int8, device=x.device)
-    scale = torch.empty((g,), dtype=torch.float32, device=x.device) if scale is None else scale
-    wsb = int(lib().intfa_quantize_per_tensor_workspace_size(g))
-    if workspace is None:
-        workspace = torch.empty((max(wsb, 1),), dtype=torch.uint8, device=x.device)
-    _check(lib().intfa_quantize_global(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q), _ptr(scale),
-                                       _ptr(workspace), workspace.numel(), _stream(stream)), "intfa_quantize_global")
+    x_q, scale = _tensor_outputs(x, transpose, x_q, scale)
+    workspace = _workspace(workspace, int(lib().intfa_quantize_per_tensor_workspace_size(g)), x.device)
+    with _on(x.device):
+        _check(lib().intfa_quantize_global(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q), _ptr(scale),
+                                           _ptr(workspace), workspace.numel(), _stream(stream)),
+               "intfa_quantize_global")
     return x_q, scale
 
 
@@ -195,42 +230,51 @@ def intfa_quantize_per_tensor_noalloc(x: torch.Tensor, transpose: bool = False, 
     if x.dim() != 3:
         raise ValueError("x must be [groups, rows, cols]")
     g, rows, cols = x.shape
-    if x_q is None:
-        shape = (g, cols, intfa_vt_ld(rows)) if transpose else (g, rows, cols)
-        x_q = torch.empty(shape, dtype=torch.int8, device=x.device)
-    scale = torch.empty((g,), dtype=torch.float32, device=x.device) if scale is None else scale
-    _check(lib().intfa_quantize_per_tensor_noalloc(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
-                                                   _ptr(scale), _stream(stream)),
-           "intfa_quantize_per_tensor_noalloc")
+    x_q, scale = _tensor_outputs(x, transpose, x_q, scale)
+    with _on(x.device):
+        _check(lib().intfa_quantize_per_tensor_noalloc(_ptr(x), g, rows, cols, int(bool(transpose)), _ptr(x_q),
+                                                       _ptr(scale), _stream(stream)),
+               "intfa_quantize_per_tensor_noalloc")
     return x_q, scale
+
+
+def _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V, nsc=None):
+    """Check the fused attention's inputs against Q_q's shape [B, H, L, d] and
+    device; nsc = scales per head of s_Q / s_K (L unless per-block)."""
+    if not isinstance(Q_q, torch.Tensor) or Q_q.dim() != 4:
+        raise ValueError("Q_q must be [B, H, L, d]")
+    B, H, L, d = Q_q.shape
+    dev = Q_q.device
+    nsc = L if nsc is None else nsc
+    _need(Q_q, torch.int8, "Q_q", device=dev)
+    _need(K_q, torch.int8, "K_q", shape=(B, H, L, d), device=dev)
+    _need(Vt_q, torch.int8, "Vt_q", shape=(B, H, d, intfa_vt_ld(L)), device=dev)
+    _need(s_Q, torch.float32, "s_Q", shape=(B, H, nsc), device=dev)
+    _need(s_K, torch.float32, "s_K", shape=(B, H, nsc), device=dev)
+    _need(s_V, torch.float32, "s_V", shape=(B, H), device=dev)
+    return B, H, L, d
 
 
 def intfa_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, O=None, stream=None):
     """Q_q, K_q int8 [B, H, L, d]; Vt_q int8 [B, H, d, intfa_vt_ld(L)];
     s_Q, s_K fp32 [B, H, L]; s_V fp32 [B, H]  ->  O fp16 [B, H, L, d]."""
-    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
-        _need(t, torch.int8, n)
-    for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
-        _need(t, torch.float32, n)
-    B, H, L, d = Q_q.shape
-    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
-    _check(lib().intfa_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
-                                     _ptr(s_V), B, H, L, d, int(bool(causal)), _ptr(O),
-                                     _stream(stream)), "intfa_attention_fwd")
+    B, H, L, d = _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V)
+    O = _out(O, (B, H, L, d), torch.float16, Q_q.device, "O")
+    with _on(Q_q.device):
+        _check(lib().intfa_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
+                                         _ptr(s_V), B, H, L, d, int(bool(causal)), _ptr(O),
+                                         _stream(stream)), "intfa_attention_fwd")
     return O
 
 
 def intfa_attention_fwd_codesum(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, O=None, stream=None):
     """intfa_attention_fwd with the row sum taken from the P codes (sum P_hat / 127)."""
-    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
-        _need(t, torch.int8, n)
-    for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
-        _need(t, torch.float32, n)
-    B, H, L, d = Q_q.shape
-    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
-    _check(lib().intfa_attention_fwd_codesum(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
-                                             B, H, L, d, int(bool(causal)), _ptr(O), _stream(stream)),
-           "intfa_attention_fwd_codesum")
+    B, H, L, d = _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V)
+    O = _out(O, (B, H, L, d), torch.float16, Q_q.device, "O")
+    with _on(Q_q.device):
+        _check(lib().intfa_attention_fwd_codesum(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
+                                                 B, H, L, d, int(bool(causal)), _ptr(O), _stream(stream)),
+               "intfa_attention_fwd_codesum")
     return O
 
 
@@ -238,16 +282,13 @@ def intfa_attention_fwd_pcodes(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, p_le
                                lsum_codes: bool = False, O=None, stream=None):
     """intfa_attention_fwd with P codes RNE(p_levels p): 127 (INT8 P) or 255
     (UINT8 P); lsum_codes takes the row sum from the codes (sum P_hat / p_levels)."""
-    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
-        _need(t, torch.int8, n)
-    for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
-        _need(t, torch.float32, n)
-    B, H, L, d = Q_q.shape
-    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
-    _check(lib().intfa_attention_fwd_pcodes(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
-                                            B, H, L, d, int(bool(causal)), int(p_levels), int(bool(lsum_codes)),
-                                            _ptr(O), _stream(stream)),
-           "intfa_attention_fwd_pcodes")
+    B, H, L, d = _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V)
+    O = _out(O, (B, H, L, d), torch.float16, Q_q.device, "O")
+    with _on(Q_q.device):
+        _check(lib().intfa_attention_fwd_pcodes(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
+                                                B, H, L, d, int(bool(causal)), int(p_levels), int(bool(lsum_codes)),
+                                                _ptr(O), _stream(stream)),
+               "intfa_attention_fwd_pcodes")
     return O
 
 
@@ -255,15 +296,14 @@ def intfa_attention_fwd_blockscale(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, 
                                    stream=None):
     """intfa_attention_fwd with one Q / K scale per block of `scale_block`
     tokens: s_Q, s_K fp32 [B, H, ceil(L / scale_block)]."""
-    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
-        _need(t, torch.int8, n)
-    for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
-        _need(t, torch.float32, n)
-    B, H, L, d = Q_q.shape
-    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
-    _check(lib().intfa_attention_fwd_blockscale(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
-                                                _ptr(s_V), B, H, L, d, int(bool(causal)), int(scale_block),
-                                                _ptr(O), _stream(stream)), "intfa_attention_fwd_blockscale")
+    L0 = Q_q.shape[2] if isinstance(Q_q, torch.Tensor) and Q_q.dim() == 4 else 0
+    sb = max(int(scale_block), 1)
+    B, H, L, d = _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V, nsc=(L0 + sb - 1) // sb)
+    O = _out(O, (B, H, L, d), torch.float16, Q_q.device, "O")
+    with _on(Q_q.device):
+        _check(lib().intfa_attention_fwd_blockscale(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
+                                                    _ptr(s_V), B, H, L, d, int(bool(causal)), int(scale_block),
+                                                    _ptr(O), _stream(stream)), "intfa_attention_fwd_blockscale")
     return O
 
 
@@ -271,18 +311,22 @@ def intfa_attention_fwd_q16(Q, K_q, Vt_q, s_K, s_V, causal: bool, O=None, s_Q=No
     """Q fp16 [B, H, L, d] (quantised per token inside the kernel); K_q, Vt_q,
     s_K, s_V as for intfa_attention_fwd  ->  O fp16 [B, H, L, d].  If s_Q (fp32
     [B, H, L]) is given, the kernel writes Q's per-token scales into it."""
-    _need(Q, torch.float16, "Q")
-    for t, n in ((K_q, "K_q"), (Vt_q, "Vt_q")):
-        _need(t, torch.int8, n)
-    for t, n in ((s_K, "s_K"), (s_V, "s_V")):
-        _need(t, torch.float32, n)
-    if s_Q is not None:
-        _need(s_Q, torch.float32, "s_Q")
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be [B, H, L, d]")
     B, H, L, d = Q.shape
-    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q.device) if O is None else O
-    _check(lib().intfa_attention_fwd_q16(_ptr(Q), _ptr(K_q), _ptr(Vt_q), _ptr(s_K), _ptr(s_V), B, H, L, d,
-                                         int(bool(causal)), _ptr(O), _ptr(s_Q) if s_Q is not None else None,
-                                         _stream(stream)), "intfa_attention_fwd_q16")
+    dev = Q.device
+    _need(Q, torch.float16, "Q", device=dev)
+    _need(K_q, torch.int8, "K_q", shape=(B, H, L, d), device=dev)
+    _need(Vt_q, torch.int8, "Vt_q", shape=(B, H, d, intfa_vt_ld(L)), device=dev)
+    _need(s_K, torch.float32, "s_K", shape=(B, H, L), device=dev)
+    _need(s_V, torch.float32, "s_V", shape=(B, H), device=dev)
+    if s_Q is not None:
+        _need(s_Q, torch.float32, "s_Q", shape=(B, H, L), device=dev)
+    O = _out(O, (B, H, L, d), torch.float16, dev, "O")
+    with _on(dev):
+        _check(lib().intfa_attention_fwd_q16(_ptr(Q), _ptr(K_q), _ptr(Vt_q), _ptr(s_K), _ptr(s_V), B, H, L, d,
+                                             int(bool(causal)), _ptr(O), _ptr(s_Q) if s_Q is not None else None,
+                                             _stream(stream)), "intfa_attention_fwd_q16")
     return O
 
 
@@ -293,20 +337,25 @@ def intfa_index_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, c: fl
     fp32 [B, H]; clip threshold c and table bits b  ->  O fp16 [B, H, L, d].
     m_out / l_out (int32 [B, H, L], optional) receive the integer row max of
     Q_hat K_hat^T and the integer row sum of the table values."""
-    for t, n in ((Q_q, "Q_q"), (K_q, "K_q"), (Vt_q, "Vt_q")):
-        _need(t, torch.int8, n)
+    if not isinstance(Q_q, torch.Tensor) or Q_q.dim() != 4:
+        raise ValueError("Q_q must be [B, H, L, d]")
+    B, H, L, d = Q_q.shape
+    dev = Q_q.device
+    _need(Q_q, torch.int8, "Q_q", device=dev)
+    _need(K_q, torch.int8, "K_q", shape=(B, H, L, d), device=dev)
+    _need(Vt_q, torch.int8, "Vt_q", shape=(B, H, d, intfa_vt_ld(L)), device=dev)
     for t, n in ((s_Q, "s_Q"), (s_K, "s_K"), (s_V, "s_V")):
-        _need(t, torch.float32, n)
+        _need(t, torch.float32, n, shape=(B, H), device=dev)
     for t, n in ((m_out, "m_out"), (l_out, "l_out")):
         if t is not None:
-            _need(t, torch.int32, n)
-    B, H, L, d = Q_q.shape
-    O = torch.empty((B, H, L, d), dtype=torch.float16, device=Q_q.device) if O is None else O
-    _check(lib().intfa_index_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
-                                           B, H, L, d, int(bool(causal)), float(c), int(b), _ptr(O),
-                                           _ptr(m_out) if m_out is not None else None,
-                                           _ptr(l_out) if l_out is not None else None,
-                                           _stream(stream)), "intfa_index_attention_fwd")
+            _need(t, torch.int32, n, shape=(B, H, L), device=dev)
+    O = _out(O, (B, H, L, d), torch.float16, dev, "O")
+    with _on(dev):
+        _check(lib().intfa_index_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
+                                               B, H, L, d, int(bool(causal)), float(c), int(b), _ptr(O),
+                                               _ptr(m_out) if m_out is not None else None,
+                                               _ptr(l_out) if l_out is not None else None,
+                                               _stream(stream)), "intfa_index_attention_fwd")
     return O
 
 
@@ -314,31 +363,63 @@ def intfa_decode_fwd(q, K_q, s_K, V_q, s_V, splits: int = 1, O=None, workspace=N
     """One query per head against an INT8 cache: q fp16 [B, H, d]; K_q, V_q
     int8 [B, H, L, d] (per-token K codes, per-head V codes); s_K fp32 [B, H, L];
     s_V fp32 [B, H]  ->  O fp16 [B, H, d]."""
-    _need(q, torch.float16, "q")
-    for t, n in ((K_q, "K_q"), (V_q, "V_q")):
-        _need(t, torch.int8, n)
-    for t, n in ((s_K, "s_K"), (s_V, "s_V")):
-        _need(t, torch.float32, n)
+    if not isinstance(K_q, torch.Tensor) or K_q.dim() != 4:
+        raise ValueError("K_q must be [B, H, L, d]")
     B, H, L, d = K_q.shape
-    O = torch.empty((B, H, d), dtype=torch.float16, device=q.device) if O is None else O
-    wsb = int(lib().intfa_decode_workspace_size(B, H, d, int(splits)))
-    if workspace is None:
-        workspace = torch.empty((max(wsb, 16),), dtype=torch.uint8, device=q.device)
-    _check(lib().intfa_decode_fwd(_ptr(q), _ptr(K_q), _ptr(s_K), _ptr(V_q), _ptr(s_V), B, H, L, d, int(splits),
-                                  _ptr(O), _ptr(workspace), workspace.numel(), _stream(stream)),
-           "intfa_decode_fwd")
+    dev = K_q.device
+    _need(q, torch.float16, "q", shape=(B, H, d), device=dev)
+    _need(K_q, torch.int8, "K_q", device=dev)
+    _need(V_q, torch.int8, "V_q", shape=(B, H, L, d), device=dev)
+    _need(s_K, torch.float32, "s_K", shape=(B, H, L), device=dev)
+    _need(s_V, torch.float32, "s_V", shape=(B, H), device=dev)
+    O = _out(O, (B, H, d), torch.float16, dev, "O")
+    workspace = _workspace(workspace, int(lib().intfa_decode_workspace_size(B, H, d, int(splits))), dev)
+    with _on(dev):
+        _check(lib().intfa_decode_fwd(_ptr(q), _ptr(K_q), _ptr(s_K), _ptr(V_q), _ptr(s_V), B, H, L, d,
+                                      int(splits), _ptr(O), _ptr(workspace), workspace.numel(), _stream(stream)),
+               "intfa_decode_fwd")
     return O
 
 
 def intfa_debug_qk(Q_q, K_q, S=None, stream=None):
     """int32 [B, H, L, L] = Q_hat K_hat^T through the tensor-core path."""
-    _need(Q_q, torch.int8, "Q_q")
-    _need(K_q, torch.int8, "K_q")
+    if not isinstance(Q_q, torch.Tensor) or Q_q.dim() != 4:
+        raise ValueError("Q_q must be [B, H, L, d]")
     B, H, L, d = Q_q.shape
-    S = torch.empty((B, H, L, L), dtype=torch.int32, device=Q_q.device) if S is None else S
-    _check(lib().intfa_debug_qk(_ptr(Q_q), _ptr(K_q), B, H, L, d, _ptr(S), _stream(stream)),
-           "intfa_debug_qk")
+    _need(Q_q, torch.int8, "Q_q")
+    _need(K_q, torch.int8, "K_q", shape=(B, H, L, d), device=Q_q.device)
+    S = _out(S, (B, H, L, L), torch.int32, Q_q.device, "S")
+    with _on(Q_q.device):
+        _check(lib().intfa_debug_qk(_ptr(Q_q), _ptr(K_q), B, H, L, d, _ptr(S), _stream(stream)), "intfa_debug_qk")
     return S
+
+
+def intfa_debug_attention_scores(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, S, O=None, stream=None):
+    """intfa_attention_fwd that also writes the integer logits its softmax
+    recovers from the tensor-memory accumulator into S (int32 [B, H, L, L];
+    entries the kernel never computes are left as they are)."""
+    B, H, L, d = _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V)
+    _need(S, torch.int32, "S", shape=(B, H, L, L), device=Q_q.device)
+    O = _out(O, (B, H, L, d), torch.float16, Q_q.device, "O")
+    with _on(Q_q.device):
+        _check(lib().intfa_debug_attention_scores(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
+                                                  _ptr(s_V), B, H, L, d, int(bool(causal)), _ptr(O), _ptr(S),
+                                                  _stream(stream)), "intfa_debug_attention_scores")
+    return O
+
+
+def intfa_debug_wait_timeout(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, cap_cycles: int, O=None, stream=None):
+    """Launch the attention kernel (d = 64) in its test form that issues no
+    copy and no MMA, every wait capped at cap_cycles: each role's wait runs
+    out, the kernel records the wait site and returns (read it with
+    intfa_device_status)."""
+    B, H, L, d = _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V)
+    O = _out(O, (B, H, L, d), torch.float16, Q_q.device, "O")
+    with _on(Q_q.device):
+        _check(lib().intfa_debug_wait_timeout(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K), _ptr(s_V),
+                                              B, H, L, d, int(bool(causal)), _ptr(O), int(cap_cycles),
+                                              _stream(stream)), "intfa_debug_wait_timeout")
+    return O
 
 
 def intfa_forward_workspace_size(B, H, L, d) -> int:
@@ -357,27 +438,32 @@ def intfa_forward_workspace_layout(B, H, L, d) -> list[int]:
 
 def intfa_forward(Q, K, V, causal: bool, O=None, workspace=None, stream=None):
     """fp16 [B, H, L, d] device tensors -> O fp16; quantisation + attention."""
-    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
-        _need(t, torch.float16, n)
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be [B, H, L, d]")
     B, H, L, d = Q.shape
-    O = torch.empty_like(Q) if O is None else O
-    wsb = intfa_forward_workspace_size(B, H, L, d)
-    if workspace is None:
-        workspace = torch.empty((max(wsb, 1),), dtype=torch.uint8, device=Q.device)
-    _check(lib().intfa_forward(_ptr(Q), _ptr(K), _ptr(V), B, H, L, d, int(bool(causal)), _ptr(O),
-                               _ptr(workspace), workspace.numel(), _stream(stream)), "intfa_forward")
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, torch.float16, n, shape=(B, H, L, d), device=Q.device)
+    O = _out(O, (B, H, L, d), torch.float16, Q.device, "O")
+    workspace = _workspace(workspace, intfa_forward_workspace_size(B, H, L, d), Q.device)
+    with _on(Q.device):
+        _check(lib().intfa_forward(_ptr(Q), _ptr(K), _ptr(V), B, H, L, d, int(bool(causal)), _ptr(O),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)), "intfa_forward")
     return O
 
 
 def intfa_forward_host(Q_host, K_host, V_host, causal: bool, O_host, workspace, stream=None):
     """Host (pinned) fp16 tensors in and out; copies run inside the call."""
-    for t, n in ((Q_host, "Q"), (K_host, "K"), (V_host, "V"), (O_host, "O")):
-        if t.is_cuda or t.dtype != torch.float16 or not t.is_contiguous():
-            raise ValueError(f"{n} must be a contiguous fp16 host tensor")
+    if not isinstance(Q_host, torch.Tensor) or Q_host.dim() != 4:
+        raise ValueError("Q must be [B, H, L, d]")
     B, H, L, d = Q_host.shape
-    _check(lib().intfa_forward_host(_ptr(Q_host), _ptr(K_host), _ptr(V_host), B, H, L, d,
-                                    int(bool(causal)), _ptr(O_host), _ptr(workspace),
-                                    workspace.numel(), _stream(stream)), "intfa_forward_host")
+    for t, n in ((Q_host, "Q"), (K_host, "K"), (V_host, "V"), (O_host, "O")):
+        if t.is_cuda or t.dtype != torch.float16 or not t.is_contiguous() or tuple(t.shape) != (B, H, L, d):
+            raise ValueError(f"{n} must be a contiguous fp16 host tensor of shape {(B, H, L, d)}")
+    _need(workspace, torch.uint8, "workspace")
+    with _on(workspace.device):
+        _check(lib().intfa_forward_host(_ptr(Q_host), _ptr(K_host), _ptr(V_host), B, H, L, d,
+                                        int(bool(causal)), _ptr(O_host), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)), "intfa_forward_host")
     return O_host
 
 
