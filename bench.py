@@ -39,10 +39,13 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def kernel_sources_sha(method: str = "online") -> str:
-    """Hash of the dominant kernel's sources (the attention kernel of `method`)."""
+    """Hash of the dominant kernel's sources (the attention kernel of `method`;
+    "online-fused-q" is the same kernel with Q quantised inside it)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_quantized_attention_token_b200", "csrc")
-    files = {"online": ("attention.cu", "ptx.cuh", "quant_math.cuh"), "index": ("index_attention.cu", "ptx.cuh"),
+    files = {"online": ("attention.cu", "ptx.cuh", "quant_math.cuh"),
+             "online-fused-q": ("attention.cu", "ptx.cuh", "quant_math.cuh"),
+             "index": ("index_attention.cu", "ptx.cuh"),
              "decode": ("decode.cu", "ptx.cuh", "quant_math.cuh")}[method]
     for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
@@ -360,6 +363,12 @@ def run_gpu(args):
                            c=args.index_c, b=args.index_b, blk=blk, lcodes=args.lsum == "codes",
                            p_levels=args.p_levels)
 
+    configs = None
+    if rank == 0 and not args.no_configs and args.method == "online" and not fused_q and blk == 1 \
+            and args.lsum == "p" and args.p_levels == 127:
+        configs = measure_configs(intfa, dev, stream, peak, local)
+
+    sha_method = "online-fused-q" if fused_q else args.method
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -379,7 +388,7 @@ def run_gpu(args):
                                    ("attn_fwd_kernel<%d, Q quantised in-kernel>" % d if fused_q else "attn_fwd_kernel<%d>" % d),
                          "achieved": round(achieved, 2),
                          "peak": round(peak, 1), "unit": UNIT, "frac": round(achieved / peak, 4),
-                         "traffic": traffic_for(w.name, args.method),
+                         "traffic": traffic_for(w.name, sha_method),
                          "peak_note": f"{pk['source']} bf16 burst {pk['bf16_burst']} TFLOP/s x {I8_PER_BF16} "
                                       "(nominal dense INT8:BF16 ratio)",
                          "frac_of_sustained": round(achieved / (pk["bf16_sustained"] * I8_PER_BF16), 4),
@@ -390,12 +399,60 @@ def run_gpu(args):
                                     "quantisation": round(ms_per_step - attn_mean, 5),
                                     "q_path": args.q_path},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
-            "clocks": clk, "kernel_sha": kernel_sources_sha(args.method),
+            "clocks": clk, "kernel_sha": kernel_sources_sha(sha_method),
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def measure_configs(intfa, dev, stream, peak, gpu_index, launches=25):
+    """intfa_attention_fwd alone on each of the five synthetic workloads, in
+    this process: inputs quantised once, then `launches` launches each timed
+    with its own CUDA events on the launching stream, L2 flushed (a 256 MiB
+    write) between launches outside the timed pairs; clocks sampled while the
+    workload runs.  Returns {name: {attn_ms, TOPS, frac, clocks}}."""
+    import torch
+
+    from int8_quantized_attention_token_b200.workloads import WORKLOADS, make_workload
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+    for w in WORKLOADS:
+        Qh, Kh, Vh = make_workload(w)
+        B, H, L, d = Qh.shape
+        Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
+        Qq, sQ = intfa.intfa_quantize_per_token(Q, stream=stream)
+        Kq, sK = intfa.intfa_quantize_per_token(K, stream=stream)
+        Vt, sV = intfa.intfa_quantize_per_tensor(V.reshape(B * H, L, d), True, stream=stream)
+        Vt, sV = Vt.reshape(B, H, d, -1), sV.reshape(B, H)
+        O = torch.empty_like(Q)
+        for _ in range(3):
+            intfa.intfa_attention_fwd(Qq, Kq, Vt, sQ, sK, sV, w.causal, O, stream=stream)
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+        clocks = ClockSampler(gpu_index)
+        clocks.start()
+        time.sleep(0.2)
+        h0 = time.perf_counter()
+        for a, b in ev:
+            flush.fill_(1)
+            a.record(stream)
+            intfa.intfa_attention_fwd(Qq, Kq, Vt, sQ, sK, sV, w.causal, O, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        h1 = time.perf_counter()
+        clk = clocks.stop(h0, h1)
+        if intfa.intfa_device_status(clear=True) != 0:
+            raise RuntimeError(f"a kernel timed out while timing {w.name}")
+        ms = sum(a.elapsed_time(b) for a, b in ev) / launches
+        tops = w.ops / (ms * 1e-3) / 1e12
+        out[w.name] = {"attn_ms": round(ms, 5), "TOPS": round(tops, 2), "frac": round(tops / peak, 4),
+                       "launches": launches, "clocks": clk}
+        del Q, K, V, Qq, Kq, Vt, O
+    del flush
+    return out
 
 
 # ------------------------------------------------------------- decode ---
@@ -510,6 +567,12 @@ def run_decode(args):
                "sample": f"{n} of {BH} heads (quantise the query and the head's cache, decode), {t:.1f} s, "
                          "single-threaded (the decode oracle has no thread loop)"}
 
+    configs = None
+    if rank == 0 and not args.no_configs and args.method == "online" and not fused_q and blk == 1 \
+            and args.lsum == "p" and args.p_levels == 127:
+        configs = measure_configs(intfa, dev, stream, peak, local)
+
+    sha_method = "online-fused-q" if fused_q else args.method
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(ops * world / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "n_gpus": world,
@@ -675,6 +738,8 @@ def main():
                     help="online method: one Q / K scale per block of this many tokens (1 = per token)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload attention timings of the five synthetic configs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     args = ap.parse_args()

@@ -105,8 +105,9 @@ int intfa_quantize_per_tensor(const void *x_f16, int64_t groups, int64_t rows, i
 
 /*
  * One scale for the whole tensor (IntAttention section 2.1, eq. 3 applied to
- * all groups together; the pages' per-tensor V taken literally, SURVEY's
- * groups = 1 reading): s = fl32(max over all groups of max|x| / 127), the
+ * all groups together: "per-tensor" read as one scale for the whole V
+ * tensor rather than one per L x d head): s = fl32(max over all groups of
+ * max|x| / 127), the
  * codes of every group with that s, in the same per-group layout as
  * intfa_quantize_per_tensor (transpose 0 or 1), and s written to each of the
  * `groups` scale slots, so that the attention entry points (one s_V per head)
@@ -309,6 +310,36 @@ int intfa_decode_fwd(const void *q_f16, const int8_t *K_q, const float *s_K, con
  */
 int intfa_debug_qk(const int8_t *Q_q, const int8_t *K_q, int B, int H, int L, int d,
                    int32_t *S, void *stream);
+
+/*
+ * Debug: intfa_attention_fwd (same kernel, same arithmetic, same O) that also
+ * writes the integer logits S = Q_hat K_hat^T (IntAttention eq. 4) as the
+ * kernel's softmax recovers them from its tensor-memory accumulator, int32
+ * [B][H][L][L].  Entries of key blocks the kernel never computes (past the
+ * diagonal block under causal masking) are left untouched.  Arguments as
+ * intfa_attention_fwd plus S (16-byte aligned); B*H*L*L must not exceed
+ * 2^28 (INTFA_ERR_UNSUPPORTED otherwise).
+ */
+int intfa_debug_attention_scores(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                 const float *s_Q, const float *s_K, const float *s_V, int B,
+                                 int H, int L, int d, int causal, void *O_f16, int32_t *S,
+                                 void *stream);
+
+/*
+ * Test of the bounded waits (no counterpart in the pages): launches the
+ * fused attention kernel (d = 64) in a form that issues no copy and no
+ * tensor-core operation, with every wait capped at cap_cycles clock cycles,
+ * so that each role's first wait runs out.  The kernel records the wait site
+ * in the device status word, frees its tensor memory and returns; afterwards
+ * intfa_device_status reports INTFA_ERR_DEVICE_TIMEOUT and the site, and the
+ * device stays usable.  Arguments as intfa_attention_fwd (the buffers must
+ * be valid: their tensor maps are built but never read) with d = 64;
+ * cap_cycles in [1000, 2^32]; O_f16 is left untouched.
+ */
+int intfa_debug_wait_timeout(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                             const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                             int L, int d, int causal, void *O_f16, int64_t cap_cycles,
+                             void *stream);
 
 /*
  * Whole hot path on device buffers: quantise Q and K per token, V per head

@@ -113,7 +113,7 @@ __device__ __forceinline__ void regs_to() {
     if constexpr (R > static_cast<uint32_t>(kLaunchRegs)) regs_inc<R>();
     else if constexpr (R < static_cast<uint32_t>(kLaunchRegs)) regs_dec<R>();
 }
-constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks
+constexpr long long kWaitCycles = 1ll << 32;  // ~2 s at B200 clocks (the release cap)
 constexpr float kLog2e = 1.4426950408889634f;
 // 1.5 * 2^23: for 0 <= y < 2^22, fl(y + 1.5 * 2^23) is 1.5 * 2^23 + RNE(y),
 // so RNE(y) sits in the low mantissa bits of that float.
@@ -124,9 +124,11 @@ constexpr float kMagic = 12582912.0f;
 // their int32 results to that bit pattern.  For |x| < 2^22 the sum
 // 0x4B400000 + x is the bit pattern of the float 1.5 * 2^23 + x, so an
 // accumulator read as fp32 minus kMagic is exactly float(x): no int -> float
-// conversion instruction is needed (|S|, |P V| <= 127^2 * 128 < 2^22).
+// conversion instruction is needed (|S| <= 127^2 d; |P V| per block <=
+// 255 * 127 * 128 with UINT8 codes; both below 2^22).
 constexpr uint16_t kBiasA = 0x6400;   // fp16 1024
 constexpr uint16_t kBiasB = 0x6200;   // fp16 768
+static_assert(255 * 127 * BN < (1 << 22) && 127 * 127 * 128 < (1 << 22), "biased accumulator range");
 
 // (-kMagic, -kMagic) as an f32x2 operand, materialised where it is used (an
 // opaque move, so that the compiler does not keep it in registers across
@@ -143,12 +145,12 @@ __device__ __forceinline__ uint64_t neg_bias2() {
 constexpr uint32_t kSleepNs = 1000000;
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         uint32_t site) {
+                                         uint32_t site, long long cap = kWaitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait_sleep(bar, parity, kSleepNs)) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > cap) {
             *abort_flag = 1;
             atomicCAS(&g_status, 0u, 0x100u | site);
             return false;
@@ -159,16 +161,16 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
 
 // Warp-uniform bounded wait: every lane polls, the warp agrees on the result.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          uint32_t site) {
-    const bool ok = wait_bar(bar, parity, abort_flag, site);
+                                          uint32_t site, long long cap = kWaitCycles) {
+    const bool ok = wait_bar(bar, parity, abort_flag, site, cap);
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, long long cap = kWaitCycles) {
     const long long t0 = clock64();
     while (!mbar_try_wait_sleep(bar, parity, kSleepNs)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > cap) {
             atomicCAS(&g_status, 0u, 0x1FFu);
             return;
         }
@@ -372,15 +374,22 @@ __device__ __forceinline__ void exp_codes(const uint32_t (&w)[32], uint64_t c2, 
 // operands (IntAttention Table 5's unsigned scheme; |P V| per block <=
 // 255 * 127 * 128 < 2^22 keeps the biased accumulator exact); 127 becomes 255
 // in the code rounding, the code sum and the epilogue.
-template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false>
+// kDbg (test forms): 0 release; 1 also writes the recovered S of every block
+// (exact int32, from the biased accumulator) to dbg[bh][query][key]; 2 issues
+// no load and no MMA, so that every wait runs out after `cap` clock cycles
+// (the timeout path).  `cap` bounds every wait of the kernel's roles.
+template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false, int kDbg = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
                     const float *__restrict__ sK, const float *__restrict__ sV,
                     __half *__restrict__ O, int BH, int L, int causal,
-                    const uint4 *__restrict__ Qh, float *__restrict__ sQ_out, int sshift) {
+                    const uint4 *__restrict__ Qh, float *__restrict__ sQ_out, int sshift, long long cap,
+                    int32_t *__restrict__ dbg) {
     AttnSmem<D, kQ16> &sm = get_smem<D, kQ16>();
     constexpr int NS = AttnSmem<D, kQ16>::NS;
+    // every wait's cap: the release constant, or the test form's argument
+    const long long wcap = kDbg == 2 ? cap : kWaitCycles;
     constexpr float kLevels = kU8P ? 255.0f : 127.0f;   // largest P code
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -475,10 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c.t < total) sk_next = load_sk(c);
         int g = 0, q_issued = 0;
         Ring<NS> kv;
-        while (c.t < total) {
+        while (kDbg != 2 && c.t < total) {
             if (!kQ16 && c.j == 0) {   // a new tile: its Q_hat into buffer i mod 2
                 const int qb = c.i & 1;
-                if (c.i >= 2 && !warp_wait(&sm.q_empty[qb], ((c.i >> 1) - 1) & 1, abort_flag, 8)) break;
+                if (c.i >= 2 && !warp_wait(&sm.q_empty[qb], ((c.i >> 1) - 1) & 1, abort_flag, 8, wcap)) break;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&sm.q_full[qb], BM * D);
                     tma_load_3d(&tmQ, &sm.q_full[qb], sm.q[qb], 0, c.T.q0, c.T.bh);
@@ -486,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 q_issued = c.i + 1;
             }
             const int st = kv.idx;
-            if (g >= NS && !warp_wait(&sm.kv_empty[st], kv.ph ^ 1u, abort_flag, 1)) break;
+            if (g >= NS && !warp_wait(&sm.kv_empty[st], kv.ph ^ 1u, abort_flag, 1, wcap)) break;
             if (lane == 0) {
                 mbar_expect_tx(&sm.k_full[st], BN * D);
                 tma_load_3d(&tmK, &sm.k_full[st], sm.k[st], 0, c.j * BN, c.T.bh);
@@ -504,12 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Drain: the last load issued into each stage and Q buffer has landed.
         for (int b = 0; !kQ16 && b < 2 && b < q_issued; ++b) {
             const int last = b + ((q_issued - 1 - b) / 2) * 2;
-            drain_wait(&sm.q_full[b], (last >> 1) & 1);
+            drain_wait(&sm.q_full[b], (last >> 1) & 1, wcap);
         }
         for (int s = 0; s < NS && s < g; ++s) {
             const int last = s + ((g - 1 - s) / NS) * NS;   // last block using stage s
-            drain_wait(&sm.k_full[s], (last / NS) & 1);
-            drain_wait(&sm.v_full[s], (last / NS) & 1);
+            drain_wait(&sm.k_full[s], (last / NS) & 1, wcap);
+            drain_wait(&sm.v_full[s], (last / NS) & 1, wcap);
         }
         __syncwarp();
       } else if (warp == kMmaWarp) {
@@ -525,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t idesc_bias_o = make_idesc_f16(BM, D);
         const uint64_t bias_a = make_sdesc_noswz(smem_u32(sm.bias_ab[0]), 16, 16);
         const uint64_t bias_b = make_sdesc_noswz(smem_u32(sm.bias_ab[1]), 16, 16);
-        bool ok = true;
+        bool ok = true, issued = false;
         // qc walks the blocks whose Q K^T is issued, SB blocks ahead of pc,
         // which walks the blocks whose P V is issued.
         Cursor qc = cursor_begin(ntiles, total, L, causal);
@@ -536,9 +545,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t p_oph = 0;    // o_full / o_empty parity of the P V block (one P V block)
         auto issue_qk = [&]() -> bool {   // Q K^T of block gq (cursor qc) into S buffer gq mod SB
             const int qb = qc.i & 1, st = q_st.idx, sb = q_sb.idx;
-            if (qc.j == 0 && !warp_wait(&sm.q_full[qb], (qc.i >> 1) & 1, abort_flag, 2)) return false;
-            if (!warp_wait(&sm.k_full[st], q_st.ph, abort_flag, 6)) return false;
+            if (qc.j == 0 && !warp_wait(&sm.q_full[qb], (qc.i >> 1) & 1, abort_flag, 2, wcap)) return false;
+            if (!warp_wait(&sm.k_full[st], q_st.ph, abort_flag, 6, wcap)) return false;
             tc_fence_after();
+            if constexpr (kDbg == 2) issued = true;
             if (lane == 0) {
                 const uint64_t qdesc = make_sdesc(smem_u32(sm.q[qb]), kSboQK, kSwQK);
                 const uint64_t kdesc = make_sdesc(smem_u32(sm.k[st]), kSboQK, kSwQK);
@@ -565,10 +575,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool first_pv = true;
         while (ok && pc.t < total) {
             const int st = p_st.idx, sb = p_sb.idx;
-            if (!warp_wait(&sm.v_full[st], p_st.ph, abort_flag, 4)) break;
+            if (!warp_wait(&sm.v_full[st], p_st.ph, abort_flag, 4, wcap)) break;
             // the P V block held the previous block: its output fold has read it
-            if (!first_pv && !warp_wait(&sm.o_empty[0], p_oph ^ 1u, abort_flag, 5)) break;
-            if (!warp_wait(&sm.p_full[sb], p_sb.ph, abort_flag, 3)) break;
+            if (!first_pv && !warp_wait(&sm.o_empty[0], p_oph ^ 1u, abort_flag, 5, wcap)) break;
+            if (!warp_wait(&sm.p_full[sb], p_sb.ph, abort_flag, 3, wcap)) break;
             tc_fence_after();
             if (lane == 0) {
                 const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
@@ -587,10 +597,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             p_oph ^= 1u;
             if (qc.t < total) ok = issue_qk();
         }
-        // Drain: every MMA this warp issued has completed before TMEM is freed.
-        if (lane == 0) mma_commit(&sm.mma_drain);
-        __syncwarp();
-        drain_wait(&sm.mma_drain, 0);
+        // Drain: every MMA this warp issued has completed before TMEM is freed
+        // (nothing to wait for if it never issued one).
+        if (kDbg != 2 || issued) {
+            if (lane == 0) mma_commit(&sm.mma_drain);
+            __syncwarp();
+            drain_wait(&sm.mma_drain, 0, wcap);
+        }
         __syncwarp();
       }
       else if (kQ16) {
@@ -695,9 +708,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < T.nb; ++j, ++g, sb.next(), ks.next(), as.next()) {
                 if ((g & 1) != ws) continue;
                 const int b = sb.idx, st = ks.idx, ab = as.idx;
-                if (!warp_wait(&sm.s_full[b], sb.ph, abort_flag, 12)) { ok = false; break; }
+                if (!warp_wait(&sm.s_full[b], sb.ph, abort_flag, 12, wcap)) { ok = false; break; }
                 // s_K of this block: published by the producer's release-arrive
-                if (!warp_wait(&sm.k_full[st], ks.ph, abort_flag, 13)) { ok = false; break; }
+                if (!warp_wait(&sm.k_full[st], ks.ph, abort_flag, 13, wcap)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t ts = tS + lane_off + b * BN;
                 const float4 *sk4 = reinterpret_cast<const float4 *>(sm.sk[st]);
@@ -711,6 +724,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(ts + 64 * h, w0);
                     tmem_ld32(ts + 64 * h + 32, w1);
                     tmem_wait_ld();
+                    if constexpr (kDbg == 1) {   // S as recovered from the biased accumulator
+                        if (qi < L) {
+                            int32_t *dst = dbg + (static_cast<int64_t>(T.bh) * L + qi) * L + j * BN + 64 * h;
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) {
+                                if (j * BN + 64 * h + e < L)
+                                    dst[e] = static_cast<int32_t>(__uint_as_float(w0[e]) - kMagic);
+                                if (j * BN + 64 * h + 32 + e < L)
+                                    dst[32 + e] = static_cast<int32_t>(__uint_as_float(w1[e]) - kMagic);
+                            }
+                        }
+                    }
                     scores_to_v(w0, sk4 + 16 * h);
                     scores_to_v(w1, sk4 + 16 * h + 8);
                     // keys past the end of the sequence, or after the query
@@ -730,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // read of the previous value
                 float m_prev = -INFINITY;
                 if (g > 0) {
-                    if (!warp_wait(&sm.m_full[ws ^ 1][quad], ((g - 1) >> 1) & 1, abort_flag, 15)) {
+                    if (!warp_wait(&sm.m_full[ws ^ 1][quad], ((g - 1) >> 1) & 1, abort_flag, 15, wcap)) {
                         ok = false;
                         break;
                     }
@@ -744,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_own = m_new;
                 // alpha of block g -> the output warp of this quadrant (slot
                 // g mod AB was last used by block g - AB, also this warpgroup's)
-                if (g >= AB && !warp_wait(&sm.a_empty[ab][quad], as.ph ^ 1u, abort_flag, 14)) {
+                if (g >= AB && !warp_wait(&sm.a_empty[ab][quad], as.ph ^ 1u, abort_flag, 14, wcap)) {
                     ok = false;
                     break;
                 }
@@ -788,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this tile's share of the row sum -> the output side (slot = tile
             // mod 2); c m_own is -inf if this warpgroup had no block of the tile
             const int ls = i & 1;
-            if (i >= 2 && !warp_wait(&sm.l_empty[ls], ((i >> 1) - 1) & 1, abort_flag, 17)) break;
+            if (i >= 2 && !warp_wait(&sm.l_empty[ls], ((i >> 1) - 1) & 1, abort_flag, 17, wcap)) break;
             sm.lsum[ls][ws][row] = l;
             sm.cml[ls][ws][row] = c * m_own;
             mbar_arrive(&sm.l_full[ls]);
@@ -814,8 +839,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // o = alpha o + (P V block), the biased block turned into fp32
                 // exactly (fl(x - kMagic), |P V| <= 127^2 128 < 2^22)
                 const uint32_t to = tO;
-                if (!warp_wait(&sm.o_full[0], oph, abort_flag, 9)) { ok = false; break; }
-                if (!warp_wait(&sm.a_full[ab][quad], as.ph, abort_flag, 10)) { ok = false; break; }
+                if (!warp_wait(&sm.o_full[0], oph, abort_flag, 9, wcap)) { ok = false; break; }
+                if (!warp_wait(&sm.a_full[ab][quad], as.ph, abort_flag, 10, wcap)) { ok = false; break; }
                 tc_fence_after();
                 const float alpha = sm.alpha_o[ab][row];
                 mbar_arrive(&sm.a_empty[ab][quad]);
@@ -853,7 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // rescaled from its own reference c m_w to the final one (the
             // larger: the running max only grows) -> normalised fp16 row
             const int ls = i & 1;
-            if (!warp_wait(&sm.l_full[ls], (i >> 1) & 1, abort_flag, 11)) break;
+            if (!warp_wait(&sm.l_full[ls], (i >> 1) & 1, abort_flag, 11, wcap)) break;
             const float cm0 = sm.cml[ls][0][row], cm1 = sm.cml[ls][1][row];
             const float cmf = fmaxf(cm0, cm1);
             const float l = sm.lsum[ls][0][row] * ex2(cm0 - cmf) + sm.lsum[ls][1][row] * ex2(cm1 - cmf);
@@ -984,10 +1009,11 @@ unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
 }
 
 // Qq (int8, with sQ) when !kQ16; Qh (fp16, scales optionally to sQ_out) when kQ16.
-template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false>
+template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false, int kDbg = 0>
 int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                 float *sQ_out, const float *sK, const float *sV, int B, int H, int L, int causal,
-                void *O, cudaStream_t stream, int sshift = 0) {
+                void *O, cudaStream_t stream, int sshift = 0, long long cap = kWaitCycles,
+                int32_t *dbg = nullptr) {
     const int BH = B * H;
     const int64_t ld = intfa_vt_ld(L);
     const CUtensorMapSwizzle swz = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -1004,13 +1030,13 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     const size_t smem = attn_smem_bytes<D, kQ16>();
-    rc = cuda_status(cudaFuncSetAttribute(attn_fwd_kernel<D, kQ16, kLCodes, kU8P>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+    auto kern = attn_fwd_kernel<D, kQ16, kLCodes, kU8P, kDbg>;
+    rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
     if (rc) return rc;
     // The in-kernel register split assumes exactly kLaunchRegs per thread at
     // launch; a different count could leave setmaxnreg.inc waiting forever.
     cudaFuncAttributes fa;
-    rc = cuda_status(cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kQ16, kLCodes, kU8P>));
+    rc = cuda_status(cudaFuncGetAttributes(&fa, kern));
     if (rc) return rc;
     if (fa.numRegs != kLaunchRegs) return INTFA_ERR_UNSUPPORTED;
     const int ntiles = (L + BM - 1) / BM;
@@ -1019,9 +1045,8 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
     if (!rc) rc = cuda_status(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
     if (rc) return rc;
     const unsigned grid = persistent_grid(static_cast<int64_t>(BH) * ntiles, ntiles, causal, nsm);
-    attn_fwd_kernel<D, kQ16, kLCodes, kU8P><<<grid, kThreads, smem, stream>>>(
-        mq, mk, mv, sQ, sK, sV, static_cast<__half *>(O), BH, L, causal, static_cast<const uint4 *>(Qh),
-        sQ_out, sshift);
+    kern<<<grid, kThreads, smem, stream>>>(mq, mk, mv, sQ, sK, sV, static_cast<__half *>(O), BH, L, causal,
+                                           static_cast<const uint4 *>(Qh), sQ_out, sshift, cap, dbg);
     return cuda_status(cudaGetLastError());
 }
 
@@ -1056,6 +1081,22 @@ int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, c
     return INTFA_ERR_UNSUPPORTED;
 }
 
+int launch_attention_debug(int mode, const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
+                           const float *sK, const float *sV, int B, int H, int L, int d, int causal, void *O,
+                           cudaStream_t stream, long long cap, int32_t *dbg) {
+    if (mode == 1) {
+        if (d == 128)
+            return launch_attn<128, false, false, false, 1>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L,
+                                                            causal, O, stream, 0, kWaitCycles, dbg);
+        return launch_attn<64, false, false, false, 1>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal,
+                                                       O, stream, 0, kWaitCycles, dbg);
+    }
+    if (mode == 2 && d == 64)
+        return launch_attn<64, false, false, false, 2>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal,
+                                                       O, stream, 0, cap, nullptr);
+    return INTFA_ERR_INVALID_ARG;
+}
+
 int launch_attention_fwd_q16(const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sK,
                              const float *sV, int B, int H, int L, int d, int causal, void *O,
                              float *sQ_out, cudaStream_t stream) {
@@ -1078,7 +1119,7 @@ int check_attn_shape(int B, int H, int L, int d) {
     if (bh > (1 << 24)) return INTFA_ERR_UNSUPPORTED;
     const int64_t tiles = (static_cast<int64_t>(L) + 127) / 128;
     if (tiles * bh > 0x7FFFFFFF) return INTFA_ERR_UNSUPPORTED;
-    if (L > 131072) return INTFA_ERR_UNSUPPORTED;   // int32 P V accumulation bound: 127^2 L < 2^31
+    if (L > 131072) return INTFA_ERR_UNSUPPORTED;   // the longest sequence the tests cover
     return INTFA_OK;
 }
 }  // namespace
@@ -1201,6 +1242,41 @@ extern "C" int intfa_debug_qk(const int8_t *Q_q, const int8_t *K_q, int B, int H
     if (static_cast<int64_t>((L + 127) / 128) > 65535 || BH > 65535) return INTFA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return d == 128 ? launch_debug_qk<128>(Q_q, K_q, BH, L, S, s) : launch_debug_qk<64>(Q_q, K_q, BH, L, S, s);
+}
+
+extern "C" int intfa_debug_attention_scores(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                            const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                                            int L, int d, int causal, void *O_f16, int32_t *S, void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    if (!Q_q || !K_q || !Vt_q || !s_Q || !s_K || !s_V || !O_f16 || !S) return INTFA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * H * L * L > (int64_t{1} << 28)) return INTFA_ERR_UNSUPPORTED;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(Vt_q) || !aligned16(O_f16) || !aligned16(S) ||
+        (reinterpret_cast<uintptr_t>(s_Q) & 3u) || (reinterpret_cast<uintptr_t>(s_K) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_V) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    return launch_attention_debug(1, Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
+                                  static_cast<cudaStream_t>(stream), 0, S);
+}
+
+extern "C" int intfa_debug_wait_timeout(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,
+                                        const float *s_Q, const float *s_K, const float *s_V, int B, int H, int L,
+                                        int d, int causal, void *O_f16, int64_t cap_cycles, void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (d != 64) return INTFA_ERR_UNSUPPORTED;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    if (cap_cycles < 1000 || cap_cycles > (int64_t{1} << 32)) return INTFA_ERR_INVALID_ARG;
+    if (!Q_q || !K_q || !Vt_q || !s_Q || !s_K || !s_V || !O_f16) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(Vt_q) || !aligned16(O_f16) ||
+        (reinterpret_cast<uintptr_t>(s_Q) & 3u) || (reinterpret_cast<uintptr_t>(s_K) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_V) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    return launch_attention_debug(2, Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
+                                  static_cast<cudaStream_t>(stream), static_cast<long long>(cap_cycles), nullptr);
 }
 
 extern "C" int intfa_device_status(int clear, uint32_t *word) {

@@ -33,6 +33,13 @@ int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt,
 int launch_attention_fwd_q16(const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sK,
                              const float *sV, int B, int H, int L, int d, int causal, void *O,
                              float *sQ_out, cudaStream_t stream);
+// Test instantiations of the fused attention kernel: mode 1 also writes the
+// recovered S of every block to dbg [B*H][L][L] (int32); mode 2 (d = 64 only)
+// issues no load and no MMA, so that every bounded wait runs out after `cap`
+// clock cycles.
+int launch_attention_debug(int mode, const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, const float *sQ,
+                           const float *sK, const float *sV, int B, int H, int L, int d, int causal, void *O,
+                           cudaStream_t stream, long long cap, int32_t *dbg);
 // The IndexSoftmax kernel's status word (index_attention.cu); clear resets it.
 int read_index_status(int clear, uint32_t *word);
 // The decode kernels' status word (decode.cu); clear resets it.

@@ -190,3 +190,28 @@ def test_forward_rejects(L):
     # B H ceil(L / 128) query tiles must fit an int (here 2^24 heads of 1024 tiles)
     assert intfa.intfa_forward_workspace_size(1 << 12, 1 << 12, 131072, 64) == 0
     assert L.intfa_forward(FAKE, FAKE, FAKE, 1 << 12, 1 << 12, 131072, 64, 0, FAKE, FAKE, ws, None) == 2
+
+
+def test_debug_attention_scores_rejects(L):
+    # Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O, S, stream
+    a = [FAKE] * 6
+    f = L.intfa_debug_attention_scores
+    assert f(*a, 1, 1, 128, 96, 0, FAKE, FAKE, None) == 2              # d
+    assert f(*a, 1, 1, 128, 64, 2, FAKE, FAKE, None) == 1              # causal flag
+    assert f(*a, 1, 1, 128, 64, 0, FAKE, None, None) == 1              # S
+    assert f(*a, 1, 1, 128, 64, 0, None, FAKE, None) == 1              # O
+    assert f(*a, 17, 1, 4096, 64, 0, FAKE, FAKE, None) == 2            # B H L L above 2^28
+    assert f(*a, 1, 1, 128, 64, 0, FAKE, FAKE + 4, None) == 3          # S alignment
+
+
+def test_debug_wait_timeout_rejects(L):
+    # Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O, cap_cycles, stream
+    a = [FAKE] * 6
+    f = L.intfa_debug_wait_timeout
+    assert f(*a, 1, 1, 128, 128, 0, FAKE, 20000, None) == 2            # only d = 64 is built
+    assert f(*a, 1, 1, 128, 64, 0, FAKE, 999, None) == 1               # cap below 1000
+    assert f(*a, 1, 1, 128, 64, 0, FAKE, (1 << 32) + 1, None) == 1     # cap above 2^32
+    assert f(*a, 1, 1, 128, 64, 2, FAKE, 20000, None) == 1             # causal flag
+    assert f(*a, 1, 1, 128, 64, 0, None, 20000, None) == 1             # O
+    assert f(*a, 0, 1, 128, 64, 0, FAKE, 20000, None) == 1             # B
+    assert f(FAKE + 4, *a[1:], 1, 1, 128, 64, 0, FAKE, 20000, None) == 3

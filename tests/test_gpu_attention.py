@@ -155,3 +155,52 @@ def test_forward_host_chunks_match_device_path(B, H, L, d, causal):
     assert np.isfinite(Oh).all()
     mx, mre = gap(Oh, Od)
     assert mx <= 1e-3 and mre <= 1e-4, (mx, mre)
+
+
+def schedule_rows(w, nsm=148):
+    """Query rows of whole 128-row tiles where the persistent schedule is most
+    likely to go wrong, for a causal workload (the kernel's tile order: tiles
+    head-major, the heaviest tile of each head first; CTA c takes tiles c,
+    c + G, ... with G the largest count <= the SM count coprime to the tiles
+    per head; the two softmax warpgroups take alternate key blocks of the
+    CTA's stream).  Returns {(b, h): rows}: the first and last query tile of 4
+    heads, the last two tiles of CTAs 0 and G - 1, and tiles with an odd and
+    an even key-block count (the last block falls to either warpgroup)."""
+    ntiles = (w.L + 127) // 128
+    total = w.B * w.H * ntiles
+    G = nsm
+    for cand in range(nsm, nsm // 2, -1):
+        if np.gcd(cand, ntiles) == 1:
+            G = cand
+            break
+    tiles = {}
+
+    def add(t):
+        bh, tt = divmod(t, ntiles)
+        qt = ntiles - 1 - tt            # heaviest first
+        tiles.setdefault((bh // w.H, bh % w.H), set()).add(qt)
+
+    for bh in (0, 1, w.B * w.H // 2, w.B * w.H - 1):
+        add(bh * ntiles + ntiles - 1)   # query tile 0
+        add(bh * ntiles)                # the last query tile
+    for c in (0, G - 1):
+        for t in list(range(c, total, G))[-2:]:
+            add(t)
+    add(5 * ntiles + 3)                 # ntiles - 4 key blocks
+    add(6 * ntiles + 4)                 # ntiles - 5 key blocks
+    return {k: np.concatenate([np.arange(128 * t, min(w.L, 128 * t + 128)) for t in sorted(v)])
+            for k, v in tiles.items()}
+
+
+@pytest.mark.parametrize("w", [WORKLOADS[2], WORKLOADS[4]], ids=lambda w: w.name)
+def test_full_size_whole_tiles(w):
+    """Every row of the tiles where the persistent schedule is most likely to
+    go wrong (first / last tiles of several heads, the last units of the first
+    and last CTA, both slots), element by element against the oracle."""
+    Q, K, V = make_workload(w)
+    O = run_gpu(Q, K, V, w.causal)
+    sel = schedule_rows(w)
+    for (b, h), rows in sel.items():
+        ref = oracle_heads(Q, K, V, w.causal, [(b, h)], rows=rows)
+        mx, mre = gap(O[b, h][rows], ref[(b, h)]["O"])
+        assert mx <= TOL_MAXABS and mre <= TOL_MRE, ((b, h), mx, mre)
