@@ -1,8 +1,8 @@
 """Benchmark of the INT8 attention forward hot path on B200.
 
 One step = the whole path on one batch of synthetic fp16 input already in HBM:
-per-token quantisation of Q and K, per-head quantisation of V (transposed),
-and the fused INT8 attention kernel.  The metric is INT8 attention TOPS:
+per-token quantisation of Q and K, per-head quantisation of V (codes in V's
+own layout), and the fused INT8 attention kernel (V_hat tiles read N-major).  The metric is INT8 attention TOPS:
 4 B H L^2 d ops (halved when causal) per step / step time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
@@ -175,7 +175,8 @@ def run_gpu(args):
     ld = intfa.intfa_vt_ld(L)
     Qq = torch.empty(B, H, L, d, dtype=torch.int8, device=dev)
     Kq = torch.empty_like(Qq)
-    Vt = torch.empty(BH, d, ld, dtype=torch.int8, device=dev)
+    Vt = torch.empty(BH, d, ld, dtype=torch.int8, device=dev)   # V_hat^T for the variant kernels
+    Vr = torch.empty(B, H, L, d, dtype=torch.int8, device=dev)   # V_hat, untransposed
     sQ = torch.empty(B, H, L, dtype=torch.float32, device=dev)
     sK = torch.empty_like(sQ)
     sV = torch.empty(BH, dtype=torch.float32, device=dev)
@@ -237,10 +238,16 @@ def run_gpu(args):
         if not fused_q:
             intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
         intfa.intfa_quantize_per_token(K, Kq, sK, stream=stream)
-        intfa.intfa_quantize_per_tensor(V3, True, Vt, sV, ws, stream=stream)
+        plain = not fused_q and args.p_levels == 127 and args.lsum != "codes"
+        if plain:   # the path of intfa_forward: V_hat untransposed
+            intfa.intfa_quantize_per_tensor(V3, False, Vr.reshape(BH, L, d), sV, ws, stream=stream)
+        else:
+            intfa.intfa_quantize_per_tensor(V3, True, Vt, sV, ws, stream=stream)
         if ev is not None:
             ev[0].record(stream)
-        if fused_q:   # Q quantised per token inside the attention kernel
+        if plain:
+            intfa.intfa_attention_fwd_vrows(Qq, Kq, Vr, sQ, sK, sV.reshape(B, H), w.causal, O, stream=stream)
+        elif fused_q:   # Q quantised per token inside the attention kernel
             intfa.intfa_attention_fwd_q16(Q, Kq, Vt.reshape(B, H, d, ld), sK, sV.reshape(B, H), w.causal, O,
                                           s_Q=sQ, stream=stream)
         elif args.p_levels != 127:   # UINT8 P codes RNE(255 p)
@@ -250,15 +257,12 @@ def run_gpu(args):
         elif args.lsum == "codes":   # row sum from the P codes
             intfa.intfa_attention_fwd_codesum(Qq, Kq, Vt.reshape(B, H, d, ld), sQ, sK, sV.reshape(B, H), w.causal,
                                               O, stream=stream)
-        else:
-            intfa.intfa_attention_fwd(Qq, Kq, Vt.reshape(B, H, d, ld), sQ, sK, sV.reshape(B, H), w.causal, O,
-                                      stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
-    # quantise K, V abs-max, V convert, attention (+ quantise Q when separate);
-    # index: abs-max and convert for each of Q, K, V, and the attention kernel
-    kernels_per_step = 7 if (index or blk > 1) else (4 if fused_q else 5)
+    # one kernel each: quantise Q (unless fused), K and V (both phases of the
+    # per-head quantiser in one kernel), and the attention kernel
+    kernels_per_step = 3 if (fused_q and not index and blk == 1) else 4
 
     for _ in range(args.warmup):
         step()
@@ -409,7 +413,7 @@ def run_gpu(args):
 
 
 def measure_configs(intfa, dev, stream, peak, gpu_index, launches=25):
-    """intfa_attention_fwd alone on each of the five synthetic workloads, in
+    """intfa_attention_fwd_vrows alone on each of the five synthetic workloads, in
     this process: inputs quantised once, then `launches` launches each timed
     with its own CUDA events on the launching stream, L2 flushed (a 256 MiB
     write) between launches outside the timed pairs; clocks sampled while the
@@ -425,11 +429,11 @@ def measure_configs(intfa, dev, stream, peak, gpu_index, launches=25):
         Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
         Qq, sQ = intfa.intfa_quantize_per_token(Q, stream=stream)
         Kq, sK = intfa.intfa_quantize_per_token(K, stream=stream)
-        Vt, sV = intfa.intfa_quantize_per_tensor(V.reshape(B * H, L, d), True, stream=stream)
-        Vt, sV = Vt.reshape(B, H, d, -1), sV.reshape(B, H)
+        Vr, sV = intfa.intfa_quantize_per_tensor(V.reshape(B * H, L, d), False, stream=stream)
+        Vr, sV = Vr.reshape(B, H, L, d), sV.reshape(B, H)
         O = torch.empty_like(Q)
         for _ in range(3):
-            intfa.intfa_attention_fwd(Qq, Kq, Vt, sQ, sK, sV, w.causal, O, stream=stream)
+            intfa.intfa_attention_fwd_vrows(Qq, Kq, Vr, sQ, sK, sV, w.causal, O, stream=stream)
         torch.cuda.synchronize(dev)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
         clocks = ClockSampler(gpu_index)
@@ -439,7 +443,7 @@ def measure_configs(intfa, dev, stream, peak, gpu_index, launches=25):
         for a, b in ev:
             flush.fill_(1)
             a.record(stream)
-            intfa.intfa_attention_fwd(Qq, Kq, Vt, sQ, sK, sV, w.causal, O, stream=stream)
+            intfa.intfa_attention_fwd_vrows(Qq, Kq, Vr, sQ, sK, sV, w.causal, O, stream=stream)
             b.record(stream)
         torch.cuda.synchronize(dev)
         h1 = time.perf_counter()
@@ -450,7 +454,7 @@ def measure_configs(intfa, dev, stream, peak, gpu_index, launches=25):
         tops = w.ops / (ms * 1e-3) / 1e12
         out[w.name] = {"attn_ms": round(ms, 5), "TOPS": round(tops, 2), "frac": round(tops / peak, 4),
                        "launches": launches, "clocks": clk}
-        del Q, K, V, Qq, Kq, Vt, O
+        del Q, K, V, Qq, Kq, Vr, O
     del flush
     return out
 

@@ -169,6 +169,18 @@ int intfa_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q
                         int L, int d, int causal, void *O_f16, void *stream);
 
 /*
+ * The same fused attention with V_hat in its natural layout: V_q int8
+ * [B][H][L][d] (intfa_quantize_per_tensor with groups = B*H and
+ * transpose = 0), 16-byte aligned; every other argument as in
+ * intfa_attention_fwd, and the output is bit-identical to it on the same
+ * codes.  The kernel's P V product reads the V_hat tile N-major, so no
+ * transposed copy of V_hat is made; intfa_forward takes this path.
+ */
+int intfa_attention_fwd_vrows(const int8_t *Q_q, const int8_t *K_q, const int8_t *V_q,
+                              const float *s_Q, const float *s_K, const float *s_V, int B, int H,
+                              int L, int d, int causal, void *O_f16, void *stream);
+
+/*
  * The same fused attention with Q given in fp16: each 128-query tile is
  * quantised per token inside the kernel (IntAttention section 2.1, eq. 3,
  * token-level as INT-FlashAttention's abstract specifies; bit-identical codes
@@ -343,14 +355,16 @@ int intfa_debug_wait_timeout(const int8_t *Q_q, const int8_t *K_q, const int8_t 
 
 /*
  * Whole hot path on device buffers: quantise Q and K per token, V per head
- * (transposed), then the fused attention.  Q, K, V, O: fp16 [B][H][L][d]
+ * (codes kept in V's [B][H][L][d] layout), then the fused attention
+ * (intfa_attention_fwd_vrows).  Q, K, V, O: fp16 [B][H][L][d]
  * device pointers; workspace: intfa_forward_workspace_size(B, H, L, d) bytes of
  * device memory, 256-byte aligned.  Optional outputs of the quantisation live
  * in the workspace at the offsets intfa_forward_workspace_layout reports.
  */
 size_t intfa_forward_workspace_size(int B, int H, int L, int d);
-/* offsets[0..5] = byte offsets of Q_q, K_q, Vt_q, s_Q, s_K, s_V inside the
- * workspace; returns INTFA_OK or INTFA_ERR_INVALID_ARG. */
+/* offsets[0..5] = byte offsets of Q_q, K_q, V_q ([B][H][L][d], untransposed),
+ * s_Q, s_K, s_V inside the workspace; returns INTFA_OK or
+ * INTFA_ERR_INVALID_ARG. */
 int intfa_forward_workspace_layout(int B, int H, int L, int d, size_t offsets[6]);
 int intfa_forward(const void *Q_f16, const void *K_f16, const void *V_f16, int B, int H, int L,
                   int d, int causal, void *O_f16, void *workspace, size_t workspace_bytes,

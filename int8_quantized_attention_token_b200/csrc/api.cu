@@ -8,7 +8,7 @@
 namespace {
 
 struct Layout {
-    size_t q, k, vt, sq, sk, sv, ws, end;       // device workspace of intfa_forward
+    size_t q, k, v, sq, sk, sv, ws, end;        // device workspace of intfa_forward
     size_t hq, hk, hv, ho, host_end;           // + fp16 staging for intfa_forward_host
 };
 
@@ -18,7 +18,6 @@ bool make_layout(int B, int H, int L, int d, Layout *lo) {
     if (bh > (1u << 24) || L > 131072) return false;
     if (bh * ((static_cast<size_t>(L) + 127) / 128) > 0x7FFFFFFFu) return false;   // tile count fits an int
     const size_t n = bh * static_cast<size_t>(L);              // token rows
-    const size_t ld = static_cast<size_t>(intfa_vt_ld(L));
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t at = off;
@@ -27,7 +26,7 @@ bool make_layout(int B, int H, int L, int d, Layout *lo) {
     };
     lo->q = take(n * d);
     lo->k = take(n * d);
-    lo->vt = take(bh * d * ld);
+    lo->v = take(n * d);                                       // V_hat, untransposed
     lo->sq = take(n * sizeof(float));
     lo->sk = take(n * sizeof(float));
     lo->sv = take(bh * sizeof(float));
@@ -71,7 +70,7 @@ extern "C" int intfa_forward_workspace_layout(int B, int H, int L, int d, size_t
     if (!offsets || !make_layout(B, H, L, d, &lo)) return INTFA_ERR_INVALID_ARG;
     offsets[0] = lo.q;
     offsets[1] = lo.k;
-    offsets[2] = lo.vt;
+    offsets[2] = lo.v;
     offsets[3] = lo.sq;
     offsets[4] = lo.sk;
     offsets[5] = lo.sv;
@@ -95,7 +94,7 @@ extern "C" int intfa_forward(const void *Q_f16, const void *K_f16, const void *V
         return INTFA_ERR_MISALIGNED;
     uint8_t *w = static_cast<uint8_t *>(workspace);
     int8_t *k = reinterpret_cast<int8_t *>(w + lo.k);
-    int8_t *vt = reinterpret_cast<int8_t *>(w + lo.vt);
+    int8_t *v = reinterpret_cast<int8_t *>(w + lo.v);
     float *sq = reinterpret_cast<float *>(w + lo.sq);
     float *sk = reinterpret_cast<float *>(w + lo.sk);
     float *sv = reinterpret_cast<float *>(w + lo.sv);
@@ -108,8 +107,9 @@ extern "C" int intfa_forward(const void *Q_f16, const void *K_f16, const void *V
     int8_t *q = reinterpret_cast<int8_t *>(w + lo.q);
     int rc = launch_quantize_per_token(Q_f16, rows, d, q, sq, s);
     if (!rc) rc = launch_quantize_per_token(K_f16, rows, d, k, sk, s);
-    if (!rc) rc = launch_quantize_per_tensor(V_f16, bh, L, d, 1, vt, sv, w + lo.ws, s);
-    if (!rc) rc = launch_attention_fwd(q, k, vt, sq, sk, sv, B, H, L, d, causal, O_f16, s);
+    // V_hat stays in V's layout: the attention reads its tiles N-major
+    if (!rc) rc = launch_quantize_per_tensor(V_f16, bh, L, d, 0, v, sv, w + lo.ws, s);
+    if (!rc) rc = launch_attention_fwd_vrows(q, k, v, sq, sk, sv, B, H, L, d, causal, O_f16, s);
     return rc;
 }
 
@@ -186,7 +186,6 @@ extern "C" int intfa_forward_host(const void *Q_f16_host, const void *K_f16_host
     uint8_t *w = static_cast<uint8_t *>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t bh = static_cast<int64_t>(B) * H;
-    const int64_t ld = intfa_vt_ld(L);
     const size_t head_bytes = static_cast<size_t>(L) * d * 2;   // fp16 of one head
     const int64_t hc = heads_per_chunk(bh, static_cast<int64_t>(head_bytes));
     // Heads are independent: chunk c's host-to-device copies (stream h2d),
@@ -211,15 +210,15 @@ extern "C" int intfa_forward_host(const void *Q_f16_host, const void *K_f16_host
         const int64_t rows = nh * L, r0 = h0 * L;
         int8_t *q = reinterpret_cast<int8_t *>(w + lo.q) + r0 * d;
         int8_t *k = reinterpret_cast<int8_t *>(w + lo.k) + r0 * d;
-        int8_t *vt = reinterpret_cast<int8_t *>(w + lo.vt) + h0 * d * ld;
+        int8_t *v = reinterpret_cast<int8_t *>(w + lo.v) + r0 * d;
         float *sq = reinterpret_cast<float *>(w + lo.sq) + r0;
         float *sk = reinterpret_cast<float *>(w + lo.sk) + r0;
         float *sv = reinterpret_cast<float *>(w + lo.sv) + h0;
         if (!rc) rc = launch_quantize_per_token(w + lo.hq + off, rows, d, q, sq, s);
         if (!rc) rc = launch_quantize_per_token(w + lo.hk + off, rows, d, k, sk, s);
-        if (!rc) rc = launch_quantize_per_tensor(w + lo.hv + off, nh, L, d, 1, vt, sv, w + lo.ws, s);
-        if (!rc) rc = launch_attention_fwd(q, k, vt, sq, sk, sv, 1, static_cast<int>(nh), L, d, causal,
-                                           w + lo.ho + off, s);
+        if (!rc) rc = launch_quantize_per_tensor(w + lo.hv + off, nh, L, d, 0, v, sv, w + lo.ws, s);
+        if (!rc) rc = launch_attention_fwd_vrows(q, k, v, sq, sk, sv, 1, static_cast<int>(nh), L, d, causal,
+                                                 w + lo.ho + off, s);
         if (!rc) rc = cuda_status(cudaEventRecord(pipe.out, s));
         if (!rc) rc = cuda_status(cudaStreamWaitEvent(pipe.d2h, pipe.out, 0));
         if (!rc) rc = cuda_status(cudaMemcpyAsync(static_cast<uint8_t *>(O_f16_host) + off, w + lo.ho + off, bytes,

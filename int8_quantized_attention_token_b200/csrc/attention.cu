@@ -378,7 +378,7 @@ __device__ __forceinline__ void exp_codes(const uint32_t (&w)[32], uint64_t c2, 
 // (exact int32, from the biased accumulator) to dbg[bh][query][key]; 2 issues
 // no load and no MMA, so that every wait runs out after `cap` clock cycles
 // (the timeout path).  `cap` bounds every wait of the kernel's roles.
-template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false, int kDbg = 0>
+template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false, int kDbg = 0, bool kVRow = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const float *__restrict__ sQ,
@@ -500,7 +500,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_expect_tx(&sm.k_full[st], BN * D);
                 tma_load_3d(&tmK, &sm.k_full[st], sm.k[st], 0, c.j * BN, c.T.bh);
                 mbar_arrive_expect_tx(&sm.v_full[st], D * BN);
-                tma_load_3d(&tmV, &sm.v_full[st], sm.v[st], c.j * BN, 0, c.T.bh);
+                if constexpr (kVRow)   // BN rows of V_hat, D bytes each
+                    tma_load_3d(&tmV, &sm.v_full[st], sm.v[st], 0, c.j * BN, c.T.bh);
+                else                   // D rows of V_hat^T, BN bytes each
+                    tma_load_3d(&tmV, &sm.v_full[st], sm.v[st], c.j * BN, 0, c.T.bh);
             }
             *reinterpret_cast<float4 *>(&sm.sk[st][4 * lane]) = sk_next;
             mbar_arrive(&sm.k_full[st]);   // 32 arrivals + the K tile's bytes
@@ -526,7 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kSwQK = (D == 128) ? kSwizzle128B : kSwizzle64B;
         constexpr uint32_t kSboQK = 8 * D;      // 8 rows of D bytes
         const uint32_t idesc_qk = make_idesc_i8(BM, BN);
-        const uint32_t idesc_pv = kU8P ? make_idesc_u8s8(BM, D) : make_idesc_i8(BM, D);
+        // kVRow: B = the V_hat tile as stored, [BN keys][D], read N-major
+        // (bit 16 of the instruction descriptor: B is MN-major)
+        const uint32_t idesc_pv = (kU8P ? make_idesc_u8s8(BM, D) : make_idesc_i8(BM, D)) | (kVRow ? (1u << 16) : 0u);
         // bias MMA operands: every element of A and B is the same constant, so
         // the descriptors may let core matrices overlap (16-byte strides keep
         // all reads inside the 384-byte arrays)
@@ -581,11 +586,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(&sm.p_full[sb], p_sb.ph, abort_flag, 3, wcap)) break;
             tc_fence_after();
             if (lane == 0) {
-                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
+                // K-major V_hat^T: 8-row groups of BN bytes, keys 32k.. at byte 32k
+                // of each row.  N-major V_hat: the swizzle atom is 8 keys x D
+                // bytes (one atom spans N = D), atoms 8 D bytes apart along K,
+                // keys 32k.. start 32 k D bytes into the tile.
+                const uint64_t vdesc = kVRow ? make_sdesc(smem_u32(sm.v[st]), kSboQK, kSwQK)
+                                             : make_sdesc(smem_u32(sm.v[st]), 8 * BN, kSwizzle128B);
+                constexpr uint64_t kVStep = kVRow ? (32 * D) >> 4 : 32 >> 4;   // 16-byte units
                 mma_f16_ss(tO, bias_a, bias_b, idesc_bias_o, 0);
 #pragma unroll
                 for (int k = 0; k < BN / 32; ++k)   // codes of keys 32k .. 32k + 31 at column 32k
-                    mma_i8_ts(tO, tS + sb * BN + 32 * k, vdesc + 2 * k, idesc_pv, 1);
+                    mma_i8_ts(tO, tS + sb * BN + 32 * k, vdesc + kVStep * k, idesc_pv, 1);
                 mma_commit(&sm.o_full[0]);
                 mma_commit(&sm.kv_empty[st]);
             }
@@ -1009,7 +1020,7 @@ unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
 }
 
 // Qq (int8, with sQ) when !kQ16; Qh (fp16, scales optionally to sQ_out) when kQ16.
-template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false, int kDbg = 0>
+template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false, int kDbg = 0, bool kVRow = false>
 int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                 float *sQ_out, const float *sK, const float *sV, int B, int H, int L, int causal,
                 void *O, cudaStream_t stream, int sshift = 0, long long cap = kWaitCycles,
@@ -1026,11 +1037,16 @@ int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t
         else
             rc = make_map(&mq, Qq, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BM, swz);
     }
-    if (!rc) rc = make_map(&mv, Vt, ld, D, BH, ld, static_cast<uint64_t>(ld) * D, BN, D,
-                           CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!rc) {
+        if (kVRow)   // V_hat [BH][L][D], tiles of BN rows like K_hat's
+            rc = make_map(&mv, Vt, D, L, BH, D, static_cast<uint64_t>(L) * D, D, BN, swz);
+        else         // V_hat^T [BH][D][ld], tiles of D rows of BN keys
+            rc = make_map(&mv, Vt, ld, D, BH, ld, static_cast<uint64_t>(ld) * D, BN, D,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     if (rc) return rc;
     const size_t smem = attn_smem_bytes<D, kQ16>();
-    auto kern = attn_fwd_kernel<D, kQ16, kLCodes, kU8P, kDbg>;
+    auto kern = attn_fwd_kernel<D, kQ16, kLCodes, kU8P, kDbg, kVRow>;
     rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
     if (rc) return rc;
     // The in-kernel register split assumes exactly kLaunchRegs per thread at
@@ -1078,6 +1094,18 @@ int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt, c
     if (d == 64)
         return launch_attn<64, false>(Qq, nullptr, Kq, Vt, sQ, nullptr, sK, sV, B, H, L, causal, O, stream,
                                       sshift);
+    return INTFA_ERR_UNSUPPORTED;
+}
+
+int launch_attention_fwd_vrows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq, const float *sQ,
+                               const float *sK, const float *sV, int B, int H, int L, int d, int causal,
+                               void *O, cudaStream_t stream) {
+    if (d == 128)
+        return launch_attn<128, false, false, false, 0, true>(Qq, nullptr, Kq, Vq, sQ, nullptr, sK, sV, B, H, L,
+                                                              causal, O, stream);
+    if (d == 64)
+        return launch_attn<64, false, false, false, 0, true>(Qq, nullptr, Kq, Vq, sQ, nullptr, sK, sV, B, H, L,
+                                                             causal, O, stream);
     return INTFA_ERR_UNSUPPORTED;
 }
 
@@ -1138,6 +1166,22 @@ extern "C" int intfa_attention_fwd(const int8_t *Q_q, const int8_t *K_q, const i
         return INTFA_ERR_MISALIGNED;
     return launch_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
                                 static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int intfa_attention_fwd_vrows(const int8_t *Q_q, const int8_t *K_q, const int8_t *V_q,
+                                         const float *s_Q, const float *s_K, const float *s_V, int B,
+                                         int H, int L, int d, int causal, void *O_f16, void *stream) {
+    using namespace intfa;
+    int rc = check_attn_shape(B, H, L, d);
+    if (rc) return rc;
+    if (causal != 0 && causal != 1) return INTFA_ERR_INVALID_ARG;
+    if (!Q_q || !K_q || !V_q || !s_Q || !s_K || !s_V || !O_f16) return INTFA_ERR_INVALID_ARG;
+    if (!aligned16(Q_q) || !aligned16(K_q) || !aligned16(V_q) || !aligned16(O_f16) ||
+        (reinterpret_cast<uintptr_t>(s_Q) & 3u) || (reinterpret_cast<uintptr_t>(s_K) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_V) & 3u))
+        return INTFA_ERR_MISALIGNED;
+    return launch_attention_fwd_vrows(Q_q, K_q, V_q, s_Q, s_K, s_V, B, H, L, d, causal, O_f16,
+                                      static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int intfa_attention_fwd_blockscale(const int8_t *Q_q, const int8_t *K_q, const int8_t *Vt_q,

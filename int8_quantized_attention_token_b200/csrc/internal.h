@@ -30,6 +30,10 @@ int launch_quantize_per_tensor(const void *x, int64_t groups, int64_t rows, int 
 int launch_attention_fwd(const int8_t *Qq, const int8_t *Kq, const int8_t *Vt,
                          const float *sQ, const float *sK, const float *sV, int B, int H, int L,
                          int d, int causal, void *O, cudaStream_t stream, int sshift = 0);
+// Same, with V_hat in its natural layout Vq [B][H][L][d] (no transpose).
+int launch_attention_fwd_vrows(const int8_t *Qq, const int8_t *Kq, const int8_t *Vq, const float *sQ,
+                               const float *sK, const float *sV, int B, int H, int L, int d, int causal,
+                               void *O, cudaStream_t stream);
 int launch_attention_fwd_q16(const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sK,
                              const float *sV, int B, int H, int L, int d, int causal, void *O,
                              float *sQ_out, cudaStream_t stream);

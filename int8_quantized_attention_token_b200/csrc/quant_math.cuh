@@ -16,6 +16,9 @@ namespace intfa {
 namespace qmath {
 
 constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+// Rounding residuals beyond this magnitude (within 2^-14 of a half-integer)
+// send an element to the IEEE quotient; see quantize.cu's header comment.
+constexpr float kNearTie = 0.5f - 1.0f / 16384.0f;
 
 // fl32(a / 127) for fp16 magnitudes a (see the header comment).
 __device__ __forceinline__ float div127(float a) {
@@ -38,7 +41,7 @@ __device__ __forceinline__ uint32_t code_bits(float x, float s, float r) {
     const float y = x * r;
     float t = y + kRound;
     const float res = y - (t - kRound);
-    if (fabsf(res) > 0.499f) t = __fdiv_rn(x, s) + kRound;
+    if (fabsf(res) > kNearTie) t = __fdiv_rn(x, s) + kRound;
     return __float_as_uint(t);
 }
 

@@ -51,6 +51,7 @@ def lib():
         "intfa_quantize_global": ([P, I64, I64, I, I, P, P, P, SZ, P], I),
         "intfa_quantize_per_tensor_noalloc": ([P, I64, I64, I, I, P, P, P], I),
         "intfa_attention_fwd": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
+        "intfa_attention_fwd_vrows": ([P, P, P, P, P, P, I, I, I, I, I, P, P], I),
         "intfa_attention_fwd_q16": ([P, P, P, P, P, I, I, I, I, I, P, P, P], I),
         "intfa_debug_qk": ([P, P, I, I, I, I, P, P], I),
         "intfa_debug_attention_scores": ([P, P, P, P, P, P, I, I, I, I, I, P, P, P], I),
@@ -238,9 +239,10 @@ def intfa_quantize_per_tensor_noalloc(x: torch.Tensor, transpose: bool = False, 
     return x_q, scale
 
 
-def _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V, nsc=None):
+def _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V, nsc=None, vrows=False):
     """Check the fused attention's inputs against Q_q's shape [B, H, L, d] and
-    device; nsc = scales per head of s_Q / s_K (L unless per-block)."""
+    device; nsc = scales per head of s_Q / s_K (L unless per-block); vrows:
+    V_hat as [B, H, L, d] rather than transposed."""
     if not isinstance(Q_q, torch.Tensor) or Q_q.dim() != 4:
         raise ValueError("Q_q must be [B, H, L, d]")
     B, H, L, d = Q_q.shape
@@ -248,7 +250,10 @@ def _attn_inputs(Q_q, K_q, Vt_q, s_Q, s_K, s_V, nsc=None):
     nsc = L if nsc is None else nsc
     _need(Q_q, torch.int8, "Q_q", device=dev)
     _need(K_q, torch.int8, "K_q", shape=(B, H, L, d), device=dev)
-    _need(Vt_q, torch.int8, "Vt_q", shape=(B, H, d, intfa_vt_ld(L)), device=dev)
+    if vrows:
+        _need(Vt_q, torch.int8, "V_q", shape=(B, H, L, d), device=dev)
+    else:
+        _need(Vt_q, torch.int8, "Vt_q", shape=(B, H, d, intfa_vt_ld(L)), device=dev)
     _need(s_Q, torch.float32, "s_Q", shape=(B, H, nsc), device=dev)
     _need(s_K, torch.float32, "s_K", shape=(B, H, nsc), device=dev)
     _need(s_V, torch.float32, "s_V", shape=(B, H), device=dev)
@@ -264,6 +269,17 @@ def intfa_attention_fwd(Q_q, K_q, Vt_q, s_Q, s_K, s_V, causal: bool, O=None, str
         _check(lib().intfa_attention_fwd(_ptr(Q_q), _ptr(K_q), _ptr(Vt_q), _ptr(s_Q), _ptr(s_K),
                                          _ptr(s_V), B, H, L, d, int(bool(causal)), _ptr(O),
                                          _stream(stream)), "intfa_attention_fwd")
+    return O
+
+
+def intfa_attention_fwd_vrows(Q_q, K_q, V_q, s_Q, s_K, s_V, causal: bool, O=None, stream=None):
+    """intfa_attention_fwd with V_q int8 [B, H, L, d] (V_hat untransposed)."""
+    B, H, L, d = _attn_inputs(Q_q, K_q, V_q, s_Q, s_K, s_V, vrows=True)
+    O = _out(O, (B, H, L, d), torch.float16, Q_q.device, "O")
+    with _on(Q_q.device):
+        _check(lib().intfa_attention_fwd_vrows(_ptr(Q_q), _ptr(K_q), _ptr(V_q), _ptr(s_Q), _ptr(s_K),
+                                               _ptr(s_V), B, H, L, d, int(bool(causal)), _ptr(O),
+                                               _stream(stream)), "intfa_attention_fwd_vrows")
     return O
 
 

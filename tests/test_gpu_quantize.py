@@ -39,11 +39,13 @@ def test_per_token_empty():
 
 @pytest.mark.parametrize("transpose", [False, True])
 @pytest.mark.parametrize("groups,rows,cols", [(1, 1, 64), (3, 129, 64), (4, 1000, 128), (2, 77, 8),
-                                              (5, 4096, 128), (1, 33, 256)])
+                                              (5, 4096, 128), (1, 33, 256), (2, 1300, 32),
+                                              (3, 2500, 64)])
 def test_per_tensor_bit_exact(groups, rows, cols, transpose):
     g = torch.Generator().manual_seed(groups * 7 + rows + cols)
     x = (torch.randn(groups, rows, cols, generator=g) * 3).half()
     x[0, 0, 0] = 0.0
+    x[0, -1, -1] = 50.0                                       # the maximum in the last row tile
     if groups > 1:
         x[1] = 0.0                                            # an all-zero group
     q, s = intfa.intfa_quantize_per_tensor(x.cuda(), transpose=transpose)
@@ -57,6 +59,59 @@ def test_per_tensor_bit_exact(groups, rows, cols, transpose):
         assert not q[:, :, rows:].any()                       # padding codes are zero
     else:
         np.testing.assert_array_equal(q, qo)
+
+
+def near_tie_values(amax):
+    """Every non-negative finite fp16 x <= amax whose IEEE quotient x / s
+    (s = fl32(amax / 127)) lies within 2e-3 of a half-integer, both signs: a
+    superset of the elements the kernels' fast rounding leaves to the IEEE
+    quotient, and of the exact ties."""
+    h = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    h = h[h <= np.float32(amax)]
+    s = np.float32(np.float32(amax) / np.float32(127.0))
+    q = h / s
+    near = h[np.abs(q - np.floor(q) - np.float32(0.5)) < np.float32(2e-3)]
+    assert near.size > 0
+    return np.concatenate([near, -near])
+
+
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("amax", [127.0, 100.0, 1.0, 0.0999755859375, 3.0517578125e-05])
+def test_per_tensor_near_ties(amax, transpose):
+    vals = near_tie_values(amax)
+    cols = 128
+    rows = max(300, -(-(vals.size + 1) // cols))
+    rng = np.random.default_rng(11)
+    x = (rng.uniform(-1, 1, (2, rows, cols)) * amax).astype(np.float16).astype(np.float32)
+    flat = x[0].reshape(-1)
+    flat[-1] = amax                                           # the maximum in the last row tile
+    flat[: vals.size] = vals
+    x[1] = np.roll(x[0], 77 * cols + 5)
+    xh = torch.from_numpy(x).half()
+    q, s = intfa.intfa_quantize_per_tensor(xh.cuda(), transpose=transpose)
+    qo, so = oracle.quantize_per_tensor(xh.float().numpy(), 2)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    q = q.cpu().numpy()
+    if transpose:
+        q = q[:, :, :rows].transpose(0, 2, 1)
+    np.testing.assert_array_equal(q, qo)
+
+
+@pytest.mark.parametrize("amax", [127.0, 100.0, 0.0999755859375])
+def test_per_token_near_ties(amax):
+    vals = near_tie_values(amax)
+    d = 128
+    n = -(-vals.size // (d - 1))
+    x = np.zeros((n, d), np.float32)
+    x[:, 0] = amax
+    body = np.zeros(n * (d - 1), np.float32)
+    body[: vals.size] = vals
+    x[:, 1:] = body.reshape(n, d - 1)
+    xh = torch.from_numpy(x).half()
+    q, s = intfa.intfa_quantize_per_token(xh.cuda())
+    qo, so = oracle.quantize_per_token(xh.float().numpy())
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
 
 
 @pytest.mark.parametrize("w", [WORKLOADS[2], WORKLOADS[3]], ids=lambda w: w.name)

@@ -1,0 +1,57 @@
+"""The fused attention with V_hat read in its natural [B, H, L, d] layout (the
+P V product takes the V_hat tile N-major) against the transposed-V form and
+the oracle: the INT32 P V products are exact either way, so the two GPU
+outputs must agree bit for bit on the same codes, and the per-head V codes of
+both quantiser layouts must be each other's transpose."""
+import numpy as np
+import pytest
+import torch
+
+from int8_quantized_attention_token_b200 import intfa
+from int8_quantized_attention_token_b200.workloads import WORKLOADS, make_qkv, make_workload
+from parity import TOL_MAXABS, TOL_MRE, gap, oracle_heads
+
+pytestmark = pytest.mark.gpu
+
+
+def both_layouts(Q, K, V, causal):
+    B, H, L, d = Q.shape
+    Qq, sQ = intfa.intfa_quantize_per_token(Q.cuda())
+    Kq, sK = intfa.intfa_quantize_per_token(K.cuda())
+    Vd = V.cuda().reshape(B * H, L, d)
+    Vt, sVt = intfa.intfa_quantize_per_tensor(Vd, transpose=True)
+    Vr, sVr = intfa.intfa_quantize_per_tensor(Vd, transpose=False)
+    assert torch.equal(sVt.view(torch.int32), sVr.view(torch.int32))
+    assert torch.equal(Vt[:, :, :L].transpose(1, 2), Vr)
+    Ot = intfa.intfa_attention_fwd(Qq, Kq, Vt.reshape(B, H, d, -1), sQ, sK, sVt.reshape(B, H), causal)
+    Or = intfa.intfa_attention_fwd_vrows(Qq, Kq, Vr.reshape(B, H, L, d), sQ, sK, sVr.reshape(B, H), causal)
+    torch.cuda.synchronize()
+    assert intfa.intfa_device_status(clear=True) == 0
+    return Ot, Or
+
+
+@pytest.mark.parametrize("B,H,L,d,causal", [
+    (1, 1, 1, 64, False),
+    (1, 1, 17, 128, True),
+    (1, 2, 128, 64, True),
+    (2, 3, 333, 64, False),
+    (2, 3, 333, 128, True),
+    (1, 2, 1000, 128, True),
+    (1, 1, 640, 64, True),
+])
+def test_vrows_bit_identical_and_oracle(B, H, L, d, causal):
+    Q, K, V = make_qkv(B, H, L, d, seed=7 * L + d + causal)
+    Ot, Or = both_layouts(Q, K, V, causal)
+    assert torch.equal(Ot.view(torch.int16), Or.view(torch.int16))
+    heads = [(b, h) for b in range(B) for h in range(H)]
+    ref = oracle_heads(Q, K, V, causal, heads)
+    O = Or.float().cpu().numpy()
+    mx, mre = gap(np.stack([O[b, h] for b, h in heads]), np.stack([ref[k]["O"] for k in heads]))
+    assert mx <= TOL_MAXABS and mre <= TOL_MRE, (mx, mre)
+
+
+@pytest.mark.parametrize("w", [WORKLOADS[2], WORKLOADS[4]], ids=lambda w: w.name)
+def test_vrows_bit_identical_full_size(w):
+    Q, K, V = make_workload(w)
+    Ot, Or = both_layouts(Q, K, V, w.causal)
+    assert torch.equal(Ot.view(torch.int16), Or.view(torch.int16))
