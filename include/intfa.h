@@ -138,7 +138,10 @@ int intfa_quantize_global(const void *x_f16, int64_t groups, int64_t rows, int c
  * the call clears what it needs before use, but calls that overlap on the GPU
  * (on different streams, or from several threads without ordering) race on it
  * and give wrong results -- serialise them.  Nothing here calls cudaMalloc,
- * cudaFree or any allocating routine.
+ * cudaFree or any allocating routine.  The looked-up address is kept for the
+ * life of the process: after cudaDeviceReset on a device the library must not
+ * be used on that device again in the same process (the module may load at
+ * another address; the same holds for intfa_forward_host's copy streams).
  */
 #define INTFA_NOALLOC_MAX_GROUPS 4096
 int intfa_quantize_per_tensor_noalloc(const void *x_f16, int64_t groups, int64_t rows, int cols,

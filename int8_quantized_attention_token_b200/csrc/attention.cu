@@ -20,8 +20,10 @@
 // the loads and Q K^T of the next tile overlap the last blocks and the
 // epilogue of the current one.  16 warps:
 //   role 12     TMA producer: each tile's Q_hat (two Q buffers), K_hat tile,
-//               V_hat^T tile and the block's s_K values into a 5-stage
-//               shared-memory ring.
+//               V_hat tile and the block's s_K values into a 5-stage
+//               shared-memory ring.  V_hat comes either as stored, [L][d]
+//               (kVRow: the P V product reads the tile N-major), or
+//               transposed, [d][Lv] (K-major).
 //   role 13     tensor-core issuer (one lane): S = Q K^T with tcgen05.mma
 //               kind::i8 into one of three TMEM S buffers, three key blocks
 //               ahead of P V; P V with the P codes read straight from TMEM
@@ -185,7 +187,7 @@ struct alignas(1024) AttnSmem {
     uint8_t q[2][BM * D];       // Q_hat tiles (two query tiles in flight), K-major, TMA-swizzled
     uint8_t qs[kQ16 ? kQHalf * D * 2 : 1024];   // half an fp16 Q tile for the in-kernel quantiser
     uint8_t k[NS][BN * D];      // K_hat tiles
-    uint8_t v[NS][D * BN];      // V_hat^T tiles (row = channel, 128 keys)
+    uint8_t v[NS][D * BN];      // V_hat tiles: 128 keys x D (kVRow) or D channels x 128 keys
     float sk[NS][BN];           // s_K of each key block
     float mrow[2][BM];          // softmax warpgroup w -> the other: running max after its latest block
     float alpha_o[AB][BM];      // softmax -> output: alpha of block g (slot g mod AB)
@@ -1020,6 +1022,7 @@ unsigned persistent_grid(int64_t total, int ntiles, int causal, int nsm) {
 }
 
 // Qq (int8, with sQ) when !kQ16; Qh (fp16, scales optionally to sQ_out) when kQ16.
+// Vt: V_hat^T [BH][D][ld], or V_hat [BH][L][D] when kVRow.
 template <int D, bool kQ16, bool kLCodes = false, bool kU8P = false, int kDbg = 0, bool kVRow = false>
 int launch_attn(const int8_t *Qq, const void *Qh, const int8_t *Kq, const int8_t *Vt, const float *sQ,
                 float *sQ_out, const float *sK, const float *sV, int B, int H, int L, int causal,
