@@ -299,6 +299,39 @@ def run_gpu(args):
     ms_per_step = elapsed_ms / args.steps
     value = w.ops * world * args.steps / (elapsed_ms * 1e-3) / 1e12
     attn_mean = sum(attn_ms) / len(attn_ms)
+
+    # The same K-step region timed again, back to back, until about a second
+    # of device time has passed (at most 50 regions): evidence that the
+    # headline region above is typical, with clocks sampled over all of them.
+    # Every rank runs the same number of regions (from the max-over-ranks time).
+    repeats = None
+    if not args.no_repeats:
+        nreg = int(max(1, min(50, 1000.0 // max(elapsed_ms, 1e-3))))
+        reg_ms = []
+        rclocks = ClockSampler(local)
+        rclocks.start()
+        time.sleep(0.3)
+        r_h0 = time.perf_counter()
+        for _ in range(nreg):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            r0.record(stream)
+            for _ in range(args.steps):
+                step()
+            r1.record(stream)
+            torch.cuda.synchronize(dev)
+            reg_ms.append(max_over_ranks(r0.elapsed_time(r1), dev) / args.steps)
+        r_h1 = time.perf_counter()
+        time.sleep(0.1)
+        rclk = rclocks.stop(r_h0, r_h1)
+        if intfa.intfa_device_status(clear=True) != 0:
+            raise RuntimeError("a kernel timed out during the repeated regions")
+        repeats = {"regions": nreg, "steps_each": args.steps,
+                   "ms_per_step_median": round(statistics.median(reg_ms), 5),
+                   "ms_per_step_min": round(min(reg_ms), 5), "ms_per_step_max": round(max(reg_ms), 5),
+                   "clocks": rclk}
     achieved = w.ops / (attn_mean * 1e-3) / 1e12
     pk = peaks()
     peak = pk["bf16_burst"] * I8_PER_BF16
@@ -404,6 +437,7 @@ def run_gpu(args):
                                     "q_path": args.q_path},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk, "kernel_sha": kernel_sources_sha(sha_method),
+            "repeats": repeats,
             "configs": configs,
         }
         print(json.dumps(line), flush=True)
@@ -742,6 +776,8 @@ def main():
                     help="online method: one Q / K scale per block of this many tokens (1 = per token)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-repeats", action="store_true",
+                    help="skip re-timing the K-step region for about a second after the headline region")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-workload attention timings of the five synthetic configs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -403,36 +403,41 @@ __device__ __forceinline__ void code_cols(const uint32_t (&wk)[4], float s, floa
 // 16 values.
 __device__ __forceinline__ uint4 codes16(const uint32_t (&w)[8], float s, float r) {
     const uint64_t r2 = f2_pack(r, r), k2 = f2_pack(kRound, kRound), m2 = f2_pack(-1.0f, -1.0f);
-    uint32_t t[16];
+    uint32_t q[4];
     float worst = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
-        const uint64_t x2 = f2_pack(f.x, f.y);
-        const uint64_t t2 = ffma2(x2, r2, k2);
-        const uint64_t e2 = ffma2(x2, r2, ffma2(t2, m2, k2));
-        float a, b, ea, eb;
-        f2_unpack(t2, a, b);
-        f2_unpack(e2, ea, eb);
-        t[2 * i] = __float_as_uint(a);
-        t[2 * i + 1] = __float_as_uint(b);
-        worst = fmaxf(worst, fmaxf(fabsf(ea), fabsf(eb)));
-    }
-    if (worst > kNearTie) {   // a near-tie: the IEEE quotient for those elements
+    for (int i = 0; i < 4; ++i) {   // output word i: values 4i .. 4i + 3 (pairs w[2i], w[2i + 1])
+        uint32_t t[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
-            const float ta = fmaf(f.x, r, kRound), tb = fmaf(f.y, r, kRound);
-            if (fabsf(fmaf(f.x, r, kRound - ta)) > kNearTie) t[2 * i] = __float_as_uint(__fdiv_rn(f.x, s) + kRound);
-            if (fabsf(fmaf(f.y, r, kRound - tb)) > kNearTie) t[2 * i + 1] = __float_as_uint(__fdiv_rn(f.y, s) + kRound);
+        for (int h = 0; h < 2; ++h) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[2 * i + h]));
+            const uint64_t x2 = f2_pack(f.x, f.y);
+            const uint64_t t2 = ffma2(x2, r2, k2);
+            const uint64_t e2 = ffma2(x2, r2, ffma2(t2, m2, k2));
+            float a, b, ea, eb;
+            f2_unpack(t2, a, b);
+            f2_unpack(e2, ea, eb);
+            t[2 * h] = __float_as_uint(a);
+            t[2 * h + 1] = __float_as_uint(b);
+            worst = fmaxf(worst, fmaxf(fabsf(ea), fabsf(eb)));
+        }
+        q[i] = prmt(prmt(t[0], t[1], 0x0040u), prmt(t[2], t[3], 0x0040u), 0x5410u);
+    }
+    if (worst > kNearTie) {   // a near-tie: redo the 16 codes, the IEEE quotient where needed
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t t[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[2 * i + h]));
+                const float ta = fmaf(f.x, r, kRound), tb = fmaf(f.y, r, kRound);
+                t[2 * h] = __float_as_uint(fabsf(fmaf(f.x, r, kRound - ta)) > kNearTie ? __fdiv_rn(f.x, s) + kRound : ta);
+                t[2 * h + 1] = __float_as_uint(fabsf(fmaf(f.y, r, kRound - tb)) > kNearTie ? __fdiv_rn(f.y, s) + kRound : tb);
+            }
+            q[i] = prmt(prmt(t[0], t[1], 0x0040u), prmt(t[2], t[3], 0x0040u), 0x5410u);
         }
     }
-    uint4 q;
-    q.x = prmt(prmt(t[0], t[1], 0x0040u), prmt(t[2], t[3], 0x0040u), 0x5410u);
-    q.y = prmt(prmt(t[4], t[5], 0x0040u), prmt(t[6], t[7], 0x0040u), 0x5410u);
-    q.z = prmt(prmt(t[8], t[9], 0x0040u), prmt(t[10], t[11], 0x0040u), 0x5410u);
-    q.w = prmt(prmt(t[12], t[13], 0x0040u), prmt(t[14], t[15], 0x0040u), 0x5410u);
-    return q;
+    return make_uint4(q[0], q[1], q[2], q[3]);
 }
 
 // 16 fp16 values (32 bytes) at p: one 32-byte load when kV8 (p 32-byte
