@@ -148,3 +148,55 @@ def test_scale_of_every_fp16_magnitude():
     qo2, so2 = oracle.quantize_per_tensor(g.astype(np.float32), n)
     np.testing.assert_array_equal(s2.cpu().numpy().view(np.uint32), so2.view(np.uint32))
     np.testing.assert_array_equal(q2.cpu().numpy()[:, :, :1].transpose(0, 2, 1), qo2)
+
+
+def offset16(x: torch.Tensor) -> torch.Tensor:
+    """x's values in a CUDA tensor whose data starts 16 bytes past a 32-byte
+    boundary (the quantisers' two-load form; torch allocations are 256-byte
+    aligned and take the 32-byte-load form)."""
+    flat = torch.empty(x.numel() + 8, dtype=x.dtype, device="cuda")
+    y = flat[8:].view(x.shape)
+    y.copy_(x.cuda())
+    assert y.data_ptr() % 32 == 16
+    return y
+
+
+@pytest.mark.parametrize("d", [16, 64, 128, 256])
+def test_per_token_16_byte_aligned_input(d):
+    g = torch.Generator().manual_seed(d + 5)
+    x = (torch.randn(777, d, generator=g) * 4).half()
+    x[3] = 0.0
+    q, s = intfa.intfa_quantize_per_token(offset16(x))
+    qo, so = oracle.quantize_per_token(x.float().numpy())
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+
+
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("cols", [32, 64, 128])
+def test_per_tensor_16_byte_aligned_input(cols, transpose):
+    g = torch.Generator().manual_seed(cols + 11)
+    rows = 1100
+    x = (torch.randn(3, rows, cols, generator=g) * 2).half()
+    x[1, -1, 0] = 30.0
+    q, s = intfa.intfa_quantize_per_tensor(offset16(x), transpose=transpose)
+    qo, so = oracle.quantize_per_tensor(x.float().numpy(), 3)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    q = q.cpu().numpy()
+    if transpose:
+        q = q[:, :, :rows].transpose(0, 2, 1)
+    np.testing.assert_array_equal(q, qo)
+
+
+@pytest.mark.parametrize("groups,rows,cols", [(70, 300, 128), (600, 20, 64), (600, 100, 64)])
+def test_per_tensor_many_groups_per_cluster(groups, rows, cols):
+    """More groups than the per-head kernel's clusters: each cluster then
+    writes one group's codes while reading the next group's abs-max."""
+    g = torch.Generator().manual_seed(groups + rows)
+    x = (torch.randn(groups, rows, cols, generator=g) * torch.rand(groups, 1, 1, generator=g) * 5).half()
+    x[groups // 2] = 0.0
+    x[-1, -1, -1] = 60.0
+    q, s = intfa.intfa_quantize_per_tensor(x.cuda(), transpose=False)
+    qo, so = oracle.quantize_per_tensor(x.float().numpy(), groups)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.uint32), so.view(np.uint32))
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
