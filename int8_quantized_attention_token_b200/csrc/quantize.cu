@@ -4,8 +4,15 @@
 // and K (INT-FlashAttention, abstract: token-level quantisation) and per
 // L x d tensor for V.
 //
-// Both are HBM-bound streaming kernels: 16-byte vector loads of 8 fp16
-// values per thread, warp-shuffle row reductions, 8-byte code stores.
+// All are HBM-bound streaming kernels, one launch per tensor:
+// - per token: 16 values per lane (one 32-byte load when the input is
+//   32-byte aligned), warp-shuffle row maxima, 16-byte code stores;
+// - per tensor: a cluster of up to 8 CTAs per group reads the group once for
+//   the abs-max, combines the CTAs' maxima through distributed shared memory
+//   and reads the group again, from L2, for the codes -- in the input's
+//   layout, or transposed to [cols][ld] through registers.
+// Two-kernel forms (abs-max, then convert) remain for the widths and the
+// one-scale-for-all-groups option the cluster kernels do not take.
 //
 // Rounding contract (bit-exact with the definition): s = fl32(amax / 127)
 // by an IEEE division; the code is RNE(fl32(x / s)) clamped to +-127.  The
