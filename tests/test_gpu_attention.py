@@ -59,6 +59,13 @@ def test_small_shapes(B, H, L, d, causal):
     check_all(Q, K, V, causal)
 
 
+def test_config_128_d64_seed0():
+    """The smallest workload exactly as specified (seed 0), every element."""
+    w = WORKLOADS[0]
+    Q, K, V = make_workload(w)
+    check_all(Q, K, V, w.causal)
+
+
 def test_config_1024_d64_full():
     w = WORKLOADS[1]
     Q, K, V = make_workload(w)
