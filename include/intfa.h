@@ -379,8 +379,8 @@ int intfa_forward(const void *Q_f16, const void *K_f16, const void *V_f16, int B
  * copies O back to O_f16_host.  workspace:
  * intfa_forward_host_workspace_size(B, H, L, d) bytes of device memory,
  * 256-byte aligned.  Asynchronous on `stream`: O_f16_host is valid after the
- * stream is synchronised.  The heads are processed in chunks (at most 8, at
- * least 4 MiB of fp16 per tensor each): chunk c's input copies, its
+ * stream is synchronised.  The heads are processed in chunks (each half of
+ * the heads left, at least 4 MiB of fp16 per tensor): chunk c's input copies, its
  * quantisation + attention and its output copy overlap with the other chunks'
  * copies in the opposite direction.  The copies run on two streams of the
  * library's own (one pair per device, created on the first call and kept for

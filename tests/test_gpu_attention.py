@@ -139,8 +139,9 @@ def test_longest_supported_sequence(L, d, causal):
 
 @pytest.mark.parametrize("B,H,L,d,causal", [(2, 5, 4096, 128, True), (1, 6, 8192, 64, False)])
 def test_forward_host_chunks_match_device_path(B, H, L, d, causal):
-    """intfa_forward_host pipelines its copies over chunks of 4 heads here
-    (1 MiB of fp16 per head and tensor; the last chunk ragged).  Each chunk is
+    """intfa_forward_host pipelines its copies over chunks of half the heads
+    left, at least 4 (1 MiB of fp16 per head and tensor): 5, 4, 1 and 4, 2
+    heads here.  Each chunk is
     its own attention launch, so tiles meet other CTAs and other softmax
     warpgroups than in one launch over all heads; the two warpgroups' shares
     of the row sum then add in another order, which may move O by an fp16 ulp.
