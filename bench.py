@@ -183,6 +183,8 @@ def run_gpu(args):
     ws = torch.empty(max(1, intfa.lib().intfa_quantize_per_tensor_workspace_size(BH)), dtype=torch.uint8, device=dev)
     O = torch.empty(B, H, L, d, dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev)   # V's quantiser, as in intfa_forward
+    fork, join = torch.cuda.Event(), torch.cuda.Event()
     V3 = V.reshape(BH, L, d)
 
     fused_q = args.q_path == "fused"
@@ -235,13 +237,20 @@ def run_gpu(args):
         if blk > 1:
             return step_blocks(ev)
         # a1 (K; and Q unless fused), a2 (V), then a3-a9 in the attention kernel
-        if not fused_q:
-            intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
-        intfa.intfa_quantize_per_token(K, Kq, sK, stream=stream)
         plain = not fused_q and args.p_levels == 127 and args.lsum != "codes"
-        if plain:   # the path of intfa_forward: V_hat untransposed
-            intfa.intfa_quantize_per_tensor(V3, False, Vr.reshape(BH, L, d), sV, ws, stream=stream)
+        if plain:   # the path of intfa_forward: V_hat untransposed, its quantiser
+            # on a side stream beside Q's and K's, joined before the attention
+            fork.record(stream)
+            side.wait_event(fork)
+            intfa.intfa_quantize_per_tensor(V3, False, Vr.reshape(BH, L, d), sV, ws, stream=side)
+            intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
+            intfa.intfa_quantize_per_token(K, Kq, sK, stream=stream)
+            join.record(side)
+            stream.wait_event(join)
         else:
+            if not fused_q:
+                intfa.intfa_quantize_per_token(Q, Qq, sQ, stream=stream)
+            intfa.intfa_quantize_per_token(K, Kq, sK, stream=stream)
             intfa.intfa_quantize_per_tensor(V3, True, Vt, sV, ws, stream=stream)
         if ev is not None:
             ev[0].record(stream)

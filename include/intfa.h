@@ -359,7 +359,12 @@ int intfa_debug_wait_timeout(const int8_t *Q_q, const int8_t *K_q, const int8_t 
 /*
  * Whole hot path on device buffers: quantise Q and K per token, V per head
  * (codes kept in V's [B][H][L][d] layout), then the fused attention
- * (intfa_attention_fwd_vrows).  Q, K, V, O: fp16 [B][H][L][d]
+ * (intfa_attention_fwd_vrows).  V's quantiser runs on a stream of the
+ * library's own (one per device, made with two events on the first call, like
+ * intfa_forward_host's copy streams) beside Q's and K's on `stream`, which
+ * waits for it before the attention; make the first call on a device before
+ * any stream capture.  Calls are serialised by a host mutex while they queue
+ * their work.  Q, K, V, O: fp16 [B][H][L][d]
  * device pointers; workspace: intfa_forward_workspace_size(B, H, L, d) bytes of
  * device memory, 256-byte aligned.  Optional outputs of the quantisation live
  * in the workspace at the offsets intfa_forward_workspace_layout reports.

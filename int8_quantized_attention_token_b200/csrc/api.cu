@@ -77,6 +77,54 @@ extern "C" int intfa_forward_workspace_layout(int B, int H, int L, int d, size_t
     return INTFA_OK;
 }
 
+namespace {
+
+// Streams and events of one device: the pipelined host path's copy streams,
+// and intfa_forward's side stream.  Made on the first call on that device and
+// kept for the life of the process (no allocation of device memory; nothing
+// is created on later calls).
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, in = nullptr, out = nullptr, done = nullptr;
+    cudaStream_t side = nullptr;                   // intfa_forward: V's quantiser beside Q's and K's
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_pipe_mu;             // guards g_pipes and keeps each call's enqueue sequence whole
+HostPipe g_pipes[kMaxDevices];
+
+int get_pipe(HostPipe **out) {
+    int dev = 0;
+    int rc = intfa::cuda_status(cudaGetDevice(&dev));
+    if (rc) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return INTFA_ERR_UNSUPPORTED;
+    HostPipe &p = g_pipes[dev];
+    if (!p.done) {
+        HostPipe n;
+        rc = intfa::cuda_status(cudaStreamCreateWithFlags(&n.h2d, cudaStreamNonBlocking));
+        if (!rc) rc = intfa::cuda_status(cudaStreamCreateWithFlags(&n.d2h, cudaStreamNonBlocking));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.start, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.in, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.out, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.done, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaStreamCreateWithFlags(&n.side, cudaStreamNonBlocking));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming));
+        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming));
+        if (rc) {
+            for (cudaStream_t t : {n.h2d, n.d2h, n.side})
+                if (t) cudaStreamDestroy(t);
+            for (cudaEvent_t e : {n.start, n.in, n.out, n.done, n.fork, n.join})
+                if (e) cudaEventDestroy(e);
+            return rc;
+        }
+        p = n;
+    }
+    *out = &p;
+    return INTFA_OK;
+}
+
+}  // namespace
+
 extern "C" int intfa_forward(const void *Q_f16, const void *K_f16, const void *V_f16, int B, int H,
                              int L, int d, int causal, void *O_f16, void *workspace,
                              size_t workspace_bytes, void *stream) {
@@ -105,53 +153,27 @@ extern "C" int intfa_forward(const void *Q_f16, const void *K_f16, const void *V
     // (intfa_attention_fwd_q16) saves the pass but costs more issue slots on
     // the attention kernel's sub-partitions than the pass takes.
     int8_t *q = reinterpret_cast<int8_t *>(w + lo.q);
-    int rc = launch_quantize_per_token(Q_f16, rows, d, q, sq, s);
+    std::lock_guard<std::mutex> lock(g_pipe_mu);   // keeps this call's fork / join whole
+    HostPipe *pp = nullptr;
+    int rc = get_pipe(&pp);
+    if (rc) return rc;
+    // V's quantiser (V_hat stays in V's layout: the attention reads its tiles
+    // N-major) runs on the library's side stream while Q's and K's run on the
+    // caller's; the three are HBM-bound and fill each other's gaps (measured
+    // on B4 H32 L4096 d128: 131 -> 115 us for the three).  The caller's stream
+    // waits for the side stream before the attention, whatever happened.
+    rc = cuda_status(cudaEventRecord(pp->fork, s));
+    if (!rc) rc = cuda_status(cudaStreamWaitEvent(pp->side, pp->fork, 0));
+    if (!rc) rc = launch_quantize_per_tensor(V_f16, bh, L, d, 0, v, sv, w + lo.ws, pp->side);
+    if (!rc) rc = launch_quantize_per_token(Q_f16, rows, d, q, sq, s);
     if (!rc) rc = launch_quantize_per_token(K_f16, rows, d, k, sk, s);
-    // V_hat stays in V's layout: the attention reads its tiles N-major
-    if (!rc) rc = launch_quantize_per_tensor(V_f16, bh, L, d, 0, v, sv, w + lo.ws, s);
-    if (!rc) rc = launch_attention_fwd_vrows(q, k, v, sq, sk, sv, B, H, L, d, causal, O_f16, s);
-    return rc;
+    int rc2 = cuda_status(cudaEventRecord(pp->join, pp->side));
+    if (!rc2) rc2 = cuda_status(cudaStreamWaitEvent(s, pp->join, 0));
+    if (!rc && !rc2) rc = launch_attention_fwd_vrows(q, k, v, sq, sk, sv, B, H, L, d, causal, O_f16, s);
+    return rc ? rc : rc2;
 }
 
 namespace {
-
-// Copy streams and events of one device for the pipelined host path: made on
-// the first call on that device and kept for the life of the process (no
-// allocation of device memory; nothing is created on later calls).
-struct HostPipe {
-    cudaStream_t h2d = nullptr, d2h = nullptr;
-    cudaEvent_t start = nullptr, in = nullptr, out = nullptr, done = nullptr;
-};
-constexpr int kMaxDevices = 64;
-std::mutex g_pipe_mu;             // guards g_pipes and keeps each call's enqueue sequence whole
-HostPipe g_pipes[kMaxDevices];
-
-int get_pipe(HostPipe **out) {
-    int dev = 0;
-    int rc = intfa::cuda_status(cudaGetDevice(&dev));
-    if (rc) return rc;
-    if (dev < 0 || dev >= kMaxDevices) return INTFA_ERR_UNSUPPORTED;
-    HostPipe &p = g_pipes[dev];
-    if (!p.done) {
-        HostPipe n;
-        rc = intfa::cuda_status(cudaStreamCreateWithFlags(&n.h2d, cudaStreamNonBlocking));
-        if (!rc) rc = intfa::cuda_status(cudaStreamCreateWithFlags(&n.d2h, cudaStreamNonBlocking));
-        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.start, cudaEventDisableTiming));
-        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.in, cudaEventDisableTiming));
-        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.out, cudaEventDisableTiming));
-        if (!rc) rc = intfa::cuda_status(cudaEventCreateWithFlags(&n.done, cudaEventDisableTiming));
-        if (rc) {
-            if (n.h2d) cudaStreamDestroy(n.h2d);
-            if (n.d2h) cudaStreamDestroy(n.d2h);
-            for (cudaEvent_t e : {n.start, n.in, n.out, n.done})
-                if (e) cudaEventDestroy(e);
-            return rc;
-        }
-        p = n;
-    }
-    *out = &p;
-    return INTFA_OK;
-}
 
 // Heads in the next chunk of the host pipeline, rem heads left: half of them
 // (large chunks first keep the launches efficient, small ones last keep the
