@@ -2,7 +2,8 @@
 
 One step = the whole path on one batch of synthetic fp16 input already in HBM:
 per-token quantisation of Q and K, per-head quantisation of V (codes in V's
-own layout), and the fused INT8 attention kernel (V_hat tiles read N-major).  The metric is INT8 attention TOPS:
+own layout, on a side stream beside Q's and K's, as intfa_forward does), and
+the fused INT8 attention kernel (V_hat tiles read N-major).  The metric is INT8 attention TOPS:
 4 B H L^2 d ops (halved when causal) per step / step time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
