@@ -615,12 +615,6 @@ def run_decode(args):
                "sample": f"{n} of {BH} heads (quantise the query and the head's cache, decode), {t:.1f} s, "
                          "single-threaded (the decode oracle has no thread loop)"}
 
-    configs = None
-    if rank == 0 and not args.no_configs and args.method == "online" and not fused_q and blk == 1 \
-            and args.lsum == "p" and args.p_levels == 127:
-        configs = measure_configs(intfa, dev, stream, peak, local)
-
-    sha_method = "online-fused-q" if fused_q else args.method
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(ops * world / (ms * 1e-3) / 1e12, 3), "unit": UNIT, "n_gpus": world,
