@@ -322,10 +322,36 @@ int cluster_ctas(int64_t groups, int64_t units) {
     want = want < kCL ? kCL : (want > kCLMax ? kCLMax : want);
     return static_cast<int>(units < want ? units : want);
 }
-// Allows cluster sizes up to kCLMax for a kernel.
-template <typename K>
-int allow_big_clusters(K kernel) {
-    return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+// Launches `kernel` (kPThreads threads per CTA) as `groups` clusters of `cl`
+// CTAs on `stream`.  A size above kCL is non-portable: the kernel is allowed
+// it first (on the current device, at every such launch), and a device that
+// cannot schedule it gets the portable size kCL instead -- the kernels read
+// their cluster size at run time.
+template <typename... KArgs, typename... Args>
+int launch_clusters(void (*kernel)(KArgs...), int64_t groups, int cl, cudaStream_t stream, Args... args) {
+    for (;;) {
+        if (cl > kCL) {
+            const int rc = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+            if (rc) return rc;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(groups * cl), 1, 1);
+        cfg.blockDim = dim3(kPThreads, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+        if (e == cudaSuccess) return INTFA_OK;
+        if (cl <= kCL) return cuda_status(e);
+        (void)cudaGetLastError();   // not sticky: retry with the portable size
+        cl = kCL;
+    }
 }
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -612,27 +638,10 @@ int launch_quant_fused(const uint4 *x, int64_t groups, int64_t n16, int8_t *xq, 
                        cudaStream_t stream) {
     const int64_t nblk = (n16 + kPThreads - 1) / kPThreads;
     const int cl = cluster_ctas(groups, nblk);
-    if (cl > kCL) {   // a non-portable cluster size (set on the current device at every such launch)
-        const int rc = allow_big_clusters(group_quant_fused_kernel<true>) |
-                       allow_big_clusters(group_quant_fused_kernel<false>);
-        if (rc) return rc;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(groups * cl), 1, 1);
-    cfg.blockDim = dim3(kPThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     uint4 *q = reinterpret_cast<uint4 *>(xq);
     if ((reinterpret_cast<uintptr_t>(x) & 31u) == 0)
-        return cuda_status(cudaLaunchKernelEx(&cfg, group_quant_fused_kernel<true>, x, n16, q, scale));
-    return cuda_status(cudaLaunchKernelEx(&cfg, group_quant_fused_kernel<false>, x, n16, q, scale));
+        return launch_clusters(group_quant_fused_kernel<true>, groups, cl, stream, x, n16, q, scale);
+    return launch_clusters(group_quant_fused_kernel<false>, groups, cl, stream, x, n16, q, scale);
 }
 
 template <int C8, bool kV8>     // kV8: the input is 32-byte aligned (one load per row)
@@ -746,26 +755,9 @@ int launch_quant_t_fused(const uint4 *x, int64_t groups, int64_t rows, int64_t l
                          cudaStream_t stream) {
     const int64_t ntile = (ld + kPRows - 1) / kPRows;
     const int cl = cluster_ctas(groups, ntile);
-    if (cl > kCL) {   // a non-portable cluster size (set on the current device at every such launch)
-        const int rc = allow_big_clusters(group_quant_t_fused_kernel<C8, true>) |
-                       allow_big_clusters(group_quant_t_fused_kernel<C8, false>);
-        if (rc) return rc;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(groups * cl), 1, 1);
-    cfg.blockDim = dim3(kPThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     if ((reinterpret_cast<uintptr_t>(x) & 31u) == 0)
-        return cuda_status(cudaLaunchKernelEx(&cfg, group_quant_t_fused_kernel<C8, true>, x, rows, ld, xq, scale));
-    return cuda_status(cudaLaunchKernelEx(&cfg, group_quant_t_fused_kernel<C8, false>, x, rows, ld, xq, scale));
+        return launch_clusters(group_quant_t_fused_kernel<C8, true>, groups, cl, stream, x, rows, ld, xq, scale);
+    return launch_clusters(group_quant_t_fused_kernel<C8, false>, groups, cl, stream, x, rows, ld, xq, scale);
 }
 
 int grid_for(int64_t work_items, int per_block) {
