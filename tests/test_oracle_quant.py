@@ -191,3 +191,22 @@ def test_bits_round_trip_and_range(bits):
     assert np.all(np.abs(q).max(axis=1) == qmax)            # the arg-max row entry hits +-qmax
     err = np.abs(x - s[:, None].astype(np.float64) * q)
     assert np.all(err <= s[:, None] / 2 * (1 + 1e-6) + 1e-12)
+
+
+@pytest.mark.parametrize("amax", [127.0, 100.0, 1.0, 0.0999755859375, 3.0517578125e-05])
+def test_near_ties_against_exact_rational(amax):
+    """Every fp16 x whose fp32 quotient x / s lies within 2e-3 of a
+    half-integer (the elements the GPU kernels send to the IEEE division,
+    and the exact ties), both signs, in one row with the row's maximum: the
+    oracle's codes equal RNE(fl32(x / s)) computed in exact arithmetic."""
+    h = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float32)
+    h = h[h <= np.float32(amax)]
+    s32 = np.float32(np.float32(amax) / np.float32(127.0))
+    q = h / s32
+    near = h[np.abs(q - np.floor(q) - np.float32(0.5)) < np.float32(2e-3)]
+    assert near.size > 0
+    row = np.concatenate([[np.float32(amax)], near, -near]).astype(np.float32)
+    codes, s = expected_codes(row)
+    qo, so = oracle.quantize_per_token(row[None, :])
+    assert so[0] == np.float32(s)
+    np.testing.assert_array_equal(qo[0], np.array(codes, np.int8))
