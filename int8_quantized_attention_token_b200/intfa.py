@@ -447,6 +447,9 @@ def intfa_forward_host_workspace_size(B, H, L, d) -> int:
 
 
 def intfa_forward_workspace_layout(B, H, L, d) -> list[int]:
+    """Byte offsets inside intfa_forward's workspace of Q_q, K_q, V_q (int8
+    [B, H, L, d] each; V's codes untransposed), s_Q, s_K (fp32 [B, H, L]) and
+    s_V (fp32 [B, H])."""
     off = (ctypes.c_size_t * 6)()
     _check(lib().intfa_forward_workspace_layout(B, H, L, d, off), "intfa_forward_workspace_layout")
     return list(off)
