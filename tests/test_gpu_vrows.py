@@ -55,3 +55,31 @@ def test_vrows_bit_identical_full_size(w):
     Q, K, V = make_workload(w)
     Ot, Or = both_layouts(Q, K, V, w.causal)
     assert torch.equal(Ot.view(torch.int16), Or.view(torch.int16))
+
+
+def test_forward_workspace_holds_the_codes():
+    """After intfa_forward, its workspace holds the quantisers' outputs at the
+    offsets intfa_forward_workspace_layout reports: Q_q, K_q, V_q (V's codes
+    untransposed) and the three scale arrays, equal to the standalone calls."""
+    B, H, L, d = 2, 3, 333, 128
+    Q, K, V = [t.cuda() for t in make_qkv(B, H, L, d, seed=5)]
+    ws = torch.empty(intfa.intfa_forward_workspace_size(B, H, L, d), dtype=torch.uint8, device="cuda")
+    intfa.intfa_forward(Q, K, V, True, workspace=ws)
+    torch.cuda.synchronize()
+    assert intfa.intfa_device_status(clear=True) == 0
+    off = intfa.intfa_forward_workspace_layout(B, H, L, d)
+    n = B * H * L * d
+
+    def view(i, count, dtype):
+        nbytes = count * torch.tensor([], dtype=dtype).element_size()
+        return ws[off[i]:off[i] + nbytes].view(dtype)
+
+    Qq, sQ = intfa.intfa_quantize_per_token(Q)
+    Kq, sK = intfa.intfa_quantize_per_token(K)
+    Vq, sV = intfa.intfa_quantize_per_tensor(V.reshape(B * H, L, d), transpose=False)
+    assert torch.equal(view(0, n, torch.int8), Qq.reshape(-1))
+    assert torch.equal(view(1, n, torch.int8), Kq.reshape(-1))
+    assert torch.equal(view(2, n, torch.int8), Vq.reshape(-1))
+    assert torch.equal(view(3, B * H * L, torch.float32).view(torch.int32), sQ.reshape(-1).view(torch.int32))
+    assert torch.equal(view(4, B * H * L, torch.float32).view(torch.int32), sK.reshape(-1).view(torch.int32))
+    assert torch.equal(view(5, B * H, torch.float32).view(torch.int32), sV.reshape(-1).view(torch.int32))
