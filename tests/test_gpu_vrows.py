@@ -83,3 +83,26 @@ def test_forward_workspace_holds_the_codes():
     assert torch.equal(view(3, B * H * L, torch.float32).view(torch.int32), sQ.reshape(-1).view(torch.int32))
     assert torch.equal(view(4, B * H * L, torch.float32).view(torch.int32), sK.reshape(-1).view(torch.int32))
     assert torch.equal(view(5, B * H, torch.float32).view(torch.int32), sV.reshape(-1).view(torch.int32))
+
+
+def test_forward_captured_in_a_cuda_graph():
+    """intfa_forward (with V's quantiser forked onto the library's side stream)
+    captured into a CUDA graph and replayed gives the eager call's bytes."""
+    B, H, L, d = 1, 4, 640, 128
+    Q, K, V = [t.cuda() for t in make_qkv(B, H, L, d, seed=9)]
+    ws = torch.empty(intfa.intfa_forward_workspace_size(B, H, L, d), dtype=torch.uint8, device="cuda")
+    O_eager = intfa.intfa_forward(Q, K, V, True, workspace=ws)   # first call: makes the side stream
+    torch.cuda.synchronize()
+    O = torch.empty_like(O_eager)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+            intfa.intfa_forward(Q, K, V, True, O=O, workspace=ws, stream=s)
+    for _ in range(3):
+        O.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    assert intfa.intfa_device_status(clear=True) == 0
+    assert torch.equal(O.view(torch.int16), O_eager.view(torch.int16))
